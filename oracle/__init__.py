@@ -1,0 +1,179 @@
+"""fp64 CPU oracle of the selective SSM scan and decode step.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The library code under
+``selective_state_space_36_b200`` never imports this package, and this package
+imports nothing from it.
+
+The arithmetic lives in ``ssm_oracle.c`` (plain C, double precision, one
+sequential loop per channel); this module compiles it with gcc on first use
+and marshals numpy arrays.  Every function takes and returns float64 arrays;
+inputs held as bf16 bits or float32 must be widened exactly first (see
+``selective_state_space_36_b200.inputs.to_f64``).
+
+Parity status of each function (what pins it lives in tests/test_oracle_pins.py):
+  scan(..., zoh_b=False)  pinned: brute-force unrolled sum, N=1 closed form,
+                          LTI convolution, Delta -> 0, split/resume, softplus
+                          and bias placement, skip and gate special cases.
+  scan(..., zoh_b=True)   pinned: brute force (ZOH form), Theorem 1.
+  state_update            pinned: 1000 decode steps == scan over 1000 steps,
+                          one-step brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB = os.path.join(_HERE, "libssm_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile ssm_oracle.c into libssm_oracle.so (gcc, -O2, IEEE semantics)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    lib.oracle_selective_scan.restype = ctypes.c_int
+    lib.oracle_selective_scan.argtypes = [_i64, _i64, _i64, _i64,
+                                          _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                          ctypes.c_int, ctypes.c_int, _dp, _dp, ctypes.c_int]
+    lib.oracle_state_update.restype = ctypes.c_int
+    lib.oracle_state_update.argtypes = [_i64, _i64, _i64, _dp, _dp, _dp, _dp,
+                                        _dp, _dp, _dp, _dp, _dp]
+    lib.oracle_default_threads.restype = ctypes.c_int
+    lib.oracle_default_threads.argtypes = []
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = _bind(_LIB)
+    return _lib
+
+
+def default_threads() -> int:
+    """Threads the oracle uses when ``nthreads`` is 0."""
+    return int(_load().oracle_default_threads())
+
+
+def _c64(a: Optional[np.ndarray], shape: Tuple[int, ...], name: str):
+    if a is None:
+        return None, None
+    arr = np.ascontiguousarray(a, dtype=np.float64)
+    if arr.shape != shape:
+        raise ValueError(f"{name}: expected shape {shape}, got {arr.shape}")
+    return arr, arr.ctypes.data_as(_dp)
+
+
+def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+         h0=None, zoh_b: bool = False, nthreads: int = 0, _lib_handle=None):
+    """Selective scan in fp64.
+
+    u, delta, z: (batch, seqlen, dim); B, C: (batch, seqlen, dstate);
+    A: (dim, dstate); D, delta_bias: (dim,); h0: (batch, dim, dstate) or None.
+    Returns (out (batch, seqlen, dim), last_state (batch, dim, dstate)).
+    """
+    u = np.asarray(u)
+    batch, seqlen, dim = u.shape
+    dstate = np.asarray(A).shape[1]
+    keep = []
+
+    def p(a, shape, name):
+        arr, ptr = _c64(a, shape, name)
+        keep.append(arr)
+        return ptr
+
+    pu = p(u, (batch, seqlen, dim), "u")
+    pd = p(delta, (batch, seqlen, dim), "delta")
+    pA = p(A, (dim, dstate), "A")
+    pB = p(B, (batch, seqlen, dstate), "B")
+    pC = p(C, (batch, seqlen, dstate), "C")
+    pD = p(D, (dim,), "D")
+    pz = p(z, (batch, seqlen, dim), "z")
+    pb = p(delta_bias, (dim,), "delta_bias")
+    out = np.zeros((batch, seqlen, dim), dtype=np.float64)
+    state = (np.zeros((batch, dim, dstate), dtype=np.float64) if h0 is None
+             else np.array(h0, dtype=np.float64, order="C", copy=True).reshape(batch, dim, dstate))
+    rc = (_lib_handle or _load()).oracle_selective_scan(batch, seqlen, dim, dstate, pu, pd, pA, pB, pC, pD, pz, pb,
+                                       int(bool(delta_softplus)), int(bool(zoh_b)),
+                                       out.ctypes.data_as(_dp), state.ctypes.data_as(_dp),
+                                       int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_selective_scan failed with code {rc}")
+    return out, state
+
+
+def state_update(state, x, dt, A, B, C, D=None, z=None, _lib_handle=None):
+    """One decode step in fp64.  Returns (out (batch, dim), new_state)."""
+    st = np.array(state, dtype=np.float64, order="C", copy=True)
+    batch, dim, dstate = st.shape
+    keep = []
+
+    def p(a, shape, name):
+        arr, ptr = _c64(a, shape, name)
+        keep.append(arr)
+        return ptr
+
+    px = p(x, (batch, dim), "x")
+    pdt = p(dt, (batch, dim), "dt")
+    pA = p(A, (dim, dstate), "A")
+    pB = p(B, (batch, dstate), "B")
+    pC = p(C, (batch, dstate), "C")
+    pD = p(D, (dim,), "D")
+    pz = p(z, (batch, dim), "z")
+    out = np.zeros((batch, dim), dtype=np.float64)
+    rc = (_lib_handle or _load()).oracle_state_update(batch, dim, dstate, st.ctypes.data_as(_dp), px, pdt, pA,
+                                     pB, pC, pD, pz, out.ctypes.data_as(_dp))
+    if rc != 0:
+        raise RuntimeError(f"oracle_state_update failed with code {rc}")
+    return out, st
+
+
+class Variant:
+    """The same API bound to another build of the oracle source (used by the
+    mutation tests, which compile deliberately broken copies)."""
+
+    def __init__(self, path: str):
+        self._h = _bind(path)
+
+    def scan(self, *a, **kw):
+        return scan(*a, _lib_handle=self._h, **kw)
+
+    def state_update(self, *a, **kw):
+        return state_update(*a, _lib_handle=self._h, **kw)
+
+
+def compile_variant(source: str, path: str) -> "Variant":
+    """Compile C source text (a modified copy of ssm_oracle.c) to ``path``."""
+    src = path + ".c"
+    with open(src, "w") as f:
+        f.write(source)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                           "-o", path, src, "-lm", "-lpthread"])
+    return Variant(path)
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()

@@ -1,0 +1,214 @@
+/*
+ * ssm_oracle.c -- plain, slow, fp64 CPU oracle of the selective SSM (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library, and the CUDA library never
+ * calls it.
+ *
+ * What it computes, and where each step comes from:
+ *
+ *  - Discretisation (NL-345, Mamba: Linear-Time Sequence Modeling with
+ *    Selective State Spaces, section 2 "Discretization"; 【論文要約】Mamba
+ *    notes, 数式解説 3 "ZOH"): Abar = exp(Delta * A), elementwise because A is
+ *    diagonal (NL-345 section 2 "Structure and Dimensions").  Bbar is either
+ *    the Euler form Delta * B (the library's convention) or the exact
+ *    zero-order hold (Delta A)^-1 (exp(Delta A) - 1) Delta B = expm1(Delta A)/A * B
+ *    (the notes' ZOH formula); with A == 0 the ZOH limit is Delta * B.
+ *  - Recurrence and readout (NL-345 section 2, eq. (2)):
+ *        h_t = Abar_t h_{t-1} + Bbar_t x_t,   y_t = C_t h_t,
+ *    so y_t reads the state *after* x_t has entered it.
+ *  - Selection (【論文要約】Mamba notes, "S6", Algorithm 2): B_t and C_t are
+ *    per-token inputs shared by all channels; Delta_t = tau_Delta(bias +
+ *    Delta_raw_t) with tau_Delta = softplus (the notes' Theorem 1), or the plain
+ *    sum when softplus is off.  A is a static (dim x dstate) parameter.
+ *  - Skip and gate (the library's fused block epilogue, not on the pages):
+ *        out = (y + D u) * silu(z),  silu(z) = z / (1 + exp(-z));
+ *    a NULL D means D = 0 and a NULL z means no gate.
+ *  - Each channel (b, d) is an independent SSM (NL-345 section 2 "Structure
+ *    and Dimensions"), so channels are distributed over threads; inside a
+ *    channel the loop runs in time order and, for each step, in state order,
+ *    exactly as written above.  Thread count never changes a result.
+ *
+ * Layouts (dense, row-major): u, delta, z, out (batch, seqlen, dim);
+ * B, C (batch, seqlen, dstate); A (dim, dstate); D, delta_bias (dim);
+ * state (batch, dim, dstate).  All values are double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <unistd.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEM 2
+
+/* softplus(s) = log(1 + e^s), evaluated as max(s, 0) + log1p(e^-|s|):
+ * the same function, without overflow for large s and without the loss of
+ * relative precision that log(1 + tiny) would have for very negative s. */
+static double oracle_softplus(double s)
+{
+    double m = s > 0.0 ? s : 0.0;
+    return m + log1p(exp(-fabs(s)));
+}
+
+static double oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+typedef struct {
+    int64_t batch, seqlen, dim, dstate;
+    const double *u, *delta, *A, *B, *C, *Dskip, *z, *bias;
+    int softplus, zoh_b;
+    double *out, *state;
+    int64_t c_begin, c_end; /* channel range, channel = b * dim + d */
+    int status;
+} scan_job;
+
+static void scan_channels(scan_job *j)
+{
+    const int64_t L = j->seqlen, Dm = j->dim, N = j->dstate;
+    double *h = (double *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+    if (!h) { j->status = ORACLE_NO_MEM; return; }
+    for (int64_t c = j->c_begin; c < j->c_end; ++c) {
+        const int64_t b = c / Dm, d = c % Dm;
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = j->state ? j->state[(b * Dm + d) * N + n] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t td = (b * L + t) * Dm + d;  /* (b, t, d) */
+            const int64_t tn = (b * L + t) * N;       /* (b, t, 0) */
+            const double x = j->u[td];
+            double s = j->delta[td] + (j->bias ? j->bias[d] : 0.0);
+            const double dlt = j->softplus ? oracle_softplus(s) : s;
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double an = j->A[d * N + n];
+                const double abar = exp(dlt * an);
+                double bbar;
+                if (j->zoh_b)
+                    bbar = (an == 0.0 ? dlt : expm1(dlt * an) / an) * j->B[tn + n];
+                else
+                    bbar = dlt * j->B[tn + n];
+                h[n] = abar * h[n] + bbar * x;
+                acc += j->C[tn + n] * h[n];
+            }
+            double y = acc + (j->Dskip ? j->Dskip[d] * x : 0.0);
+            if (j->z) y *= oracle_silu(j->z[td]);
+            j->out[td] = y;
+        }
+        if (j->state)
+            for (int64_t n = 0; n < N; ++n)
+                j->state[(b * Dm + d) * N + n] = h[n];
+    }
+    free(h);
+    j->status = ORACLE_OK;
+}
+
+static void *scan_thread(void *p)
+{
+    scan_channels((scan_job *)p);
+    return NULL;
+}
+
+static int resolve_threads(int nthreads, int64_t channels)
+{
+    if (nthreads <= 0) {
+        long n = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = n > 0 ? (int)n : 1;
+    }
+    if (nthreads > 1024) nthreads = 1024;
+    if ((int64_t)nthreads > channels) nthreads = (int)(channels > 0 ? channels : 1);
+    return nthreads;
+}
+
+/* Number of threads a call with nthreads <= 0 would use on this host. */
+int oracle_default_threads(void)
+{
+    return resolve_threads(0, INT64_MAX);
+}
+
+/*
+ * Selective scan over all (batch, dim) channels.
+ *   zoh_b = 0: Bbar = Delta * B (Euler);  zoh_b = 1: exact ZOH Bbar.
+ *   state: NULL => h0 = 0 and the final state is not returned; otherwise it
+ *          holds h0 on entry and h_L on return.
+ *   nthreads <= 0 uses every online core.
+ * Returns 0 on success.
+ */
+int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                          const double *u, const double *delta, const double *A,
+                          const double *B, const double *C, const double *Dskip,
+                          const double *z, const double *delta_bias, int delta_softplus,
+                          int zoh_b, double *out, double *state, int nthreads)
+{
+    if (batch < 0 || seqlen < 0 || dim < 0 || dstate < 0) return ORACLE_BAD_ARG;
+    const int64_t channels = batch * dim;
+    if (channels == 0) return ORACLE_OK;
+    if (seqlen > 0 && (!u || !delta || !B || !C || !out)) return ORACLE_BAD_ARG;
+    if (dstate > 0 && !A) return ORACLE_BAD_ARG;
+    int nt = resolve_threads(nthreads, channels);
+    scan_job *jobs = (scan_job *)calloc((size_t)nt, sizeof(scan_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nt, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEM; }
+    for (int i = 0; i < nt; ++i) {
+        scan_job *j = &jobs[i];
+        j->batch = batch; j->seqlen = seqlen; j->dim = dim; j->dstate = dstate;
+        j->u = u; j->delta = delta; j->A = A; j->B = B; j->C = C;
+        j->Dskip = Dskip; j->z = z; j->bias = delta_bias;
+        j->softplus = delta_softplus; j->zoh_b = zoh_b;
+        j->out = out; j->state = state;
+        j->c_begin = channels * i / nt;
+        j->c_end = channels * (i + 1) / nt;
+        j->status = ORACLE_BAD_ARG;
+    }
+    int started = 0;
+    for (int i = 1; i < nt; ++i) {
+        if (pthread_create(&th[i], NULL, scan_thread, &jobs[i]) != 0) break;
+        started = i;
+    }
+    scan_channels(&jobs[0]);
+    for (int i = 1; i <= started; ++i) pthread_join(th[i], NULL);
+    for (int i = started + 1; i < nt; ++i) scan_channels(&jobs[i]); /* threads that failed to start */
+    int rc = ORACLE_OK;
+    for (int i = 0; i < nt; ++i)
+        if (jobs[i].status != ORACLE_OK) rc = jobs[i].status;
+    free(jobs);
+    free(th);
+    return rc;
+}
+
+/*
+ * One recurrent (decode) step for every channel (NL-345 section 1: constant
+ * time per generated step; section 2 eq. (2) for one t).  dt is the time step
+ * itself (already positive: no bias, no softplus).  state (batch, dim, dstate)
+ * is updated in place; x, dt, z, out are (batch, dim); B, C are (batch, dstate).
+ */
+int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, double *state,
+                        const double *x, const double *dt, const double *A,
+                        const double *B, const double *C, const double *Dskip,
+                        const double *z, double *out)
+{
+    if (batch < 0 || dim < 0 || dstate < 0) return ORACLE_BAD_ARG;
+    if (batch * dim == 0) return ORACLE_OK;
+    if (!state || !x || !dt || !B || !C || !out || (dstate > 0 && !A)) return ORACLE_BAD_ARG;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const double dlt = dt[b * dim + d];
+            const double xv = x[b * dim + d];
+            double *h = state + (b * dim + d) * dstate;
+            double acc = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                const double abar = exp(dlt * A[d * dstate + n]);
+                h[n] = abar * h[n] + dlt * B[b * dstate + n] * xv;
+                acc += C[b * dstate + n] * h[n];
+            }
+            double y = acc + (Dskip ? Dskip[d] * xv : 0.0);
+            if (z) y *= oracle_silu(z[b * dim + d]);
+            out[b * dim + d] = y;
+        }
+    }
+    return ORACLE_OK;
+}

@@ -1,0 +1,343 @@
+"""Pins of the fp64 oracle to facts fixed by the pages and by mathematics.
+
+None of these re-types the oracle's loop: each compares it with an independent
+route to the same number (an unrolled closed sum, a closed form, a library
+convolution, a library softplus/sigmoid, an exact invariant), so a dropped
+term, a wrong sign, a wrong index or a transposed operand in the oracle fails
+at least one of them.  No GPU is involved.
+
+Sources: NL-345, Mamba: Linear-Time Sequence Modeling with Selective State
+Spaces (section 2: eq. (2) recurrence, eq. (3) convolution, "Linear Time
+Invariance", "Structure and Dimensions"; section 1: recurrent inference);
+【論文要約】Mamba notes (数式解説 3 ZOH; 4 Theorem 1; S6 Algorithm 2).
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _rand_case(rng, batch=2, L=11, dim=3, N=4, softplus=True, bias=True, gate=True,
+               dskip=True, h0=True):
+    u = rng.standard_normal((batch, L, dim))
+    delta = rng.standard_normal((batch, L, dim)) * 0.7
+    A = -rng.uniform(0.2, 2.5, size=(dim, N))
+    B = rng.standard_normal((batch, L, N))
+    C = rng.standard_normal((batch, L, N))
+    D = rng.standard_normal(dim) if dskip else None
+    z = rng.standard_normal((batch, L, dim)) if gate else None
+    bvec = rng.standard_normal(dim) * 0.5 if bias else None
+    hh = rng.standard_normal((batch, dim, N)) if h0 else None
+    return dict(u=u, delta=delta, A=A, B=B, C=C, D=D, z=z, delta_bias=bvec,
+                delta_softplus=softplus, h0=hh)
+
+
+def _brute(case, zoh_b=False):
+    """Fully unrolled y_t = sum_{s<=t} C_t (prod_{r=s+1..t} Abar_r) Bbar_s x_s
+    + C_t (prod_{r<=t} Abar_r) h0 + D x_t, then the silu(z) gate; pure-Python
+    loops with explicit products (no running state)."""
+    u, delta, A, B, C = case["u"], case["delta"], case["A"], case["B"], case["C"]
+    batch, L, dim = u.shape
+    N = A.shape[1]
+    out = np.zeros_like(u)
+    last = np.zeros((batch, dim, N))
+    for b in range(batch):
+        for d in range(dim):
+            dl = []
+            for t in range(L):
+                s = delta[b, t, d] + (case["delta_bias"][d] if case["delta_bias"] is not None else 0.0)
+                dl.append(math.log1p(math.exp(s)) if case["delta_softplus"] else s)
+            abar = [[math.exp(dl[t] * A[d, n]) for n in range(N)] for t in range(L)]
+            if zoh_b:
+                bbar = [[(math.exp(dl[t] * A[d, n]) - 1.0) / (dl[t] * A[d, n]) * dl[t] * B[b, t, n]
+                         for n in range(N)] for t in range(L)]
+            else:
+                bbar = [[dl[t] * B[b, t, n] for n in range(N)] for t in range(L)]
+
+            def state_at(t, n):
+                tot = 0.0
+                if case["h0"] is not None:
+                    p = 1.0
+                    for r in range(0, t + 1):
+                        p *= abar[r][n]
+                    tot += p * case["h0"][b, d, n]
+                for s in range(t + 1):
+                    p = 1.0
+                    for r in range(s + 1, t + 1):
+                        p *= abar[r][n]
+                    tot += p * bbar[s][n] * u[b, s, d]
+                return tot
+
+            for t in range(L):
+                y = sum(C[b, t, n] * state_at(t, n) for n in range(N))
+                if case["D"] is not None:
+                    y += case["D"][d] * u[b, t, d]
+                if case["z"] is not None:
+                    zz = case["z"][b, t, d]
+                    y *= zz * expit(zz)
+                out[b, t, d] = y
+            for n in range(N):
+                last[b, d, n] = state_at(L - 1, n)
+    return out, last
+
+
+def _run(oracle_mod, case, **kw):
+    return oracle_mod.scan(case["u"], case["delta"], case["A"], case["B"], case["C"],
+                           D=case["D"], z=case["z"], delta_bias=case["delta_bias"],
+                           delta_softplus=case["delta_softplus"], h0=case["h0"], **kw)
+
+
+def _close(a, b, tol):
+    a, b = np.asarray(a), np.asarray(b)
+    err = np.max(np.abs(a - b) / (1.0 + np.abs(b))) if a.size else 0.0
+    assert err <= tol, f"max rel err {err:.3e} > {tol:.1e}"
+
+
+@pytest.mark.parametrize("zoh_b", [False, True])
+@pytest.mark.parametrize("variant", ["full", "no_softplus", "no_gate_no_skip", "no_bias_no_h0"])
+def test_brute_force_unrolled_sum(oracle_mod, zoh_b, variant):
+    rng = np.random.default_rng(100 + 7 * zoh_b + len(variant))
+    kw = {}
+    if variant == "no_softplus":
+        kw = dict(softplus=False)
+    elif variant == "no_gate_no_skip":
+        kw = dict(gate=False, dskip=False)
+    elif variant == "no_bias_no_h0":
+        kw = dict(bias=False, h0=False)
+    case = _rand_case(rng, **kw)
+    if variant == "no_softplus":
+        case["delta"] = np.abs(case["delta"]) + 0.05  # keep Delta positive
+    out, last = _run(oracle_mod, case, zoh_b=zoh_b)
+    ref_out, ref_last = _brute(case, zoh_b=zoh_b)
+    _close(out, ref_out, 1e-12)
+    _close(last, ref_last, 1e-12)
+
+
+def test_brute_force_distinguishes_transposes(oracle_mod):
+    """B and C swapped, or A read transposed, must be visible: the pins use
+    dim != dstate != seqlen and asymmetric data."""
+    rng = np.random.default_rng(5)
+    case = _rand_case(rng, batch=1, L=7, dim=2, N=5)
+    out, _ = _run(oracle_mod, case)
+    swapped = dict(case, B=case["C"], C=case["B"])
+    ref_swapped, _ = _brute(swapped)
+    assert np.max(np.abs(out - ref_swapped)) > 1e-3
+
+
+def test_n1_closed_form_constant_input(oracle_mod):
+    """N=1, constant Delta, A, B, C, x, h0 = 0:
+    h_t = Delta B x (1 - a^{t+1}) / (1 - a), a = exp(Delta A)."""
+    L, dlt, a_c, b_c, c_c, x_c, d_c = 40, 0.37, -0.8, 1.3, 0.9, 0.6, 0.25
+    u = np.full((1, L, 1), x_c)
+    delta = np.full((1, L, 1), dlt)
+    out, last = oracle_mod.scan(u, delta, np.array([[a_c]]), np.full((1, L, 1), b_c),
+                                np.full((1, L, 1), c_c), D=np.array([d_c]), delta_softplus=False)
+    a = math.exp(dlt * a_c)
+    t = np.arange(L)
+    h = dlt * b_c * x_c * (1 - a ** (t + 1)) / (1 - a)
+    _close(out[0, :, 0], c_c * h + d_c * x_c, 1e-13)
+    _close(last[0, 0, 0], h[-1], 1e-13)
+
+
+def test_n1_closed_form_impulse(oracle_mod):
+    """Impulse x_0 = 1: h_t = a^t Delta B."""
+    L, dlt, a_c = 30, 0.21, -1.7
+    u = np.zeros((1, L, 1)); u[0, 0, 0] = 1.0
+    out, _ = oracle_mod.scan(u, np.full((1, L, 1), dlt), np.array([[a_c]]),
+                             np.ones((1, L, 1)), np.ones((1, L, 1)), delta_softplus=False)
+    a = math.exp(dlt * a_c)
+    _close(out[0, :, 0], dlt * a ** np.arange(L), 1e-14)
+
+
+@pytest.mark.parametrize("softplus", [False, True])
+def test_lti_equals_convolution(oracle_mod, softplus):
+    """With Delta, B, C constant in time the recurrence is the convolution
+    y = x * K + D x, K_k = sum_n C_n exp(k Delta A_n) Delta B_n (NL-345
+    section 2, eq. (3) and "Linear Time Invariance"); numpy.convolve is the
+    independent route."""
+    rng = np.random.default_rng(11)
+    batch, L, dim, N = 2, 64, 3, 5
+    A = -rng.uniform(0.1, 3.0, size=(dim, N))
+    Bv, Cv = rng.standard_normal((batch, N)), rng.standard_normal((batch, N))
+    draw = rng.uniform(-2.0, 0.5, size=(batch, dim))
+    bias = rng.uniform(-0.5, 0.5, size=dim)
+    D = rng.standard_normal(dim)
+    u = rng.standard_normal((batch, L, dim))
+    delta = np.repeat(draw[:, None, :], L, axis=1)
+    B = np.repeat(Bv[:, None, :], L, axis=1)
+    C = np.repeat(Cv[:, None, :], L, axis=1)
+    out, _ = oracle_mod.scan(u, delta, A, B, C, D=D, delta_bias=bias, delta_softplus=softplus)
+    k = np.arange(L)
+    for b in range(batch):
+        for d in range(dim):
+            s = draw[b, d] + bias[d]
+            dlt = np.logaddexp(0.0, s) if softplus else s
+            K = sum(Cv[b, n] * np.exp(k * dlt * A[d, n]) * dlt * Bv[b, n] for n in range(N))
+            ref = np.convolve(u[b, :, d], K)[:L] + D[d] * u[b, :, d]
+            _close(out[b, :, d], ref, 1e-12)
+
+
+def test_delta_zero_keeps_state_exactly(oracle_mod):
+    """Delta = 0 (raw 0, no bias, softplus off): Abar = 1, Bbar = 0, so the state
+    is kept bit for bit and y = C h0 + D u (NL-345 section 2 / the notes: Delta
+    controls how much is remembered)."""
+    rng = np.random.default_rng(3)
+    batch, L, dim, N = 2, 20, 4, 6
+    h0 = rng.standard_normal((batch, dim, N))
+    u = rng.standard_normal((batch, L, dim))
+    C = rng.standard_normal((batch, L, N))
+    D = rng.standard_normal(dim)
+    out, last = oracle_mod.scan(u, np.zeros((batch, L, dim)), -rng.uniform(0.5, 2, (dim, N)),
+                                rng.standard_normal((batch, L, N)), C, D=D,
+                                delta_softplus=False, h0=h0)
+    assert np.array_equal(last, h0)
+    ref = np.einsum("btn,bdn->btd", C, h0) + D[None, None, :] * u
+    _close(out, ref, 1e-14)
+
+
+@pytest.mark.parametrize("zoh_b", [False, True])
+def test_split_and_resume_equals_one_pass(oracle_mod, zoh_b):
+    """Running [0, k) then [k, L) from the returned state is one pass."""
+    rng = np.random.default_rng(21)
+    case = _rand_case(rng, batch=2, L=37, dim=5, N=3)
+    full_out, full_last = _run(oracle_mod, case, zoh_b=zoh_b)
+    for k in (1, 9, 36):
+        first = {key: (v[:, :k] if isinstance(v, np.ndarray) and v.ndim == 3 and v.shape[1] == 37 else v)
+                 for key, v in case.items()}
+        second = {key: (v[:, k:] if isinstance(v, np.ndarray) and v.ndim == 3 and v.shape[1] == 37 else v)
+                  for key, v in case.items()}
+        o1, s1 = _run(oracle_mod, first, zoh_b=zoh_b)
+        second["h0"] = s1
+        o2, s2 = _run(oracle_mod, second, zoh_b=zoh_b)
+        assert np.array_equal(np.concatenate([o1, o2], axis=1), full_out)
+        assert np.array_equal(s2, full_last)
+
+
+def test_theorem1_gated_rnn_under_zoh(oracle_mod):
+    """N=1, A=-1, B=C=1, Delta = softplus(raw + bias): under exact ZOH the scan is
+    h_t = (1 - g_t) h_{t-1} + g_t x_t with g_t = sigmoid(raw_t + bias)
+    (【論文要約】Mamba notes, 数式解説 4, Theorem 1).  Under Euler it is not."""
+    rng = np.random.default_rng(8)
+    L, dim = 50, 3
+    raw = rng.standard_normal((1, L, dim))
+    bias = rng.standard_normal(dim)
+    x = rng.standard_normal((1, L, dim))
+    h0 = rng.standard_normal((1, dim, 1))
+    args = (x, raw, -np.ones((dim, 1)), np.ones((1, L, 1)), np.ones((1, L, 1)))
+    out_zoh, last_zoh = oracle_mod.scan(*args, delta_bias=bias, delta_softplus=True, h0=h0, zoh_b=True)
+    out_eul, _ = oracle_mod.scan(*args, delta_bias=bias, delta_softplus=True, h0=h0, zoh_b=False)
+    ref = np.zeros((L, dim))
+    h = h0[0, :, 0].copy()
+    for t in range(L):
+        g = expit(raw[0, t] + bias)
+        h = (1.0 - g) * h + g * x[0, t]
+        ref[t] = h
+    _close(out_zoh[0], ref, 1e-13)
+    _close(last_zoh[0, :, 0], ref[-1], 1e-13)
+    assert np.max(np.abs(out_eul[0] - ref)) > 1e-2
+
+
+def test_softplus_and_bias_placement(oracle_mod):
+    """N=1, A=0 (Abar = 1), B=C=u=1: y_t = sum_{s<=t} Delta_s with
+    Delta_s = softplus(raw_s + bias) -- the bias goes inside tau_Delta
+    (Algorithm 2).  np.logaddexp is the independent softplus, including
+    arguments far outside the range where log(1 + e^s) is safe."""
+    L = 64
+    raw = np.linspace(-60.0, 60.0, L).reshape(1, L, 1)
+    bias = np.array([0.75])
+    out, _ = oracle_mod.scan(np.ones((1, L, 1)), raw, np.zeros((1, 1)), np.ones((1, L, 1)),
+                             np.ones((1, L, 1)), delta_bias=bias, delta_softplus=True)
+    ref = np.cumsum(np.logaddexp(0.0, raw[0, :, 0] + bias[0]))
+    _close(out[0, :, 0] / (1 + ref), ref / (1 + ref), 1e-14)
+    wrong = np.cumsum(np.logaddexp(0.0, raw[0, :, 0]) + bias[0])
+    assert np.max(np.abs(out[0, :, 0] - wrong)) > 1e-3
+
+
+def test_skip_and_gate(oracle_mod):
+    """No input into the state (B = 0, h0 = 0): out = D u silu(z) with the
+    library sigmoid; C = 0 leaves the same; D absent gives 0."""
+    rng = np.random.default_rng(4)
+    batch, L, dim, N = 2, 9, 3, 4
+    u, z = rng.standard_normal((batch, L, dim)), rng.standard_normal((batch, L, dim)) * 3
+    D = rng.standard_normal(dim)
+    A = -rng.uniform(0.5, 2, (dim, N))
+    zeros_bn = np.zeros((batch, L, N))
+    out, _ = oracle_mod.scan(u, rng.standard_normal((batch, L, dim)), A, zeros_bn,
+                             rng.standard_normal((batch, L, N)), D=D, z=z)
+    _close(out, D * u * z * expit(z), 1e-15)
+    out0, _ = oracle_mod.scan(u, rng.standard_normal((batch, L, dim)), A, zeros_bn, zeros_bn, z=z)
+    assert np.array_equal(out0, np.zeros_like(out0))
+
+
+def test_thread_count_and_channel_subset_invariance(oracle_mod):
+    """Channels are independent (NL-345 section 2, "Structure and Dimensions"):
+    any thread count, and any subset of channels, reproduces the same bits."""
+    rng = np.random.default_rng(6)
+    case = _rand_case(rng, batch=3, L=25, dim=7, N=4)
+    o1, s1 = _run(oracle_mod, case, nthreads=1)
+    o8, s8 = _run(oracle_mod, case, nthreads=8)
+    assert np.array_equal(o1, o8) and np.array_equal(s1, s8)
+    sel = [1, 4, 6]
+    sub = dict(case)
+    for key in ("u", "delta", "z"):
+        sub[key] = case[key][:, :, sel]
+    sub["A"], sub["D"], sub["delta_bias"] = case["A"][sel], case["D"][sel], case["delta_bias"][sel]
+    sub["h0"] = case["h0"][:, sel]
+    os_, ss = _run(oracle_mod, sub)
+    assert np.array_equal(os_, o1[:, :, sel]) and np.array_equal(ss, s1[:, sel])
+
+
+def test_decode_one_step_brute_force(oracle_mod):
+    rng = np.random.default_rng(9)
+    batch, dim, N = 3, 5, 4
+    h = rng.standard_normal((batch, dim, N))
+    x, dt, z = rng.standard_normal((batch, dim)), rng.uniform(0.01, 0.5, (batch, dim)), rng.standard_normal((batch, dim))
+    A = -rng.uniform(0.5, 3, (dim, N))
+    B, C, D = rng.standard_normal((batch, N)), rng.standard_normal((batch, N)), rng.standard_normal(dim)
+    out, hn = oracle_mod.state_update(h, x, dt, A, B, C, D=D, z=z)
+    for b in range(batch):
+        for d in range(dim):
+            newh = [math.exp(dt[b, d] * A[d, n]) * h[b, d, n] + dt[b, d] * B[b, n] * x[b, d] for n in range(N)]
+            y = sum(C[b, n] * newh[n] for n in range(N)) + D[d] * x[b, d]
+            y *= z[b, d] * expit(z[b, d])
+            assert abs(out[b, d] - y) <= 1e-14 * (1 + abs(y))
+            assert np.allclose(hn[b, d], newh, rtol=1e-15, atol=0)
+
+
+def test_decode_steps_equal_scan(oracle_mod):
+    """Recurrent mode (NL-345 section 1: constant time per step, no cache of
+    past elements): 1000 decode steps equal one scan over the same 1000 steps,
+    same Delta (softplus off, no bias), starting from the same state."""
+    rng = np.random.default_rng(12)
+    batch, dim, N, L = 2, 3, 4, 1000
+    h0 = rng.standard_normal((batch, dim, N)) * 0.1
+    x, z = rng.standard_normal((batch, L, dim)), rng.standard_normal((batch, L, dim))
+    dt = np.logaddexp(0.0, rng.standard_normal((batch, L, dim)) * 0.5 - 4.0)
+    B, C = rng.standard_normal((batch, L, N)), rng.standard_normal((batch, L, N))
+    A = -np.tile(np.arange(1, N + 1, dtype=float), (dim, 1))
+    D = rng.uniform(0.5, 1.5, dim)
+    out_scan, last_scan = oracle_mod.scan(x, dt, A, B, C, D=D, z=z, delta_softplus=False, h0=h0)
+    h = h0
+    outs = []
+    for t in range(L):
+        o, h = oracle_mod.state_update(h, x[:, t], dt[:, t], A, B[:, t], C[:, t], D=D, z=z[:, t])
+        outs.append(o)
+    assert np.array_equal(np.stack(outs, axis=1), out_scan)
+    assert np.array_equal(h, last_scan)
+
+
+def test_empty_and_degenerate_shapes(oracle_mod):
+    rng = np.random.default_rng(1)
+    # seqlen 0: no output, state passes through
+    h0 = rng.standard_normal((2, 3, 4))
+    out, last = oracle_mod.scan(np.zeros((2, 0, 3)), np.zeros((2, 0, 3)), -np.ones((3, 4)),
+                                np.zeros((2, 0, 4)), np.zeros((2, 0, 4)), h0=h0)
+    assert out.shape == (2, 0, 3) and np.array_equal(last, h0)
+    # dstate 0: y = D u silu(z)
+    u, z = rng.standard_normal((1, 5, 2)), rng.standard_normal((1, 5, 2))
+    out, last = oracle_mod.scan(u, rng.standard_normal((1, 5, 2)), np.zeros((2, 0)),
+                                np.zeros((1, 5, 0)), np.zeros((1, 5, 0)), D=np.array([2.0, -1.0]), z=z)
+    _close(out, np.array([2.0, -1.0]) * u * z * expit(z), 1e-15)
