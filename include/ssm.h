@@ -1,0 +1,166 @@
+/*
+ * ssm.h -- C ABI of the B200 selective state-space (S6) library.
+ *
+ * The library computes the selective SSM of Mamba ("Mamba: Linear-Time
+ * Sequence Modeling with Selective State Spaces") with hand-written sm_100a
+ * CUDA kernels.  For every channel (b, d) independently (NL-345 Mamba
+ * translation, section 2 "Structure and Dimensions"):
+ *
+ *   Delta_t = softplus(delta[b,t,d] + delta_bias[d])   (or the plain sum)
+ *   Abar    = exp(Delta_t * A[d,n])                    (zero-order hold on A)
+ *   Bbar    = Delta_t * B[b,t,n]                       (Euler form on B)
+ *   h_t[n]  = Abar * h_{t-1}[n] + Bbar * u[b,t,d]      (section 2, eq. (2))
+ *   y_t     = sum_n C[b,t,n] * h_t[n] + D[d] * u[b,t,d]
+ *   out     = y_t * silu(z[b,t,d])                      (if z is given)
+ *
+ * Sources: NL-345 translation, section 2 "Discretization" and eq. (2)
+ * (recurrence, readout after the update); 【論文要約】Mamba notes, 数式解説 3
+ * (ZOH for Abar) and the "S6" section, Algorithm 2 (B, C per token, Delta =
+ * softplus(parameter + projection)).  The pages give the exact ZOH form for
+ * Bbar; this library uses the Euler form Delta * B.  The D skip and the silu(z)
+ * gate are the Mamba block's epilogue fused into the scan.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc / cudaMallocAsync /
+ *    torch CUDA memory) on the current device; the caller owns every buffer.
+ *  - Layouts are dense and row-major:
+ *      u, delta, z, out : (batch, seqlen, dim)     dim contiguous
+ *      B, C             : (batch, seqlen, dstate)  dstate contiguous
+ *      A                : (dim, dstate)            float32
+ *      D, delta_bias    : (dim)                    float32
+ *      state/last_state : (batch, dim, dstate)     float32
+ *    "io" selects the element type of u, delta, z, B, C (and x, dt for the
+ *    decode step) and out: SSM_F32 = float, SSM_BF16 = bfloat16 (out rounded
+ *    to nearest even).  All arithmetic is fp32.
+ *  - Every pointer must be aligned to its element size; no other alignment is
+ *    required.  Sizes are arbitrary (ragged tails are masked); 1 <= dstate <= 64.
+ *  - Work is enqueued on "stream" (a cudaStream_t; NULL is the legacy default
+ *    stream).  No entry point synchronises the stream or the device.
+ *  - Argument errors return SSM_ERR_INVALID_ARG or SSM_ERR_UNSUPPORTED before
+ *    anything is enqueued.  A failed launch returns SSM_ERR_CUDA.  The message
+ *    of the last failure on the calling thread is ssm_last_error().
+ *  - out must not overlap any input.  Calls are thread-safe.
+ */
+#ifndef SSM_B200_H
+#define SSM_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad flag */
+    SSM_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (dstate > 64) */
+    SSM_ERR_CUDA = 3         /* a CUDA call failed; see ssm_last_error() */
+} ssm_status;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+typedef struct {
+    int64_t batch;  /* Bt */
+    int64_t seqlen; /* L (ignored by the decode step) */
+    int64_t dim;    /* D: channels */
+    int64_t dstate; /* N: state size per channel */
+} ssm_dims;
+
+/* A cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st *ssm_stream;
+
+/*
+ * Selective scan, forward (one pass over the whole sequence).
+ *
+ *   u, delta       : (batch, seqlen, dim) io; delta is the raw Delta.
+ *   A              : (dim, dstate) float32, used as given (no sign check).
+ *   B, C           : (batch, seqlen, dstate) io, shared by all channels.
+ *   D              : (dim) float32 or NULL (no skip term).
+ *   z              : (batch, seqlen, dim) io or NULL (no gate).
+ *   delta_bias     : (dim) float32 or NULL (zero bias).
+ *   delta_softplus : 1 => Delta = softplus(delta + bias); 0 => delta + bias.
+ *   out            : (batch, seqlen, dim) io, written.
+ *   last_state     : (batch, dim, dstate) float32 or NULL.  In: h_0 (the scan
+ *                    resumes from it).  Out: h_L.  NULL => h_0 = 0, h_L not
+ *                    returned.  With seqlen == 0 it is left unchanged.
+ *
+ * The expanded (batch, seqlen, dim, dstate) state never exists in memory; the
+ * fp32 state lives in registers.  When batch * dim is too small to fill the
+ * GPU, the sequence is split into segments scanned in parallel and joined
+ * with the associative combine (a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2); the
+ * per-segment carries (8 bytes per (batch, segment, dim, dstate) plus 4 per
+ * (batch, segment, dim)) are allocated with cudaMallocAsync on "stream" and
+ * released with cudaFreeAsync on the same stream.
+ */
+ssm_status ssm_selective_scan_fwd(ssm_dims dims, ssm_dtype io,
+                                  const void *u, const void *delta, const float *A,
+                                  const void *B, const void *C, const float *D,
+                                  const void *z, const float *delta_bias, int delta_softplus,
+                                  void *out, float *last_state, ssm_stream stream);
+
+/* Execution choices for ssm_selective_scan_fwd_ex; zero-initialise for defaults. */
+typedef enum {
+    SSM_VARIANT_AUTO = 0,  /* pick by shape */
+    SSM_VARIANT_SLAB = 1,  /* one pass: each thread group owns channels for all of L */
+    SSM_VARIANT_SPLIT = 2  /* sequence split: segment carries, then a second pass */
+} ssm_variant;
+
+typedef enum {
+    SSM_KERNEL_AUTO = 0,     /* staged when eligible, else generic */
+    SSM_KERNEL_GENERIC = 1,  /* direct global loads; any size and element alignment */
+    SSM_KERNEL_STAGED = 2    /* inputs staged through shared memory with 16-byte async
+                                copies; needs dim and dstate rows of a multiple of 16
+                                bytes and 16-byte aligned u, delta, z, B, C
+                                (SSM_ERR_UNSUPPORTED otherwise) */
+} ssm_kernel_family;
+
+typedef struct {
+    int32_t variant;  /* ssm_variant */
+    int32_t segments; /* SPLIT only: number of sequence segments, 0 = automatic */
+    int32_t lanes;    /* lanes sharing one channel: 0 = automatic, else 1, 2 or 4
+                         (honoured for 9 <= dstate <= 32) */
+    int32_t family;   /* ssm_kernel_family */
+    int32_t reserved[4]; /* must be zero */
+} ssm_scan_opts;
+
+/* ssm_selective_scan_fwd with explicit execution choices (opts may be NULL).
+ * Every variant computes the same function; results agree to fp32 rounding. */
+ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io,
+                                     const void *u, const void *delta, const float *A,
+                                     const void *B, const void *C, const float *D,
+                                     const void *z, const float *delta_bias, int delta_softplus,
+                                     void *out, float *last_state, const ssm_scan_opts *opts,
+                                     ssm_stream stream);
+
+/*
+ * One recurrent (decode) step for every channel: constant time and memory per
+ * generated token, no cache of past inputs (NL-345 section 1, "Fast training
+ * and inference"; section 2 eq. (2) for a single t).
+ *
+ *   state : (batch, dim, dstate) float32, updated in place (h_{t-1} -> h_t).
+ *   x, dt : (batch, dim) io; dt is the time step itself (already positive:
+ *           no bias and no softplus are applied).
+ *   A     : (dim, dstate) float32.     B, C : (batch, dstate) io.
+ *   D     : (dim) float32 or NULL.     z    : (batch, dim) io or NULL.
+ *   out   : (batch, dim) io.
+ * dims.seqlen is ignored.
+ */
+ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
+                                      const void *x, const void *dt, const float *A,
+                                      const void *B, const void *C, const float *D,
+                                      const void *z, void *out, ssm_stream stream);
+
+/* Static description of a status code. */
+const char *ssm_status_string(ssm_status status);
+
+/* Detail of the last non-OK status returned on the calling thread ("" if none). */
+const char *ssm_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_B200_H */

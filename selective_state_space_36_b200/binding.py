@@ -1,0 +1,167 @@
+"""Thin ctypes binding of the C ABI in include/ssm.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libssm_b200.so.  torch supplies device memory and the stream.  If
+the library is missing this module raises at import; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssm_b200.so")
+
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA = 0, 1, 2, 3
+SSM_F32, SSM_BF16 = 0, 1
+VARIANTS = {"auto": 0, "slab": 1, "split": 2}
+FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
+
+# every symbol include/ssm.h declares
+EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_state_update",
+            "ssm_status_string", "ssm_last_error", "ssm_version")
+
+
+class SSMDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("dim", ctypes.c_int64), ("dstate", ctypes.c_int64)]
+
+
+class SSMScanOpts(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
+                ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
+
+
+class SSMError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{_status_str(status)}: {detail}")
+
+
+_vp = ctypes.c_void_p
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m selective_state_space_36_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    scan_args = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _vp, _vp]
+    lib.ssm_selective_scan_fwd.argtypes = scan_args + [_vp]
+    lib.ssm_selective_scan_fwd.restype = ctypes.c_int
+    lib.ssm_selective_scan_fwd_ex.argtypes = scan_args + [ctypes.POINTER(SSMScanOpts), _vp]
+    lib.ssm_selective_scan_fwd_ex.restype = ctypes.c_int
+    lib.ssm_selective_state_update.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _vp]
+    lib.ssm_selective_state_update.restype = ctypes.c_int
+    lib.ssm_status_string.argtypes = [ctypes.c_int]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_last_error.argtypes = []
+    lib.ssm_last_error.restype = ctypes.c_char_p
+    lib.ssm_version.argtypes = []
+    lib.ssm_version.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _status_str(s: int) -> str:
+    return lib.ssm_status_string(s).decode()
+
+
+def check(status: int) -> None:
+    if status != SSM_OK:
+        raise SSMError(status, lib.ssm_last_error().decode())
+
+
+def _io_of(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SSM_F32
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    raise TypeError(f"unsupported I/O dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, shape=None, device=None) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr() if t.numel() else None
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                       out=None, last_state=None, variant: str = "auto", segments: int = 0,
+                       lanes: int = 0, family: str = "auto", stream=None):
+    """Selective scan forward on CUDA tensors; returns ``out``.
+
+    u, delta, z: (batch, seqlen, dim); B, C: (batch, seqlen, dstate) -- all
+    float32 or all bfloat16.  A (dim, dstate), D and delta_bias (dim,) float32.
+    last_state (batch, dim, dstate) float32 is read as h_0 and overwritten with
+    h_L.  ``variant``/``segments``/``lanes``/``family`` force an execution
+    choice (sequence split, lanes per channel, generic or staged kernel).
+    """
+    io = _io_of(u)
+    batch, seqlen, dim = u.shape
+    dstate = A.shape[1]
+    dev = u.device
+    if out is None:
+        out = torch.empty_like(u)
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate)
+    args = [
+        _ptr(u, "u", u.dtype, seq, dev), _ptr(delta, "delta", u.dtype, seq, dev),
+        _ptr(A, "A", torch.float32, (dim, dstate), dev), _ptr(B, "B", u.dtype, bc, dev),
+        _ptr(C, "C", u.dtype, bc, dev), _ptr(D, "D", torch.float32, (dim,), dev),
+        _ptr(z, "z", u.dtype, seq, dev), _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev),
+        int(bool(delta_softplus)), _ptr(out, "out", u.dtype, seq, dev),
+        _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate), dev),
+    ]
+    dims = SSMDims(batch, seqlen, dim, dstate)
+    if variant == "auto" and not segments and not lanes and family == "auto":
+        check(lib.ssm_selective_scan_fwd(dims, io, *args, _stream_handle(stream)))
+    else:
+        opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
+        check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
+    return out
+
+
+def selective_state_update(state, x, dt, A, B, C, D=None, z=None, out=None, stream=None):
+    """One decode step on CUDA tensors; ``state`` is updated in place; returns ``out``.
+
+    state (batch, dim, dstate) float32; x, dt, z (batch, dim) and B, C
+    (batch, dstate) float32 or bfloat16; A (dim, dstate), D (dim,) float32.
+    """
+    io = _io_of(x)
+    batch, dim = x.shape
+    dstate = A.shape[1]
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    bd, bn = (batch, dim), (batch, dstate)
+    check(lib.ssm_selective_state_update(
+        SSMDims(batch, 0, dim, dstate), io,
+        _ptr(state, "state", torch.float32, (batch, dim, dstate), dev),
+        _ptr(x, "x", x.dtype, bd, dev), _ptr(dt, "dt", x.dtype, bd, dev),
+        _ptr(A, "A", torch.float32, (dim, dstate), dev), _ptr(B, "B", x.dtype, bn, dev),
+        _ptr(C, "C", x.dtype, bn, dev), _ptr(D, "D", torch.float32, (dim,), dev),
+        _ptr(z, "z", x.dtype, bd, dev), _ptr(out, "out", x.dtype, bd, dev), _stream_handle(stream)))
+    return out

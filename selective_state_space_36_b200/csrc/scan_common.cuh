@@ -1,0 +1,128 @@
+// scan_common.cuh -- per-lane pieces shared by the scan kernels: the lane's
+// slice of A and D, the initial state (h_0, or the carry folded from earlier
+// segments), and the final write of the state or the segment aggregate.
+#pragma once
+
+#include "scan_kernels.cuh"
+
+namespace ssm {
+
+// Cooperative-group geometry of a scan block: G lanes per channel.
+template <int G>
+struct LaneGeom {
+    static constexpr int CPB = kBlock / G;  // channels per block
+    int q;                                   // lane within the channel group
+    int ch;                                  // channel within the block
+    int64_t b, d;                            // batch row, channel
+    bool active;
+    __device__ LaneGeom(const ScanArgs &a) {
+        q = threadIdx.x % G;
+        ch = threadIdx.x / G;
+        const int64_t tiles = (a.dim + CPB - 1) / CPB;
+        b = blockIdx.x / tiles;
+        d = (blockIdx.x % tiles) * CPB + ch;
+        active = d < a.dim;
+    }
+};
+
+// A (pre-scaled for the decay tier) and the initial state of this lane.
+template <int NS, int G, bool PRECISE, int MODE>
+__device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneGeom<G> &g, int seg,
+                                          float (&Aw)[NS], float (&h)[NS]) {
+    const int N = a.dstate;
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int n = g.q * NS + i;
+        const bool ok = g.active && n < N;
+        Aw[i] = ok ? scale_A<PRECISE>(a.A[g.d * N + n]) : 0.f;
+        h[i] = 0.f;
+    }
+    if (!g.active) return;
+    const int64_t soff = (g.b * a.dim + g.d) * N;
+    if (MODE == kFull && a.last_state) {
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int n = g.q * NS + i;
+            if (n < N) h[i] = a.last_state[soff + n];
+        }
+    }
+    // The split passes read h_0 from last_state only in segment 0 of the first
+    // pass, which copies it to the workspace: the last segment of the second
+    // pass overwrites last_state while other segments may still be starting.
+    if (MODE == kSegAgg && seg == 0 && a.last_state) {
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int n = g.q * NS + i;
+            if (n < N) a.seg_h0[soff + n] = a.last_state[soff + n];
+        }
+    }
+    if (MODE == kSegFinal) {
+        if (a.last_state) {
+#pragma unroll
+            for (int i = 0; i < NS; ++i) {
+                const int n = g.q * NS + i;
+                if (n < N) h[i] = a.seg_h0[soff + n];
+            }
+        }
+        // carry-in: left fold of the earlier segments' (P, h_loc) with
+        // (P1, h1) o (P2, h2) = (P1 P2, P2 h1 + h2), applied to h_0
+        for (int s = 0; s < seg; ++s) {
+            const int64_t agg = (g.b * a.nseg + s) * a.dim + g.d;
+            const float dsum = a.seg_dsum[agg];
+#pragma unroll
+            for (int i = 0; i < NS; ++i) {
+                const int n = g.q * NS + i;
+                if (n < N) h[i] = fmaf(decay<PRECISE>(dsum, Aw[i]), h[i], a.seg_h[agg * N + n]);
+            }
+        }
+    }
+}
+
+// Final state (one pass, or the last segment) or the segment aggregate.
+template <int NS, int G, int MODE>
+__device__ __forceinline__ void lane_finish(const ScanArgs &a, const LaneGeom<G> &g, int seg,
+                                            int64_t t_end, const float (&h)[NS], double dsum) {
+    if (!g.active) return;
+    const int N = a.dstate;
+    if (MODE == kSegAgg) {
+        const int64_t agg = (g.b * a.nseg + seg) * a.dim + g.d;
+        if (g.q == 0) a.seg_dsum[agg] = (float)dsum;
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int n = g.q * NS + i;
+            if (n < N) a.seg_h[agg * N + n] = h[i];
+        }
+    } else if (a.last_state && t_end == a.seqlen) {
+        const int64_t soff = (g.b * a.dim + g.d) * N;
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int n = g.q * NS + i;
+            if (n < N) a.last_state[soff + n] = h[i];
+        }
+    }
+}
+
+// One time step of one channel: discretise, recur, read out.  Returns this
+// lane's partial y (its states only).  du = Delta * u.
+template <int NS, bool PRECISE>
+__device__ __forceinline__ float lane_step(float dl, float du, const float *Bs, const float *Cs,
+                                           const float (&Aw)[NS], float (&h)[NS]) {
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NS; i += 4) {
+        const float4 bv = *reinterpret_cast<const float4 *>(Bs + i);
+        const float4 cv = *reinterpret_cast<const float4 *>(Cs + i);
+        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+        const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float a = decay<PRECISE>(dl, Aw[i + k]);
+            h[i + k] = fmaf(a, h[i + k], du * bb[k]);
+            if (k & 1) y1 = fmaf(cc[k], h[i + k], y1);
+            else y0 = fmaf(cc[k], h[i + k], y0);
+        }
+    }
+    return y0 + y1;
+}
+
+}  // namespace ssm

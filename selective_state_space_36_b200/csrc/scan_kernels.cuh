@@ -1,0 +1,55 @@
+// scan_kernels.cuh -- argument block and launch entry points of the scan and
+// decode kernels (internal to the library; the public ABI is include/ssm.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "ssm_device.cuh"
+
+namespace ssm {
+
+constexpr int kBlock = 128;  // threads per block
+constexpr int kChunk = 64;   // time steps of B/C staged in shared memory at once
+
+enum ScanMode { kFull = 0, kSegAgg = 1, kSegFinal = 2 };
+enum { kVariantSlab = 1, kVariantSplit = 2 };
+// kernel family: generic (direct global loads, any alignment) or staged
+// (cp.async pipeline through shared memory, 16-byte aligned rows)
+enum { kFamilyAuto = 0, kFamilyGeneric = 1, kFamilyStaged = 2 };
+
+struct ScanArgs {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *Dskip, *bias;
+    void *out;
+    float *last_state;
+    // sequence-split workspace: h_0 copy (batch, dim, N), local end states
+    // (batch, nseg, dim, N), Delta sums (batch, nseg, dim)
+    float *seg_h0, *seg_h, *seg_dsum;
+    int64_t batch, seqlen, dim;
+    int dstate;
+    int softplus;
+    int64_t seg_len;  // time steps per segment (== seqlen for one pass)
+    int nseg;
+};
+
+struct DecodeArgs {
+    float *state;
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *Dskip;
+    void *out;
+    int64_t batch, dim;
+    int dstate;
+};
+
+cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int variant, int family,
+                            cudaStream_t st);
+cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int variant,
+                               cudaStream_t st);
+bool staged_eligible(const ScanArgs &a, int es);
+bool scan_shape_supported(int ns, int g);
+cudaError_t launch_state_update(const DecodeArgs &a, bool bf16, int ns, int g, cudaStream_t st);
+
+}  // namespace ssm

@@ -1,0 +1,266 @@
+// ssm_api.cu -- the C ABI declared in include/ssm.h: argument validation,
+// choice of kernel variant and thread layout, launch, error reporting.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/ssm.h"
+#include "scan_kernels.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+ssm_status fail(ssm_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ssm_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SSM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool misaligned(const void *p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) != 0; }
+
+constexpr int64_t kMaxDstate = 64;
+constexpr int64_t kMaxGridX = 2147483647LL;
+
+// Resident 128-thread blocks the scan kernels aim to keep per SM; used to
+// size the sequence split.
+constexpr int kTargetBlocksPerSm = 6;
+
+struct DeviceInfo {
+    int sms = 148;
+};
+
+DeviceInfo device_info() {
+    DeviceInfo di;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            di.sms = v;
+    }
+    return di;
+}
+
+// Lanes per channel (G) and states per lane (NS) for the scan.  lanes_req
+// (0 = automatic) is honoured where a kernel exists for it.
+void scan_layout(int64_t dstate, int64_t channels, int sms, int lanes_req, int *ns, int *g) {
+    if (dstate <= 4) { *ns = 4; *g = 1; return; }
+    if (dstate <= 8) { *ns = 8; *g = 1; return; }
+    if (dstate <= 16) {
+        int G = lanes_req;
+        if (G != 1 && G != 2 && G != 4) {
+            // one lane per channel while the channels alone fill the SMs
+            const int64_t want = (int64_t)sms * kTargetBlocksPerSm * ssm::kBlock;
+            G = channels >= want / 2 ? 1 : (channels >= want / 4 ? 2 : 4);
+        }
+        *g = G;
+        *ns = 16 / G;
+        return;
+    }
+    if (dstate <= 32) {
+        if (lanes_req == 4) { *ns = 8; *g = 4; } else { *ns = 16; *g = 2; }
+        return;
+    }
+    *ns = 16;
+    *g = 4;
+}
+
+ssm_status check_io(ssm_dtype io, size_t *elem) {
+    if (io == SSM_F32) { *elem = 4; return SSM_OK; }
+    if (io == SSM_BF16) { *elem = 2; return SSM_OK; }
+    return fail(SSM_ERR_INVALID_ARG, "io dtype %d is not SSM_F32 or SSM_BF16", (int)io);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ssm_status_string(ssm_status s) {
+    switch (s) {
+        case SSM_OK: return "ok";
+        case SSM_ERR_INVALID_ARG: return "invalid argument";
+        case SSM_ERR_UNSUPPORTED: return "unsupported";
+        case SSM_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char *ssm_last_error(void) { return g_last_error; }
+
+int ssm_version(void) { return 100; }
+
+ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, const float *delta_bias, int delta_softplus,
+                                     void *out, float *last_state, const ssm_scan_opts *opts,
+                                     ssm_stream stream) {
+    g_last_error[0] = 0;
+    size_t es = 0;
+    if (ssm_status s = check_io(io, &es)) return s;
+    if (dims.batch < 0 || dims.seqlen < 0 || dims.dim < 0 || dims.dstate < 0)
+        return fail(SSM_ERR_INVALID_ARG, "negative size (batch %lld, seqlen %lld, dim %lld, dstate %lld)",
+                    (long long)dims.batch, (long long)dims.seqlen, (long long)dims.dim,
+                    (long long)dims.dstate);
+    if (dims.dstate < 1) return fail(SSM_ERR_INVALID_ARG, "dstate must be >= 1");
+    if (dims.dstate > kMaxDstate)
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %lld > %lld", (long long)dims.dstate, (long long)kMaxDstate);
+    if (delta_softplus != 0 && delta_softplus != 1)
+        return fail(SSM_ERR_INVALID_ARG, "delta_softplus must be 0 or 1");
+    int variant = opts ? opts->variant : SSM_VARIANT_AUTO;
+    if (variant < SSM_VARIANT_AUTO || variant > SSM_VARIANT_SPLIT)
+        return fail(SSM_ERR_INVALID_ARG, "unknown variant %d", variant);
+    const int lanes_req = opts ? opts->lanes : 0;
+    const int family = opts ? opts->family : 0;
+    if (opts && (opts->reserved[0] || opts->reserved[1] || opts->reserved[2] || opts->reserved[3]))
+        return fail(SSM_ERR_INVALID_ARG, "ssm_scan_opts.reserved must be zero");
+    if (family < ssm::kFamilyAuto || family > ssm::kFamilyStaged)
+        return fail(SSM_ERR_INVALID_ARG, "kernel family must be 0 (auto), 1 (generic) or 2 (staged)");
+    if (lanes_req != 0 && lanes_req != 1 && lanes_req != 2 && lanes_req != 4)
+        return fail(SSM_ERR_INVALID_ARG, "lanes per channel must be 0, 1, 2 or 4");
+    if (opts && opts->segments < 0) return fail(SSM_ERR_INVALID_ARG, "segments must be >= 0");
+    const int64_t channels = dims.batch * dims.dim;
+    if (dims.batch != 0 && channels / dims.batch != dims.dim)
+        return fail(SSM_ERR_INVALID_ARG, "batch * dim overflows");
+    if (channels == 0 || dims.seqlen == 0) return SSM_OK;  // nothing to compute; state unchanged
+    if (dims.seqlen > INT64_MAX / channels / dims.dstate)
+        return fail(SSM_ERR_INVALID_ARG, "batch * seqlen * dim * dstate overflows");
+    if (!u || !delta || !A || !B || !C || !out)
+        return fail(SSM_ERR_INVALID_ARG, "u, delta, A, B, C and out are required");
+    if (misaligned(u, es) || misaligned(delta, es) || misaligned(B, es) || misaligned(C, es) ||
+        misaligned(z, es) || misaligned(out, es) || misaligned(A, 4) || misaligned(D, 4) ||
+        misaligned(delta_bias, 4) || misaligned(last_state, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+
+    const DeviceInfo di = device_info();
+    int ns = 16, g = 1;
+    scan_layout(dims.dstate, channels, di.sms, lanes_req, &ns, &g);
+    if (family == ssm::kFamilyStaged) {
+        ssm::ScanArgs probe{};
+        probe.u = u; probe.delta = delta; probe.z = z; probe.B = B; probe.C = C;
+        probe.dim = dims.dim; probe.dstate = (int)dims.dstate;
+        if (!ssm::staged_eligible(probe, (int)es))
+            return fail(SSM_ERR_UNSUPPORTED, "staged kernel needs 16-byte aligned rows (dim and dstate "
+                        "multiples of %d, 16-byte aligned u, delta, z, B, C)", (int)(16 / es));
+    }
+    if (!ssm::scan_shape_supported(ns, g))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for %d states x %d lanes", ns, g);
+    const int64_t cpb = ssm::kBlock / g;
+    const int64_t blocks = dims.batch * ((dims.dim + cpb - 1) / cpb);
+    if (blocks > kMaxGridX) return fail(SSM_ERR_UNSUPPORTED, "grid too large");
+
+    // Sequence split when the channel blocks alone cannot fill the GPU.
+    int nseg = opts ? opts->segments : 0;
+    if (variant == SSM_VARIANT_AUTO) {
+        const int64_t full = (int64_t)di.sms * kTargetBlocksPerSm;
+        variant = (blocks * 2 <= full && dims.seqlen >= 4 * 1024) ? SSM_VARIANT_SPLIT : SSM_VARIANT_SLAB;
+    }
+    if (variant == SSM_VARIANT_SPLIT && nseg == 0) {
+        const int64_t full = (int64_t)di.sms * kTargetBlocksPerSm;
+        int64_t s = (full + blocks - 1) / blocks;
+        const int64_t max_by_len = (dims.seqlen + ssm::kChunk - 1) / ssm::kChunk;  // >= 1 chunk each
+        if (s > max_by_len) s = max_by_len;
+        if (s > 65535) s = 65535;
+        nseg = (int)(s < 1 ? 1 : s);
+    }
+    if (nseg > 65535) return fail(SSM_ERR_INVALID_ARG, "at most 65535 segments");
+    if (variant == SSM_VARIANT_SPLIT && nseg > dims.seqlen) nseg = (int)dims.seqlen;
+    if (variant == SSM_VARIANT_SPLIT && nseg <= 1) variant = SSM_VARIANT_SLAB;
+
+    ssm::ScanArgs a{};
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.Dskip = D; a.bias = delta_bias;
+    a.out = out; a.last_state = last_state;
+    a.batch = dims.batch; a.seqlen = dims.seqlen; a.dim = dims.dim;
+    a.dstate = (int)dims.dstate;
+    a.softplus = delta_softplus;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    if (variant == SSM_VARIANT_SLAB) {
+        a.seg_len = dims.seqlen;
+        a.nseg = 1;
+        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, ns, g, ssm::kVariantSlab, family, st);
+        if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+        return SSM_OK;
+    }
+
+    // even segments, each a whole number of chunks except the last
+    int64_t seg_len = (dims.seqlen + nseg - 1) / nseg;
+    seg_len = (seg_len + ssm::kChunk - 1) / ssm::kChunk * ssm::kChunk;
+    nseg = (int)((dims.seqlen + seg_len - 1) / seg_len);
+    if (nseg <= 1) {
+        a.seg_len = dims.seqlen;
+        a.nseg = 1;
+        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, ns, g, ssm::kVariantSlab, family, st);
+        if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+        return SSM_OK;
+    }
+    a.seg_len = seg_len;
+    a.nseg = nseg;
+    const size_t n_h0 = (size_t)channels * dims.dstate;
+    const size_t n_h = (size_t)nseg * channels * dims.dstate;
+    const size_t n_ds = (size_t)nseg * channels;
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, (n_h0 + n_h + n_ds) * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    a.seg_h0 = static_cast<float *>(ws);
+    a.seg_h = a.seg_h0 + n_h0;
+    a.seg_dsum = a.seg_h + n_h;
+    e = ssm::launch_scan_fwd(a, io == SSM_BF16, ns, g, ssm::kVariantSplit, family, st);
+    cudaError_t ef = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "split scan launch");
+    if (ef != cudaSuccess) return cuda_fail(ef, "workspace release");
+    return SSM_OK;
+}
+
+ssm_status ssm_selective_scan_fwd(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                  const float *A, const void *B, const void *C, const float *D,
+                                  const void *z, const float *delta_bias, int delta_softplus,
+                                  void *out, float *last_state, ssm_stream stream) {
+    return ssm_selective_scan_fwd_ex(dims, io, u, delta, A, B, C, D, z, delta_bias, delta_softplus,
+                                     out, last_state, nullptr, stream);
+}
+
+ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state, const void *x,
+                                      const void *dt, const float *A, const void *B, const void *C,
+                                      const float *D, const void *z, void *out, ssm_stream stream) {
+    g_last_error[0] = 0;
+    size_t es = 0;
+    if (ssm_status s = check_io(io, &es)) return s;
+    if (dims.batch < 0 || dims.dim < 0 || dims.dstate < 0)
+        return fail(SSM_ERR_INVALID_ARG, "negative size");
+    if (dims.dstate < 1) return fail(SSM_ERR_INVALID_ARG, "dstate must be >= 1");
+    if (dims.dstate > kMaxDstate)
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %lld > %lld", (long long)dims.dstate, (long long)kMaxDstate);
+    const int64_t channels = dims.batch * dims.dim;
+    if (dims.batch != 0 && channels / dims.batch != dims.dim)
+        return fail(SSM_ERR_INVALID_ARG, "batch * dim overflows");
+    if (channels == 0) return SSM_OK;
+    if (channels > INT64_MAX / dims.dstate) return fail(SSM_ERR_INVALID_ARG, "state size overflows");
+    if (!state || !x || !dt || !A || !B || !C || !out)
+        return fail(SSM_ERR_INVALID_ARG, "state, x, dt, A, B, C and out are required");
+    if (misaligned(x, es) || misaligned(dt, es) || misaligned(B, es) || misaligned(C, es) ||
+        misaligned(z, es) || misaligned(out, es) || misaligned(A, 4) || misaligned(D, 4) ||
+        misaligned(state, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+    int g = 1;
+    while (g * 4 < dims.dstate) g *= 2;
+    const int64_t cpb = ssm::kBlock / g;
+    if (dims.batch * ((dims.dim + cpb - 1) / cpb) > kMaxGridX)
+        return fail(SSM_ERR_UNSUPPORTED, "grid too large");
+    ssm::DecodeArgs a{};
+    a.state = state; a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.Dskip = D; a.out = out;
+    a.batch = dims.batch; a.dim = dims.dim; a.dstate = (int)dims.dstate;
+    cudaError_t e = ssm::launch_state_update(a, io == SSM_BF16, 4, g, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+    return SSM_OK;
+}
+
+}  // extern "C"

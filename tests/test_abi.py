@@ -1,0 +1,115 @@
+"""The C-ABI library: it loads, exports every symbol include/ssm.h declares,
+and rejects bad arguments before touching a GPU.  Runs without a GPU: every
+call here returns during host-side validation (or is a no-op on empty sizes),
+so nothing is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm.h")
+
+
+@pytest.fixture(scope="module")
+def b():
+    from selective_state_space_36_b200 import build
+    build.build()
+    from selective_state_space_36_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(b):
+    names = declared_functions()
+    assert set(names) == set(b.EXPORTED)
+    for n in names:
+        assert hasattr(b.lib, n), f"{n} not exported"
+    assert b.lib.ssm_version() >= 100
+    assert b.lib.ssm_status_string(0) == b"ok"
+
+
+def _scan(b, dims, io=1, ptrs=None, softplus=1, opts=None):
+    # ptrs: u, delta, A, B, C, D, z, bias, out, last_state
+    p = dict(u=0x10000, delta=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None,
+             bias=None, out=0x60000, state=None)
+    p.update(ptrs or {})
+    args = [b.SSMDims(*dims), io, p["u"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["z"],
+            p["bias"], softplus, p["out"], p["state"]]
+    if opts is None:
+        return b.lib.ssm_selective_scan_fwd(*args, None)
+    return b.lib.ssm_selective_scan_fwd_ex(*args, ctypes.byref(opts), None)
+
+
+def test_scan_argument_validation(b):
+    ok = (2, 16, 8, 16)
+    assert _scan(b, ok, io=7) == b.SSM_ERR_INVALID_ARG
+    assert b"io dtype" in b.lib.ssm_last_error()
+    assert _scan(b, (2, -1, 8, 16)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, (2, 16, 8, 0)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, (2, 16, 8, 65)) == b.SSM_ERR_UNSUPPORTED
+    assert _scan(b, ok, softplus=2) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, ok, ptrs=dict(u=None)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, ok, ptrs=dict(out=None)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, ok, ptrs=dict(C=None)) == b.SSM_ERR_INVALID_ARG
+    # misaligned: bf16 needs 2-byte, float32 params 4-byte alignment
+    assert _scan(b, ok, ptrs=dict(u=0x10001)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, ok, ptrs=dict(A=0x30002)) == b.SSM_ERR_INVALID_ARG
+    assert _scan(b, ok, io=0, ptrs=dict(z=0x70002)) == b.SSM_ERR_INVALID_ARG
+    assert b"aligned" in b.lib.ssm_last_error()
+    # overflow of the index space
+    assert _scan(b, (1 << 40, 1 << 40, 8, 16)) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(9, 0)
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(2, -3)
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(1, 0, 3)
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(1, 0, 0, 5)
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(1, 0, 0, 0)
+    opts.reserved[2] = 1
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    # staged kernel on rows that are not 16-byte multiples: refused before launch
+    opts = b.SSMScanOpts(1, 0, 0, 2)
+    assert _scan(b, (2, 16, 37, 16), opts=opts) == b.SSM_ERR_UNSUPPORTED
+
+
+def test_scan_empty_sizes_are_noops(b):
+    # nothing is dereferenced or launched when there is no work
+    for dims in [(0, 16, 8, 16), (2, 0, 8, 16), (2, 16, 0, 16)]:
+        assert _scan(b, dims, ptrs=dict(u=None, delta=None, A=None, B=None, C=None, out=None)) == b.SSM_OK
+
+
+def test_state_update_argument_validation(b):
+    f = b.lib.ssm_selective_state_update
+    good = dict(state=0x10000, x=0x20000, dt=0x30000, A=0x40000, B=0x50000, C=0x60000, D=None,
+                z=None, out=0x70000)
+
+    def call(dims, io=1, **kw):
+        p = dict(good, **kw)
+        return f(b.SSMDims(*dims), io, p["state"], p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"],
+                 p["z"], p["out"], None)
+
+    assert call((4, 0, 8, 16), io=5) == b.SSM_ERR_INVALID_ARG
+    assert call((4, 0, 8, 99)) == b.SSM_ERR_UNSUPPORTED
+    assert call((4, 0, -8, 16)) == b.SSM_ERR_INVALID_ARG
+    assert call((4, 0, 8, 16), state=None) == b.SSM_ERR_INVALID_ARG
+    assert call((4, 0, 8, 16), state=0x10002) == b.SSM_ERR_INVALID_ARG
+    assert call((0, 0, 8, 16), state=None, x=None) == b.SSM_OK
+
+
+def test_python_binding_rejects_bad_tensors(b):
+    import torch
+    u = torch.zeros(1, 4, 8)
+    A = torch.zeros(8, 16)
+    with pytest.raises(TypeError):
+        b.selective_scan_fwd(u.double(), u.double(), A, torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
+    with pytest.raises(ValueError):
+        b.selective_scan_fwd(u, u[:, :2], A, torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))

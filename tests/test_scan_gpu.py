@@ -1,0 +1,174 @@
+"""GPU parity of ssm_selective_scan_fwd against the fp64 oracle.
+
+Every case compares the CUDA path (called through the C ABI) element by
+element with the oracle on the same seeded inputs: small shapes spanning
+several chunks, blocks and ragged tails for every kernel layout and variant,
+and the tiny fp32, Mamba-130M and Mamba-1.4B workloads in full (the last in
+the launch configuration the benchmark times).  The L = 1,048,576 workload is
+in test_longseq_gpu.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from selective_state_space_36_b200 import inputs as I
+from tests import ssm_testlib as T
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from selective_state_space_36_b200 import binding
+    return binding
+
+
+def _case(io, batch, L, dim, N, seed, **kw):
+    cfg = I.ScanConfig("case", batch, L, dim, N, io=io, seed=seed, **kw)
+    return cfg, I.scan_inputs(cfg)
+
+
+def _check(x, io, **kw):
+    out, state = T.gpu_scan(x, io, **kw)
+    ref_out, ref_state = T.oracle_scan(x, io)
+    e1 = T.check_out(T.from_dev(out), ref_out, io)
+    e2 = T.check_state(T.from_dev(state), ref_state, io)
+    return e1, e2
+
+
+# ------------------------------------------------------------- named workloads
+def test_tiny_fp32_workload():
+    x = I.scan_inputs(I.TINY_F32)
+    _check(x, "f32")
+
+
+def test_tiny_fp32_workload_with_h0_and_every_variant():
+    x = I.scan_inputs(I.TINY_F32.with_(h0_sigma=0.5))
+    for kw in [dict(variant="slab", lanes=1), dict(variant="slab", lanes=2),
+               dict(variant="slab", lanes=4), dict(variant="split", segments=3),
+               dict(variant="split", segments=4, lanes=4)]:
+        _check(x, "f32", **kw)
+
+
+@pytest.mark.slow
+def test_mamba130m_workload_full():
+    x = I.scan_inputs(I.MAMBA130M)
+    _check(x, "bf16")
+
+
+@pytest.mark.slow
+def test_mamba1p4b_workload_full():
+    """The benchmark's workload and launch configuration, every element."""
+    x = I.scan_inputs(I.MAMBA1P4B)
+    _check(x, "bf16")
+
+
+# ------------------------------------------------------ layouts and variants
+LAYOUTS = [dict(variant="slab", lanes=1), dict(variant="slab", lanes=2), dict(variant="slab", lanes=4),
+           dict(variant="split", segments=2), dict(variant="split", segments=5, lanes=2),
+           dict(variant="split", segments=7, lanes=4)]
+
+
+@pytest.mark.parametrize("family", ["generic", "staged"])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("layout", range(len(LAYOUTS)))
+def test_layouts_ragged(io, layout, family):
+    # dim 200: one full 128-channel tile + a ragged one; L 333 = several chunks + a tail
+    _, x = _case(io, 3, 333, 200, 16, seed=10 + layout, h0_sigma=0.3, d_skip="uniform")
+    _check(x, io, family=family, **LAYOUTS[layout])
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [1, 3, 4, 5, 8, 13, 16, 17, 24, 32, 33, 64])
+def test_state_sizes(io, N):
+    # dim 37: no 16-byte rows, so the generic kernel runs
+    _, x = _case(io, 2, 130, 37, N, seed=N, h0_sigma=0.2)
+    _check(x, io)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [8, 16, 24, 32, 64])
+@pytest.mark.parametrize("lanes", [1, 2, 4])
+def test_state_sizes_staged(io, N, lanes):
+    _, x = _case(io, 2, 130, 40, N, seed=N + lanes, h0_sigma=0.2)
+    _check(x, io, family="staged", lanes=lanes, variant="slab")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("flags", ["no_z", "no_d", "no_bias", "no_softplus", "bare"])
+def test_optional_inputs(io, flags):
+    kw = dict(has_z=flags not in ("no_z", "bare"), has_d=flags not in ("no_d", "bare"),
+              has_bias=flags not in ("no_bias", "bare"), softplus=flags not in ("no_softplus",))
+    if flags == "no_softplus":
+        kw["delta_sigma"] = 0.02  # keep raw + bias (the Delta itself) mostly positive
+    _, x = _case(io, 2, 150, 70, 16, seed=3, **kw)
+    if flags == "no_softplus":
+        # without softplus Delta = raw + bias; make the bias small and positive
+        x["delta_bias"] = np.abs(x["delta_bias"]).astype(np.float32) * 0.01
+    _check(x, io)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_single_step_and_single_channel(io):
+    for (batch, L, dim) in [(1, 1, 1), (1, 1, 300), (2, 65, 1), (1, 64, 129), (5, 2, 3)]:
+        _, x = _case(io, batch, L, dim, 16, seed=L + dim, h0_sigma=0.5)
+        _check(x, io)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_split_equals_slab_long(io):
+    """Sequence split vs one pass at many segment counts, both vs the oracle."""
+    _, x = _case(io, 1, 4 * 1024 + 77, 24, 16, seed=7, h0_sigma=0.3)
+    ref_out, ref_state = T.oracle_scan(x, io)
+    for family in ("generic", "staged"):
+        for seg in (2, 3, 16, 65):
+            out, st = T.gpu_scan(x, io, variant="split", segments=seg, family=family)
+            T.check_out(T.from_dev(out), ref_out, io)
+            T.check_state(T.from_dev(st), ref_state, io)
+
+
+def test_delta_zero_keeps_state_bit_exact():
+    """Delta = 0 (raw 0, no bias, softplus off): Abar = 1 and Bbar = 0, so the
+    state comes back bit for bit and out = C h0 + D u."""
+    for io in ("f32", "bf16"):
+        _, x = _case(io, 2, 100, 50, 16, seed=2, h0_sigma=1.0, softplus=False, has_bias=False, has_z=False)
+        x["delta"] = np.zeros_like(x["delta"])
+        out, st = T.gpu_scan(x, io)
+        assert np.array_equal(st.cpu().numpy(), x["h0"])
+        ref_out, _ = T.oracle_scan(x, io)
+        T.check_out(T.from_dev(out), ref_out, io)
+
+
+def test_resume_from_last_state_equals_one_pass():
+    """Scanning [0, k) then [k, L) from the returned state equals one pass."""
+    for io in ("f32", "bf16"):
+        _, x = _case(io, 2, 700, 96, 16, seed=5)
+        full_out, full_st = T.gpu_scan(x, io)
+        parts, st = [], torch.zeros_like(full_st)
+        for t0, t1 in [(0, 1), (1, 200), (200, 333), (333, 700)]:
+            sl = {k: (v[:, t0:t1] if isinstance(v, np.ndarray) and v.ndim == 3 and k != "h0" else v)
+                  for k, v in x.items()}
+            from selective_state_space_36_b200 import binding
+            d = {k: T.to_dev(v, io) for k, v in sl.items() if isinstance(v, np.ndarray)}
+            parts.append(binding.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],
+                                                    z=d["z"], delta_bias=d["delta_bias"], last_state=st))
+        out = torch.cat(parts, dim=1)
+        ref_out, ref_st = T.oracle_scan(x, io)
+        T.check_out(T.from_dev(out), ref_out, io)
+        T.check_state(T.from_dev(st), ref_st, io)
+        # and against the one-pass GPU result
+        T.check_out(T.from_dev(out), T.from_dev(full_out), io)
+
+
+def test_empty_inputs_leave_state_untouched(lib):
+    for (batch, L, dim) in [(2, 0, 8), (0, 5, 8), (2, 5, 0)]:
+        u = torch.zeros(batch, L, dim, device="cuda", dtype=torch.bfloat16)
+        A = -torch.ones(dim, 16, device="cuda")
+        Bm = torch.zeros(batch, L, 16, device="cuda", dtype=torch.bfloat16)
+        st = torch.randn(batch, dim, 16, device="cuda")
+        st0 = st.clone()
+        out = lib.selective_scan_fwd(u, u, A, Bm, Bm, last_state=st)
+        torch.cuda.synchronize()
+        assert out.shape == (batch, L, dim) and torch.equal(st, st0)
