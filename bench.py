@@ -1,0 +1,371 @@
+"""Benchmark: selective-scan forward throughput at the Mamba-1.4B layer shape.
+
+One step = one ssm_selective_scan_fwd call over one batch of the workload
+(batch 8, L 2048, dim 4096, N 16, bf16 I/O, fp32 state) -- the whole hot path:
+softplus(Delta), discretisation, recurrence, readout, D skip, silu(z) gate, the
+fp32 state in and out.  Inputs are seeded synthetic data of that shape.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of
+the workload on its GPU (independent batches, no collective on the data path:
+weak scaling); the timed region is bracketed by a barrier and a device
+synchronisation and its length is the maximum over ranks.
+
+The reference arm (--impl reference) times the fp64 CPU oracle on the host
+cores on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_36_b200 import inputs as I  # noqa: E402
+
+METRIC = "selective-scan fwd Gelem/s (B·L·D) at 1.4B-layer shape; % of HBM roofline"
+UNIT = "Gelem/s"
+WORKLOAD = I.MAMBA1P4B
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic_bytes(cfg: I.ScanConfig) -> int:
+    """Bytes the method must move once: u, delta, z, B, C read and out written
+    (the fp32 state in/out and A, D, bias are excluded, as in the metric)."""
+    es = 2 if cfg.io == "bf16" else 4
+    return cfg.elements * es * 4 + cfg.batch * cfg.seqlen * cfg.dstate * es * 2
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    """Hash of the CUDA sources: a committed ncu traffic figure is valid only
+    for the kernels it was captured on."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_36_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(sha: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "scan_fwd_mamba1p4b_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_source_sha") != sha:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        self.period = period_s
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._t = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self) -> dict:
+        if self._t:
+            self._stop.set()
+            self._t.join()
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_rate(cfg: I.ScanConfig, budget_s: float, max_rows=None):
+    """The fp64 oracle, as it stands, on whole batch rows of the workload until
+    ``budget_s`` of CPU time has been spent (at least one row).  Returns
+    (Gelem/s, threads, elements, seconds)."""
+    import oracle
+    A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip)
+    one = cfg.with_(batch=1)
+    done, spent, rows = 0, 0.0, 0
+    threads = min(oracle.default_threads(), cfg.dim)
+    while (spent < budget_s or rows == 0) and rows < (max_rows or cfg.batch):
+        x = {k: I.to_f64(I.draw_rows(cfg, k, rows % cfg.batch, 0, cfg.seqlen), cfg.io)[None]
+             for k in I.SEQ_NAMES}
+        t0 = time.perf_counter()
+        oracle.scan(x["u"], x["delta"], A.astype(np.float64), x["B"], x["C"], D=D.astype(np.float64),
+                    z=x["z"], delta_bias=bias.astype(np.float64), delta_softplus=True)
+        spent += time.perf_counter() - t0
+        done += one.seqlen * one.dim
+        rows += 1
+    return done / spent / 1e9, threads, done, spent
+
+
+def run_reference(args, rank: int) -> int:
+    if rank != 0:
+        return 0
+    per_step = []
+    # each step: the oracle on REF_CHANNELS channels of one batch row of the
+    # workload, all 2048 time steps (channels are independent, so this is the
+    # workload's own arithmetic on a bounded sample)
+    REF_CHANNELS = 1024
+    total_el = 0
+    gen_cfg = WORKLOAD
+    A, D, bias = I.channel_params(gen_cfg.seed, gen_cfg.dim, gen_cfg.dstate, gen_cfg.d_skip)
+    A, D, bias = A[:REF_CHANNELS], D[:REF_CHANNELS], bias[:REF_CHANNELS]
+    import oracle
+    xs = []
+    for b in range(min(2, gen_cfg.batch)):
+        row = {k: I.to_f64(I.draw_rows(gen_cfg, k, b, 0, gen_cfg.seqlen), gen_cfg.io)[None]
+               for k in I.SEQ_NAMES}
+        for k in ("u", "delta", "z"):
+            row[k] = np.ascontiguousarray(row[k][:, :, :REF_CHANNELS])
+        xs.append(row)
+    threads = min(oracle.default_threads(), REF_CHANNELS)
+    for i in range(args.warmup + args.steps):
+        x = xs[i % len(xs)]
+        t0 = time.perf_counter()
+        oracle.scan(x["u"], x["delta"], A.astype(np.float64), x["B"], x["C"], D=D.astype(np.float64),
+                    z=x["z"], delta_bias=bias.astype(np.float64), delta_softplus=True)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            per_step.append(dt)
+            total_el += gen_cfg.seqlen * REF_CHANNELS
+    secs = sum(per_step)
+    value = total_el / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD.name, "batch": WORKLOAD.batch, "seqlen": WORKLOAD.seqlen,
+                   "dim": WORKLOAD.dim, "dstate": WORKLOAD.dstate, "io": WORKLOAD.io,
+                   "parallelism": "host threads over channels"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {REF_CHANNELS} channels x {WORKLOAD.seqlen} steps of "
+                                   f"one batch row of the {WORKLOAD.name} workload"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank: int, world: int, local_rank: int) -> int:
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_36_b200 import binding as lib
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    cfg = WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank) if rank else WORKLOAD
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch, name=f"{cfg.name}_batch{args.batch}")
+    x = I.scan_inputs(cfg)
+
+    def up(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    d = {k: up(v) for k, v in x.items() if isinstance(v, np.ndarray)}
+    state0 = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
+    state = state0.clone()
+    out = torch.empty_like(d["u"])
+    stream = torch.cuda.current_stream(dev)
+    plan = lib.scan_plan(cfg.batch, cfg.seqlen, cfg.dim, cfg.dstate, cfg.io)
+
+    # Each step scans one batch of the workload and resumes from the state the
+    # previous step left in last_state (a continued sequence): same work.
+    def step():
+        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e_all0, e_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_all0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+        ev[i][1].record(stream)
+    e_all1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = e_all0.elapsed_time(e_all1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    t = torch.tensor([elapsed_ms, statistics.mean(launch_ms)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, kernel_ms = float(t[0]), float(t[1])
+
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": world * cfg.elements / (elapsed_ms / args.steps * 1e-3) / 1e9,
+                              "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": cfg.name},
+                              "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # end to end through the public call with host buffers: pinned host inputs
+    # copied in, the scan, the output and final state copied back, every step
+    host = {k: v.cpu().pin_memory() for k, v in d.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    host_state = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
+    host_state0 = torch.zeros(state.shape, dtype=state.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + state0.numel() * 4
+    d2h = host_out.numel() * host_out.element_size() + host_state.numel() * 4
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for k in d:
+            d[k].copy_(host[k], non_blocking=True)
+        state.copy_(host_state0, non_blocking=True)
+        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+        host_out.copy_(out, non_blocking=True)
+        host_state.copy_(state, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t2 = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(t2[0]) / e2e_steps
+
+    if rank == 0:
+        peaks = measured_peaks()
+        ms_per_step = elapsed_ms / args.steps
+        value = world * cfg.elements / (ms_per_step * 1e-3) / 1e9
+        abytes = algorithmic_bytes(cfg)
+        achieved_gbs = abytes / (kernel_ms * 1e-3) / 1e9
+        sha = kernel_source_sha()
+        traffic = committed_traffic(sha)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "dim": cfg.dim,
+                       "dstate": cfg.dstate, "io": cfg.io, "per_gpu": "one full workload per GPU",
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"inputs {abytes / 1e6:.0f} MB > {L2_BYTES >> 20} MB L2; no flush",
+                       "plan": plan},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                         "algorithmic_bytes_per_launch": abytes, "kernel_ms": kernel_ms,
+                         "peak_source": peaks["source"] + " (copy bandwidth)",
+                         "kernel_source_sha": sha},
+            "e2e": {"value": world * cfg.elements / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps * plan["launches"],
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, threads, el, secs = oracle_rate(cfg, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"{el // (cfg.seqlen * cfg.dim)} of {cfg.batch} batch rows "
+                                              f"({el} elements, {secs:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true", help="device-timed loop only (profiling cases)")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

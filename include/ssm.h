@@ -132,6 +132,23 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io,
                                      void *out, float *last_state, const ssm_scan_opts *opts,
                                      ssm_stream stream);
 
+/* What a scan call with these arguments would do (nothing is launched or
+ * allocated; data pointers are only inspected for alignment and may be
+ * fake).  Lets a caller size the workspace and count kernel launches. */
+typedef struct {
+    int32_t variant;         /* ssm_variant chosen: SLAB or SPLIT */
+    int32_t segments;        /* sequence segments (1 for SLAB) */
+    int32_t lanes;           /* lanes per channel */
+    int32_t family;          /* ssm_kernel_family chosen: GENERIC or STAGED */
+    int32_t launches;        /* kernels the call enqueues (0 for an empty problem) */
+    int32_t reserved0;
+    int64_t workspace_bytes; /* device scratch the call allocates (SPLIT), else 0 */
+} ssm_scan_plan_info;
+
+ssm_status ssm_scan_plan(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                         const void *B, const void *C, const void *z, const ssm_scan_opts *opts,
+                         ssm_scan_plan_info *info);
+
 /*
  * One recurrent (decode) step for every channel: constant time and memory per
  * generated token, no cache of past inputs (NL-345 section 1, "Fast training

@@ -22,7 +22,7 @@ FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
 
 # every symbol include/ssm.h declares
 EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_state_update",
-            "ssm_status_string", "ssm_last_error", "ssm_version")
+            "ssm_scan_plan", "ssm_status_string", "ssm_last_error", "ssm_version")
 
 
 class SSMDims(ctypes.Structure):
@@ -34,6 +34,13 @@ class SSMScanOpts(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
                 ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
                 ("reserved", ctypes.c_int32 * 4)]
+
+
+class SSMScanPlanInfo(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
+                ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_int64)]
 
 
 class SSMError(RuntimeError):
@@ -58,6 +65,9 @@ def _load() -> ctypes.CDLL:
     lib.ssm_selective_state_update.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp]
     lib.ssm_selective_state_update.restype = ctypes.c_int
+    lib.ssm_scan_plan.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                  ctypes.POINTER(SSMScanOpts), ctypes.POINTER(SSMScanPlanInfo)]
+    lib.ssm_scan_plan.restype = ctypes.c_int
     lib.ssm_status_string.argtypes = [ctypes.c_int]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_last_error.argtypes = []
@@ -142,6 +152,23 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
         opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
     return out
+
+
+def scan_plan(batch: int, seqlen: int, dim: int, dstate: int, io: str = "bf16",
+              variant: str = "auto", segments: int = 0, lanes: int = 0, family: str = "auto",
+              aligned: bool = True) -> dict:
+    """What ssm_selective_scan_fwd would do for this shape (no GPU work).
+    ``aligned`` describes the data pointers (16-byte aligned or not)."""
+    base = 0x100000 if aligned else 0x100002
+    opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
+    info = SSMScanPlanInfo()
+    check(lib.ssm_scan_plan(SSMDims(batch, seqlen, dim, dstate), SSM_BF16 if io == "bf16" else SSM_F32,
+                            base, base, base, base, base, ctypes.byref(opts), ctypes.byref(info)))
+    inv_v = {v: k for k, v in VARIANTS.items()}
+    inv_f = {v: k for k, v in FAMILIES.items()}
+    return {"variant": inv_v.get(info.variant, "none"), "segments": info.segments, "lanes": info.lanes,
+            "family": inv_f.get(info.family, "none"), "launches": info.launches,
+            "workspace_bytes": info.workspace_bytes}
 
 
 def selective_state_update(state, x, dt, A, B, C, D=None, z=None, out=None, stream=None):

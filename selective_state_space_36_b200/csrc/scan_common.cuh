@@ -125,4 +125,48 @@ __device__ __forceinline__ float lane_step(float dl, float du, const float *Bs, 
     return y0 + y1;
 }
 
+// K consecutive time steps of one channel (this lane's NS states, NS a
+// multiple of 4), with the per-step scalars Delta (dl) and Delta * u (du)
+// already computed.  Step k reads B/C row k at Bs + k * stride and
+// Cs + k * stride.  The states are handled in pairs (n, n + 1); in the fast
+// tier the pair's products and fused multiply-adds are single f32x2
+// instructions.  Returns this lane's partial y of each step.
+template <int K, int NS, bool PRECISE>
+__device__ __forceinline__ void recur_block(const float (&dl)[K], const float (&du)[K],
+                                            const float *Bs, const float *Cs, int stride,
+                                            const float2 (&A2)[NS / 2], float2 (&h2)[NS / 2],
+                                            float (&y)[K]) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const float2 d2 = make_float2(dl[k], dl[k]);
+        const float2 u2 = make_float2(du[k], du[k]);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < NS / 4; ++j) {
+            const float4 bv = *reinterpret_cast<const float4 *>(Bs + k * stride + 4 * j);
+            const float4 cv = *reinterpret_cast<const float4 *>(Cs + k * stride + 4 * j);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                const int p = 2 * j + hlf;
+                const float2 b2 = hlf ? make_float2(bv.z, bv.w) : make_float2(bv.x, bv.y);
+                const float2 c2 = hlf ? make_float2(cv.z, cv.w) : make_float2(cv.x, cv.y);
+                if (!PRECISE) {
+                    // fast tier: the state pairs on f32x2 (half the issue slots)
+                    const float2 x2 = mul2(d2, A2[p]);
+                    const float2 a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
+                    h2[p] = fma2(a2, h2[p], mul2(u2, b2));
+                    acc = fma2(c2, h2[p], acc);
+                } else {
+                    const float ax = decay_of<PRECISE>(d2.x * A2[p].x), ay = decay_of<PRECISE>(d2.y * A2[p].y);
+                    h2[p].x = fmaf(ax, h2[p].x, u2.x * b2.x);
+                    h2[p].y = fmaf(ay, h2[p].y, u2.y * b2.y);
+                    acc.x = fmaf(c2.x, h2[p].x, acc.x);
+                    acc.y = fmaf(c2.y, h2[p].y, acc.y);
+                }
+            }
+        }
+        y[k] = acc.x + acc.y;
+    }
+}
+
 }  // namespace ssm

@@ -21,6 +21,16 @@
 
 namespace ssm {
 
+#ifndef SSM_KSTEP
+#define SSM_KSTEP 4
+#endif
+// Time steps processed together: a multiple of 2G (so each lane owns an even
+// number of them) that divides the chunk.
+template <int G>
+struct KStep {
+    static constexpr int value = SSM_KSTEP > 2 * G ? SSM_KSTEP : 2 * G;
+};
+
 template <typename IO>
 struct StagedCfg {
     static constexpr int T = sizeof(IO) == 2 ? 32 : 16;  // time steps per chunk
@@ -59,6 +69,8 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP;
     constexpr int EPV = 16 / sizeof(IO);  // elements per 16-byte piece
     constexpr int ROWV = CPB / EPV;       // pieces per tile row
+    constexpr int KSTEP = KStep<G>::value;
+    constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
     extern __shared__ __align__(16) unsigned char smem[];
     float *fB = reinterpret_cast<float *>(smem + S * Lay::STAGE_BYTES);
     float *fC = fB + T * NSP;
@@ -109,6 +121,12 @@ scan_fwd_staged_kernel(const ScanArgs args) {
 
     float Aw[NS], h[NS];
     lane_init<NS, G, PRECISE, MODE>(args, g, seg, Aw, h);
+    float2 A2[NS / 2], h2[NS / 2];
+#pragma unroll
+    for (int p = 0; p < NS / 2; ++p) {
+        A2[p] = make_float2(Aw[2 * p], Aw[2 * p + 1]);
+        h2[p] = make_float2(h[2 * p], h[2 * p + 1]);
+    }
     const float bias = (g.active && args.bias) ? args.bias[g.d] : 0.f;
     const float dskip = (g.active && args.Dskip) ? args.Dskip[g.d] : 0.f;
     double dsum = 0.0;
@@ -136,22 +154,57 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         __syncthreads();
         if (g.active) {
             const IO *su = st + g.ch, *sd = st + Lay::TILE + g.ch, *sz = st + 2 * Lay::TILE + g.ch;
-            int64_t off = (g.b * L + tc) * Dm + g.d;
-#pragma unroll 2
-            for (int r = 0; r < rows; ++r, off += Dm) {
-                const float uv = io::load_smem(su + r * CPB);
-                const float s = io::load_smem(sd + r * CPB) + bias;
-                const float dl = args.softplus ? softplus<PRECISE>(s) : s;
-                const float yl = lane_step<NS, PRECISE>(dl, dl * uv, fB + r * NSP + g.q * NS,
-                                                        fC + r * NSP + g.q * NS, Aw, h);
+            const int64_t off0 = (g.b * L + tc) * Dm + g.d;
+            // KSTEP steps at a time.  The G lanes of a channel split its states;
+            // the per-step scalar work (softplus, Delta u, skip, gate, store) of
+            // step r0 + j G + q is done once, by lane q, and Delta, Delta u and
+            // the partial readouts travel between the lanes by shuffles.  Rows
+            // past the end of the sequence were zero-filled by the copy and get
+            // Delta = 0 (decay 1, no input): the state passes through them.
+            for (int r0 = 0; r0 < rows; r0 += KSTEP) {
+                float uvo[KG], dlo[KG], duo[KG];
+#pragma unroll
+                for (int j = 0; j < KG; ++j) {
+                    const int r = r0 + j * G + g.q;
+                    uvo[j] = io::load_smem(su + r * CPB);
+                    dlo[j] = io::load_smem(sd + r * CPB) + bias;
+                }
+                if (args.softplus) {
+                    if (!PRECISE && KG % 2 == 0) {
+#pragma unroll
+                        for (int j = 0; j < KG; j += 2) {
+                            const float2 sp = softplus2_fast(make_float2(dlo[j], dlo[j + 1]));
+                            dlo[j] = sp.x;
+                            dlo[j + 1] = sp.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < KG; ++j) dlo[j] = softplus<PRECISE>(dlo[j]);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < KG; ++j) {
+                    if (r0 + j * G + g.q >= rows) dlo[j] = 0.f;
+                    duo[j] = dlo[j] * uvo[j];
+                }
+                float dl[KSTEP], du[KSTEP], y[KSTEP];
+                exchange_steps<KSTEP, G>(dlo, duo, dl, du);
+                recur_block<KSTEP, NS, PRECISE>(dl, du, fB + r0 * NSP + g.q * NS, fC + r0 * NSP + g.q * NS,
+                                                NSP, A2, h2, y);
                 if (MODE == kSegAgg) {
-                    dsum += (double)dl;
+#pragma unroll
+                    for (int j = 0; j < KG; ++j) dsum += (double)dlo[j];
                 } else {
-                    float y = group_sum<G>(yl);
-                    if (g.q == 0) {
-                        y = fmaf(dskip, uv, y);
-                        if (pz) y *= silu<PRECISE>(io::load_smem(sz + r * CPB));
-                        io::store(po + off, y);
+                    float yo[KG];
+                    reduce_scatter_steps<KSTEP, G>(y, yo, g.q);
+#pragma unroll
+                    for (int j = 0; j < KG; ++j) {
+                        const int r = r0 + j * G + g.q;
+                        if (r < rows) {
+                            float yy = fmaf(dskip, uvo[j], yo[j]);
+                            if (pz) yy *= silu<PRECISE>(io::load_smem(sz + r * CPB));
+                            io::store(po + off0 + (int64_t)r * Dm, yy);
+                        }
                     }
                 }
             }
@@ -159,6 +212,12 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         __syncthreads();  // stage c % S and the fp32 B/C buffers are free again
     }
     cp_async_wait<0>();
+    if (MODE == kSegAgg) dsum = group_sum_d<G>(dsum);
+#pragma unroll
+    for (int p = 0; p < NS / 2; ++p) {
+        h[2 * p] = h2[p].x;
+        h[2 * p + 1] = h2[p].y;
+    }
     lane_finish<NS, G, MODE>(args, g, seg, t_end, h, dsum);
 }
 

@@ -63,33 +63,47 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ------------------------------------------------------------------ softplus
 // softplus(s) = log(1 + e^s) = max(s, 0) + log1p(e), e = exp(-|s|) in (0, 1].
+//
+// Fast tier: e from the SFU, then log1p(e) = e * q(e) with q a degree-8
+// polynomial fitted to log1p(e)/e on [0, 1] (Lawson-weighted least squares on
+// 4000 Chebyshev nodes, relative error; q(0) = 1 exactly).  Evaluated in fp32
+// its relative error is below 1.6e-7 over the whole interval, so Delta keeps
+// full fp32-level relative accuracy even when it is ~1e-3 (the common case,
+// where an absolute-error logarithm would lose three digits).
+#define SSM_LOG1P_Q                                                                          \
+    {1.0f, -0.49999648332595825f, 0.3332132399082184f, -0.24857163429260254f,               \
+     0.1915365308523178f, -0.13753798604011536f, 0.0792044997215271f, -0.03006576932966709f, \
+     0.005364818498492241f}
+
+__device__ __forceinline__ float log1p_unit(float e) {  // e in [0, 1]
+    constexpr float q[9] = SSM_LOG1P_Q;
+    float p = q[8];
+#pragma unroll
+    for (int k = 7; k >= 0; --k) p = fmaf(p, e, q[k]);
+    return p * e;
+}
+
 template <bool PRECISE>
 __device__ __forceinline__ float softplus(float s) {
     if (PRECISE) return fmaxf(s, 0.f) + log1pf(expf(-fabsf(s)));
-    const float e = ex2_approx(-fabsf(s) * kLog2e);
-    // Small e: alternating Taylor series of log1p truncated after e^7; the
-    // remainder is below e^8 / 8, i.e. < 7e-8 relative for e < 1/8.
-    float p = 1.f / 7.f;
-    p = fmaf(p, e, -1.f / 6.f);
-    p = fmaf(p, e, 1.f / 5.f);
-    p = fmaf(p, e, -1.f / 4.f);
-    p = fmaf(p, e, 1.f / 3.f);
-    p = fmaf(p, e, -1.f / 2.f);
-    p = fmaf(p, e, 1.f);
-    const float series = p * e;
-    // Larger e: 1 + e >= 1.125, where the SFU logarithm's absolute error is
-    // small relative to the result.
-    const float direct = lg2_approx(1.f + e) * kLn2;
-    return fmaxf(s, 0.f) + (e < 0.125f ? series : direct);
+    return fmaxf(s, 0.f) + log1p_unit(ex2_approx(-fabsf(s) * kLog2e));
 }
 
 // -------------------------------------------------------------------- silu
+// Fast tier: silu(z) = z sigmoid(z) = h (1 + tanh(h)), h = z / 2 -- one SFU op.
 template <bool PRECISE>
 __device__ __forceinline__ float silu(float z) {
     if (PRECISE) return z / (1.f + expf(-z));
-    return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
+    const float hz = 0.5f * z;
+    return fmaf(hz, tanh_approx(hz), hz);
 }
 
 // Decay Abar = exp(Delta * A).  The fast tier takes A pre-multiplied by log2(e).
@@ -97,6 +111,41 @@ template <bool PRECISE>
 __device__ __forceinline__ float decay(float dl, float a_scaled) {
     if (PRECISE) return expf(dl * a_scaled);
     return ex2_approx(dl * a_scaled);
+}
+
+// The same, given the product x = Delta * A (times log2(e) in the fast tier).
+template <bool PRECISE>
+__device__ __forceinline__ float decay_of(float x) {
+    if (PRECISE) return expf(x);
+    return ex2_approx(x);
+}
+
+// ------------------------------------------------- packed fp32 pairs (f32x2)
+// One instruction operates on two fp32 lanes held in a register pair; each
+// lane is rounded exactly like the scalar instruction (round to nearest even).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n.reg .b64 ra, rb, rc, rd;\nmov.b64 ra, {%2,%3};\nmov.b64 rb, {%4,%5};\n"
+        "mov.b64 rc, {%6,%7};\nfma.rn.f32x2 rd, ra, rb, rc;\nmov.b64 {%0,%1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n.reg .b64 ra, rb, rd;\nmov.b64 ra, {%2,%3};\nmov.b64 rb, {%4,%5};\n"
+        "add.rn.f32x2 rd, ra, rb;\nmov.b64 {%0,%1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n.reg .b64 ra, rb, rd;\nmov.b64 ra, {%2,%3};\nmov.b64 rb, {%4,%5};\n"
+        "mul.rn.f32x2 rd, ra, rb;\nmov.b64 {%0,%1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
 }
 
 template <bool PRECISE>
@@ -114,6 +163,79 @@ __device__ __forceinline__ float group_sum(float v) {
         for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
     }
     return v;
+}
+
+// Fast-tier softplus of two values at once (log1p polynomial on fp32 pairs).
+__device__ __forceinline__ float2 softplus2_fast(float2 s) {
+    constexpr float q[9] = SSM_LOG1P_Q;
+    const float2 e = make_float2(ex2_approx(-fabsf(s.x) * kLog2e), ex2_approx(-fabsf(s.y) * kLog2e));
+    float2 p = make_float2(q[8], q[8]);
+#pragma unroll
+    for (int k = 7; k >= 0; --k) p = fma2(p, e, make_float2(q[k], q[k]));
+    return add2(make_float2(fmaxf(s.x, 0.f), fmaxf(s.y, 0.f)), mul2(p, e));
+}
+
+template <int G>
+__device__ __forceinline__ double group_sum_d(double v) {
+    if (G > 1) {
+        const unsigned lane = threadIdx.x & 31u;
+        const unsigned mask = ((1u << G) - 1u) << (lane & ~(unsigned)(G - 1));
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
+    }
+    return v;
+}
+
+// Lane q of a group of G consecutive lanes holds the scalars of steps
+// q, q + G, q + 2G, ... (own[j] is step j G + q); afterwards every lane of
+// the group holds all K steps.
+template <int K, int G>
+__device__ __forceinline__ void exchange_steps(const float (&dlo)[K / G], const float (&duo)[K / G],
+                                               float (&dl)[K], float (&du)[K]) {
+    if (G == 1) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) { dl[k] = dlo[k]; du[k] = duo[k]; }
+        return;
+    }
+    const unsigned lane = threadIdx.x & 31u;
+    const unsigned base = lane & ~(unsigned)(G - 1);
+    const unsigned mask = ((1u << G) - 1u) << base;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        dl[k] = __shfl_sync(mask, dlo[k / G], base + k % G);
+        du[k] = __shfl_sync(mask, duo[k / G], base + k % G);
+    }
+}
+
+// Each lane holds partial sums y[k] for K steps; afterwards lane q of the
+// group holds the full sums of its own steps, yo[j] = sum over the group of
+// y[j G + q] (a butterfly reduce-scatter: log2 G rounds, each halving the
+// steps a lane keeps).
+template <int K, int G>
+__device__ __forceinline__ void reduce_scatter_steps(const float (&y)[K], float (&yo)[K / G], int q) {
+    if (G == 1) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) yo[k] = y[k];
+        return;
+    }
+    const unsigned lane = threadIdx.x & 31u;
+    const unsigned mask = ((1u << G) - 1u) << (lane & ~(unsigned)(G - 1));
+#pragma unroll
+    for (int j = 0; j < K / G; ++j) {
+        if (G == 2) {
+            const float keep = q ? y[2 * j + 1] : y[2 * j];
+            const float send = q ? y[2 * j] : y[2 * j + 1];
+            yo[j] = keep + __shfl_xor_sync(mask, send, 1);
+        } else {  // G == 4
+            const bool hi = (q & 2) != 0;
+            const float k0 = hi ? y[4 * j + 2] : y[4 * j + 0], k1 = hi ? y[4 * j + 3] : y[4 * j + 1];
+            const float s0 = hi ? y[4 * j + 0] : y[4 * j + 2], s1 = hi ? y[4 * j + 1] : y[4 * j + 3];
+            const float m0 = k0 + __shfl_xor_sync(mask, s0, 2);
+            const float m1 = k1 + __shfl_xor_sync(mask, s1, 2);
+            const bool odd = (q & 1) != 0;
+            yo[j] = (odd ? m1 : m0) + __shfl_xor_sync(mask, odd ? m0 : m1, 1);
+        }
+    }
 }
 
 }  // namespace ssm
