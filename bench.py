@@ -213,8 +213,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
         dist.init_process_group("nccl", device_id=dev)
 
     cfg = WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank) if rank else WORKLOAD
-    if args.batch:
-        cfg = cfg.with_(batch=args.batch, name=f"{cfg.name}_batch{args.batch}")
+    if args.batch or args.seqlen:
+        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
+        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"mamba1p4b_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
     x = I.scan_inputs(cfg)
 
     def up(a):
@@ -357,6 +358,7 @@ def main() -> int:
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
+    ap.add_argument("--seqlen", type=int, default=0, help="override the workload's length (profiling cases)")
     ap.add_argument("--no-e2e", action="store_true", help="device-timed loop only (profiling cases)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
