@@ -81,6 +81,28 @@ def committed_traffic(sha: str):
     return d.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------ multi-GPU logic
+def rank_config(rank: int) -> I.ScanConfig:
+    """Each rank scans its own copy of the workload (independent batches: no
+    exchange on the data path); rank 0's is the single-GPU workload."""
+    return WORKLOAD if rank == 0 else WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a few timings over all ranks (one all-reduce)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, elements_per_rank: int, ms_per_step: float) -> float:
+    """Gelem/s of the whole job: every rank's elements over the slowest rank's time."""
+    return world * elements_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
@@ -212,7 +234,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
 
-    cfg = WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank) if rank else WORKLOAD
+    cfg = rank_config(rank)
     if args.batch or args.seqlen:
         b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
         cfg = cfg.with_(batch=b_, seqlen=l_, name=f"mamba1p4b_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
@@ -261,14 +283,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
         dist.barrier()
     elapsed_ms = e_all0.elapsed_time(e_all1)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    t = torch.tensor([elapsed_ms, statistics.mean(launch_ms)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, kernel_ms = float(t[0]), float(t[1])
+    elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, statistics.mean(launch_ms)], dev)
 
     if args.no_e2e:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": world * cfg.elements / (elapsed_ms / args.steps * 1e-3) / 1e9,
+            print(json.dumps({"metric": METRIC, "value": whole_job_rate(world, cfg.elements, elapsed_ms / args.steps),
                               "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": cfg.name},
                               "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
         if world > 1:
@@ -305,16 +324,14 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    t2 = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0] / e2e_steps
     if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(t2[0]) / e2e_steps
 
     if rank == 0:
         peaks = measured_peaks()
         ms_per_step = elapsed_ms / args.steps
-        value = world * cfg.elements / (ms_per_step * 1e-3) / 1e9
+        value = whole_job_rate(world, cfg.elements, ms_per_step)
         abytes = algorithmic_bytes(cfg)
         achieved_gbs = abytes / (kernel_ms * 1e-3) / 1e9
         sha = kernel_source_sha()
@@ -333,7 +350,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
                          "algorithmic_bytes_per_launch": abytes, "kernel_ms": kernel_ms,
                          "peak_source": peaks["source"] + " (copy bandwidth)",
                          "kernel_source_sha": sha},
-            "e2e": {"value": world * cfg.elements / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+            "e2e": {"value": whole_job_rate(world, cfg.elements, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": args.steps * plan["launches"],
             "clocks": clocks,
