@@ -132,6 +132,48 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io,
                                      void *out, float *last_state, const ssm_scan_opts *opts,
                                      ssm_stream stream);
 
+/*
+ * ssm_selective_scan_fwd for callers that cannot allocate device memory at
+ * call time.  (The paper has no counterpart: this is a deployment option.)
+ *
+ * Who needs it: a serving runtime that reserved nearly all of the GPU's memory
+ * for its own pool at start-up, so a cudaMallocAsync from the driver's pool
+ * would fail or fragment that reservation; a real-time or latency-budgeted
+ * path that may not take the allocator's locks; an embedding where all device
+ * memory is owned by the host application.  The only scratch the scan needs
+ * is the carry buffer of the sequence split, and this entry point takes it
+ * from a fixed static array inside the library instead of allocating.
+ *
+ * Same arguments and results as ssm_selective_scan_fwd, with the sequence
+ * split always requested: segments = the number of segments (0 = automatic,
+ * capped so the carries fit).  When the sequence is too short to split, one
+ * pass runs and no scratch is used.
+ *
+ * Limits and behaviour:
+ *  - The scratch holds SSM_NOALLOC_SCRATCH_BYTES (16 MiB).  A split needs
+ *    4 * batch * dim * (dstate * (segments + 1) + segments) bytes; a request
+ *    that does not fit returns SSM_ERR_UNSUPPORTED before anything is
+ *    enqueued.  Every GPU on which the library is loaded holds these 16 MiB
+ *    until the process exits.
+ *  - No cudaMalloc, cudaMallocAsync, cudaFree or allocating library routine is
+ *    called.  The first call on each device looks up the scratch's device
+ *    address (cudaGetSymbolAddress) with that device current; make that first
+ *    call before any stream capture.
+ *  - All calls share the one scratch array, which keeps the last call's
+ *    contents.  Nothing in it needs to start at zero (each call writes every
+ *    word it later reads), but calls whose GPU work overlaps in time -- on
+ *    different streams, or from different threads -- race on it: order them
+ *    on one stream or synchronise between them.
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io,
+                                          const void *u, const void *delta, const float *A,
+                                          const void *B, const void *C, const float *D,
+                                          const void *z, const float *delta_bias, int delta_softplus,
+                                          void *out, float *last_state, int segments,
+                                          ssm_stream stream);
+
 /* What a scan call with these arguments would do (nothing is launched or
  * allocated; data pointers are only inspected for alignment and may be
  * fake).  Lets a caller size the workspace and count kernel launches. */

@@ -21,8 +21,10 @@ VARIANTS = {"auto": 0, "slab": 1, "split": 2}
 FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
 
 # every symbol include/ssm.h declares
-EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_state_update",
-            "ssm_scan_plan", "ssm_status_string", "ssm_last_error", "ssm_version")
+EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
+            "ssm_selective_state_update", "ssm_scan_plan", "ssm_status_string", "ssm_last_error",
+            "ssm_version")
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class SSMDims(ctypes.Structure):
@@ -62,6 +64,8 @@ def _load() -> ctypes.CDLL:
     lib.ssm_selective_scan_fwd.restype = ctypes.c_int
     lib.ssm_selective_scan_fwd_ex.argtypes = scan_args + [ctypes.POINTER(SSMScanOpts), _vp]
     lib.ssm_selective_scan_fwd_ex.restype = ctypes.c_int
+    lib.ssm_selective_scan_fwd_noalloc.argtypes = scan_args + [ctypes.c_int, _vp]
+    lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_selective_state_update.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp]
     lib.ssm_selective_state_update.restype = ctypes.c_int
@@ -151,6 +155,32 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     else:
         opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
+    return out
+
+
+def selective_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                               delta_softplus=True, out=None, last_state=None, segments: int = 0,
+                               stream=None):
+    """The sequence-split scan without device allocation (carries live in the
+    library's static scratch; see ssm_selective_scan_fwd_noalloc in ssm.h).
+    ``out`` must be given by callers that cannot allocate (torch.empty_like
+    is used otherwise)."""
+    io = _io_of(u)
+    batch, seqlen, dim = u.shape
+    dstate = A.shape[1]
+    dev = u.device
+    if out is None:
+        out = torch.empty_like(u)
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate)
+    check(lib.ssm_selective_scan_fwd_noalloc(
+        SSMDims(batch, seqlen, dim, dstate), io,
+        _ptr(u, "u", u.dtype, seq, dev), _ptr(delta, "delta", u.dtype, seq, dev),
+        _ptr(A, "A", torch.float32, (dim, dstate), dev), _ptr(B, "B", u.dtype, bc, dev),
+        _ptr(C, "C", u.dtype, bc, dev), _ptr(D, "D", torch.float32, (dim,), dev),
+        _ptr(z, "z", u.dtype, seq, dev), _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev),
+        int(bool(delta_softplus)), _ptr(out, "out", u.dtype, seq, dev),
+        _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate), dev),
+        int(segments), _stream_handle(stream)))
     return out
 
 

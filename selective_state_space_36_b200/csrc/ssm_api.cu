@@ -2,6 +2,8 @@
 // choice of kernel variant and thread layout, launch, error reporting.
 #include <cuda_runtime.h>
 #include <stdarg.h>
+
+#include <mutex>
 #include <stdio.h>
 #include <string.h>
 
@@ -274,6 +276,110 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     cudaError_t ef = cudaFreeAsync(ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "split scan launch");
     if (ef != cudaSuccess) return cuda_fail(ef, "workspace release");
+    return SSM_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Sequence-split scan without any device allocation.
+//
+// The split scan needs a carry buffer (segment end states and Delta sums).
+// ssm_selective_scan_fwd takes it from cudaMallocAsync; this variant takes it
+// from the fixed scratch array below, which the CUDA runtime places in device
+// memory when the library's module is loaded on a GPU and keeps until the
+// process exits.  Host code must not pass the array's name to a kernel (on the
+// host it is only a shadow symbol): the device address is looked up once per
+// device with cudaGetSymbolAddress while that device is current.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)SSM_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+ssm_status noalloc_scratch_address(void **addr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SSM_ERR_UNSUPPORTED, "device index %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                          const float *A, const void *B, const void *C, const float *D,
+                                          const void *z, const float *delta_bias, int delta_softplus,
+                                          void *out, float *last_state, int segments, ssm_stream stream) {
+    g_last_error[0] = 0;
+    if (segments < 0) return fail(SSM_ERR_INVALID_ARG, "segments must be >= 0");
+    ssm_scan_opts o{};
+    o.variant = SSM_VARIANT_SPLIT;
+    o.segments = segments;
+    ScanPlan p;
+    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, delta_softplus, &o, &p)) return s;
+    if (p.launches == 0) return SSM_OK;  // empty problem
+    if (p.ws_bytes > kNoAllocScratchBytes && segments == 0) {
+        // automatic segment count: take the largest that fits the scratch
+        const size_t per_seg = ((size_t)dims.batch * dims.dim * (dims.dstate + 1)) * sizeof(float);
+        const size_t fixed = (size_t)dims.batch * dims.dim * dims.dstate * sizeof(float);
+        const size_t fit = kNoAllocScratchBytes > fixed ? (kNoAllocScratchBytes - fixed) / per_seg : 0;
+        if (fit >= 2) {
+            o.segments = (int)(fit > 65535 ? 65535 : fit);
+            if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, delta_softplus, &o, &p)) return s;
+        }
+    }
+    if (p.ws_bytes > kNoAllocScratchBytes)
+        return fail(SSM_ERR_UNSUPPORTED, "the split needs %zu bytes of scratch but the static scratch holds %zu "
+                    "(use fewer segments, a smaller batch * dim, or ssm_selective_scan_fwd)",
+                    p.ws_bytes, kNoAllocScratchBytes);
+    const size_t es = io == SSM_BF16 ? 2 : 4;
+    if (!u || !delta || !A || !B || !C || !out)
+        return fail(SSM_ERR_INVALID_ARG, "u, delta, A, B, C and out are required");
+    if (misaligned(u, es) || misaligned(delta, es) || misaligned(B, es) || misaligned(C, es) ||
+        misaligned(z, es) || misaligned(out, es) || misaligned(A, 4) || misaligned(D, 4) ||
+        misaligned(delta_bias, 4) || misaligned(last_state, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+
+    ssm::ScanArgs a{};
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.Dskip = D; a.bias = delta_bias;
+    a.out = out; a.last_state = last_state;
+    a.batch = dims.batch; a.seqlen = dims.seqlen; a.dim = dims.dim;
+    a.dstate = (int)dims.dstate;
+    a.softplus = delta_softplus;
+    a.seg_len = p.seg_len;
+    a.nseg = p.nseg;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (p.variant == SSM_VARIANT_SLAB) {  // too short to split: one pass, no scratch
+        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSlab, p.family, st);
+        if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+        return SSM_OK;
+    }
+    void *ws = nullptr;
+    if (ssm_status s = noalloc_scratch_address(&ws)) return s;
+    // Every scratch word the second pass reads is written by the first pass of
+    // the same call (the h0 copy, and the aggregates of segments 0..nseg-2), so
+    // nothing has to be cleared between calls.
+    const size_t n_h0 = (size_t)dims.batch * dims.dim * dims.dstate;
+    a.seg_h0 = static_cast<float *>(ws);
+    a.seg_h = a.seg_h0 + n_h0;
+    a.seg_dsum = a.seg_h + n_h0 * p.nseg;
+    cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSplit, p.family, st);
+    if (e != cudaSuccess) return cuda_fail(e, "split scan launch");
     return SSM_OK;
 }
 
