@@ -6,6 +6,13 @@ softplus(Delta), discretisation, recurrence, readout, D skip, silu(z) gate, the
 fp32 state in and out.  Inputs are seeded synthetic data of that shape.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload mamba1p4b|mamba130m|longseq|decode]
+
+The other workloads measure the remaining hot-path kernels the same way:
+mamba130m (batch 8, L 2048, dim 1536), longseq (batch 1, L 1,048,576, dim 1536:
+the sequence-split variant) and decode (one ssm_selective_state_update step at
+batch 256, dim 5120, N 16; two state buffers alternate so that the 84 MB state
+cannot simply stay in the 126 MB L2).
 
 Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of
 the workload on its GPU (independent batches, no collective on the data path:
@@ -37,6 +44,35 @@ METRIC = "selective-scan fwd Gelem/s (B·L·D) at 1.4B-layer shape; % of HBM roo
 UNIT = "Gelem/s"
 WORKLOAD = I.MAMBA1P4B
 L2_BYTES = 126 * 1024 * 1024
+WORKLOADS = {"mamba1p4b": I.MAMBA1P4B, "mamba130m": I.MAMBA130M, "longseq": I.LONGSEQ,
+             "decode": I.DECODE}
+SCAN_METRICS = {
+    "mamba1p4b": METRIC,
+    "mamba130m": "selective-scan fwd Gelem/s (B·L·D) at 130M-layer shape; % of HBM roofline",
+    "longseq": "selective-scan fwd Gelem/s (B·L·D) at L=1,048,576 (sequence split); % of HBM roofline",
+}
+DECODE_METRIC = "decode state-update steps/s at batch 256, dim 5120, N 16; % of HBM roofline"
+
+
+def alu_ceiling_per_sm_clock(dstate: int = 16) -> float:
+    """Elements per SM clock that the arithmetic of the scan allows on B200.
+
+    Model built from measured unit costs (probes/pipe_rates.cu): an SFU op
+    (ex2, tanh) occupies ~4 issue cycles of its SM sub-partition and its unit
+    for 8 cycles per warp; an f32x2 op 1 issue cycle.  Per element the method
+    needs dstate decays exp(Delta A_n), 2 SFU ops for softplus and silu, 2
+    packed FP32 issue cycles per state (Delta A, Delta u B, state FMA, readout
+    FMA) and ~14 more issue cycles (softplus polynomial, gate, loads, stores).
+    A decay costs 4 issue cycles on the SFU or ~4.5 as an FMA-pipe polynomial;
+    the best split of the decays between the two balances the SFU unit
+    against the issue slots.  Four sub-partitions x 32 lanes per SM clock.
+    """
+    best = 0.0
+    for m in range(dstate + 1):            # decays on the SFU
+        sfu_cycles = 8.0 * (m + 2)
+        issue_cycles = 4.0 * (m + 2) + 4.5 * (dstate - m) + 2.0 * dstate + 14.0
+        best = max(best, 128.0 / max(sfu_cycles, issue_cycles))
+    return best
 
 
 def algorithmic_bytes(cfg: I.ScanConfig) -> int:
@@ -56,15 +92,24 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
+SCAN_KERNEL_SOURCES = ("scan_fwd_staged.cu", "scan_common.cuh", "scan_kernels.cuh", "ssm_device.cuh")
+
+
 def kernel_source_sha() -> str:
-    """Hash of the CUDA sources: a committed ncu traffic figure is valid only
-    for the kernels it was captured on."""
+    """Hash of the staged scan kernel's sources with comments and blank space
+    removed: a committed ncu traffic figure is valid only for the code it was
+    captured on."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_36_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in SCAN_KERNEL_SOURCES:
+        if True:
+            with open(os.path.join(csrc, f)) as fh:
+                code = fh.read()
+            code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+            code = re.sub(r"//[^\n]*", "", code)
+            code = re.sub(r"\s+", " ", code)
+            h.update(f.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 
@@ -153,24 +198,27 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_rate(cfg: I.ScanConfig, budget_s: float, max_rows=None):
-    """The fp64 oracle, as it stands, on whole batch rows of the workload until
-    ``budget_s`` of CPU time has been spent (at least one row).  Returns
+def oracle_rate(cfg: I.ScanConfig, budget_s: float):
+    """The fp64 oracle, as it stands, on blocks of the workload (one batch row,
+    every channel, 2048 consecutive steps each) until ``budget_s`` seconds have
+    been spent (at least one block) or the workload is done.  Returns
     (Gelem/s, threads, elements, seconds)."""
     import oracle
-    A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip)
-    one = cfg.with_(batch=1)
-    done, spent, rows = 0, 0.0, 0
+    A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip, cfg.dt_min, cfg.dt_max)
+    A, D, bias = A.astype(np.float64), D.astype(np.float64), bias.astype(np.float64)
     threads = min(oracle.default_threads(), cfg.dim)
-    while (spent < budget_s or rows == 0) and rows < (max_rows or cfg.batch):
-        x = {k: I.to_f64(I.draw_rows(cfg, k, rows % cfg.batch, 0, cfg.seqlen), cfg.io)[None]
-             for k in I.SEQ_NAMES}
-        t0 = time.perf_counter()
-        oracle.scan(x["u"], x["delta"], A.astype(np.float64), x["B"], x["C"], D=D.astype(np.float64),
-                    z=x["z"], delta_bias=bias.astype(np.float64), delta_softplus=True)
-        spent += time.perf_counter() - t0
-        done += one.seqlen * one.dim
-        rows += 1
+    blocks = [(b, t0, t1) for b in range(cfg.batch) for t0, t1 in I.iter_time_blocks(cfg.seqlen, 2048)]
+    done, spent = 0, 0.0
+    state = {}
+    for b, t0, t1 in blocks:
+        if spent >= budget_s and done:
+            break
+        x = {k: I.to_f64(I.draw_rows(cfg, k, b, t0, t1), cfg.io)[None] for k in I.SEQ_NAMES}
+        t_start = time.perf_counter()
+        _, state[b] = oracle.scan(x["u"], x["delta"], A, x["B"], x["C"], D=D, z=x["z"], delta_bias=bias,
+                                  delta_softplus=True, h0=state.get(b))
+        spent += time.perf_counter() - t_start
+        done += (t1 - t0) * cfg.dim
     return done / spent / 1e9, threads, done, spent
 
 
@@ -224,146 +272,274 @@ def run_reference(args, rank: int) -> int:
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rank: int, world: int, local_rank: int) -> int:
+def _upload(a, dev):
+    import torch
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def _scan_device_inputs(cfg: I.ScanConfig, dev):
+    """Device copies of a scan workload's inputs.  Long sequences are drawn and
+    copied block by block so that the host never holds them whole."""
+    import torch
+    A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip, cfg.dt_min, cfg.dt_max)
+    dt = torch.bfloat16 if cfg.io == "bf16" else torch.float32
+    d = {}
+    for k in I.SEQ_NAMES:
+        w = cfg.dstate if k in ("B", "C") else cfg.dim
+        d[k] = torch.empty((cfg.batch, cfg.seqlen, w), dtype=dt, device=dev)
+        for b in range(cfg.batch):
+            for t0, t1 in I.iter_time_blocks(cfg.seqlen, 1 << 16):
+                d[k][b, t0:t1].copy_(_upload(I.draw_rows(cfg, k, b, t0, t1), dev))
+    d.update(A=_upload(A, dev), D=_upload(D, dev), delta_bias=_upload(bias, dev))
+    return d
+
+
+def _time_steps(step, steps, warmup, stream, dev, world, sample_clocks=True):
+    """Warm-up, then K steps bracketed by barrier + synchronize, CUDA events on
+    the launching stream around the region and around each step; max over ranks."""
     import torch
     import torch.distributed as dist
-    from selective_state_space_36_b200 import binding as lib
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
-
-    cfg = rank_config(rank)
-    if args.batch or args.seqlen:
-        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
-        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"mamba1p4b_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
-    x = I.scan_inputs(cfg)
-
-    def up(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(a).to(dev)
-
-    d = {k: up(v) for k, v in x.items() if isinstance(v, np.ndarray)}
-    state0 = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
-    state = state0.clone()
-    out = torch.empty_like(d["u"])
-    stream = torch.cuda.current_stream(dev)
-    plan = lib.scan_plan(cfg.batch, cfg.seqlen, cfg.dim, cfg.dstate, cfg.io)
-
-    # Each step scans one batch of the workload and resumes from the state the
-    # previous step left in last_state (a continued sequence): same work.
-    def step():
-        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
-
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
-
-    sampler = ClockSampler(local_rank)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index or 0)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
-    e_all0, e_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_all0.record(stream)
-    for i in range(args.steps):
+    if sample_clocks:
+        sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
         ev[i][0].record(stream)
-        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+        step()
         ev[i][1].record(stream)
-    e_all1.record(stream)
+    e1.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    elapsed_ms = e_all0.elapsed_time(e_all1)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, statistics.mean(launch_ms)], dev)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    elapsed_ms, launch_ms = max_over_ranks([e0.elapsed_time(e1), launch_ms], dev)
+    return elapsed_ms, launch_ms, clocks
 
-    if args.no_e2e:
-        if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": whole_job_rate(world, cfg.elements, elapsed_ms / args.steps),
-                              "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": cfg.name},
-                              "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
-        return 0
 
-    # end to end through the public call with host buffers: pinned host inputs
-    # copied in, the scan, the output and final state copied back, every step
-    host = {k: v.cpu().pin_memory() for k, v in d.items()}
-    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    host_state = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
-    host_state0 = torch.zeros(state.shape, dtype=state.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values()) + state0.numel() * 4
-    d2h = host_out.numel() * host_out.element_size() + host_state.numel() * 4
-    e2e_steps = max(3, min(args.steps, 20))
-
-    def e2e_step():
-        for k in d:
-            d[k].copy_(host[k], non_blocking=True)
-        state.copy_(host_state0, non_blocking=True)
-        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
-        host_out.copy_(out, non_blocking=True)
-        host_state.copy_(state, non_blocking=True)
-
+def _e2e(step_with_copies, steps, stream, dev, world):
+    import torch
+    import torch.distributed as dist
     for _ in range(2):
-        e2e_step()
+        step_with_copies()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    for _ in range(steps):
+        step_with_copies()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0] / e2e_steps
+    ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0] / steps
     if world > 1:
         dist.barrier()
+    return ms
+
+
+def _base_line(metric, unit, value, world, args, ms_per_step, higher=True):
+    return {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": higher,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic"}
+
+
+def run_scan(args, rank, world, dev):
+    import torch
+    from selective_state_space_36_b200 import binding as lib
+
+    cfg = WORKLOADS[args.workload]
+    if rank:
+        cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
+    if args.batch or args.seqlen:
+        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
+        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"{args.workload}_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
+    d = _scan_device_inputs(cfg, dev)
+    state = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
+    out = torch.empty_like(d["u"])
+    stream = torch.cuda.current_stream(dev)
+    plan = lib.scan_plan(cfg.batch, cfg.seqlen, cfg.dim, cfg.dstate, cfg.io)
+
+    # Each step scans one batch of the workload and resumes from the state the
+    # previous step left in last_state (a continued sequence): the same work.
+    def step():
+        lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                               delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+
+    elapsed_ms, kernel_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
+    ms_per_step = elapsed_ms / args.steps
+    metric = SCAN_METRICS.get(args.workload, METRIC)
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"metric": metric, "value": whole_job_rate(world, cfg.elements, ms_per_step),
+                              "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": cfg.name},
+                              "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
+        return 0
+
+    e2e = None
+    if cfg.elements <= 1 << 28:
+        # end to end through the public call with host buffers: pinned host
+        # inputs copied in, the scan, the output and the final state copied
+        # back, every step
+        host = {k: v.cpu().pin_memory() for k, v in d.items()}
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        host_state = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
+        host_state0 = torch.zeros(state.shape, dtype=state.dtype, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for v in host.values()) + host_state0.numel() * 4
+        d2h = host_out.numel() * host_out.element_size() + host_state.numel() * 4
+        e2e_steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            for k in d:
+                d[k].copy_(host[k], non_blocking=True)
+            state.copy_(host_state0, non_blocking=True)
+            lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                   delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+            host_out.copy_(out, non_blocking=True)
+            host_state.copy_(state, non_blocking=True)
+
+        e2e_ms = _e2e(e2e_step, e2e_steps, stream, dev, world)
+        e2e = {"value": whole_job_rate(world, cfg.elements, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     if rank == 0:
         peaks = measured_peaks()
-        ms_per_step = elapsed_ms / args.steps
-        value = whole_job_rate(world, cfg.elements, ms_per_step)
         abytes = algorithmic_bytes(cfg)
         achieved_gbs = abytes / (kernel_ms * 1e-3) / 1e9
+        sm_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        alu_peak = alu_ceiling_per_sm_clock(cfg.dstate) * sms * sm_mhz * 1e6 / 1e9
+        kernel_gelem = cfg.elements / (kernel_ms * 1e-3) / 1e9
         sha = kernel_source_sha()
-        traffic = committed_traffic(sha)
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        line = _base_line(metric, UNIT, whole_job_rate(world, cfg.elements, ms_per_step), world, args,
+                          ms_per_step)
+        line.update({
             "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "dim": cfg.dim,
                        "dstate": cfg.dstate, "io": cfg.io, "per_gpu": "one full workload per GPU",
                        "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": f"inputs {abytes / 1e6:.0f} MB > {L2_BYTES >> 20} MB L2; no flush",
                        "plan": plan},
-            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                         "algorithmic_bytes_per_launch": abytes, "kernel_ms": kernel_ms,
-                         "peak_source": peaks["source"] + " (copy bandwidth)",
-                         "kernel_source_sha": sha},
-            "e2e": {"value": whole_job_rate(world, cfg.elements, e2e_ms), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "roofline": {
+                "bound": "alu", "achieved": kernel_gelem, "peak": alu_peak, "unit": "Gelem/s",
+                "frac": kernel_gelem / alu_peak,
+                "peak_source": (f"derived: {alu_ceiling_per_sm_clock(cfg.dstate):.3f} elem/clk/SM x {sms} SMs x "
+                                f"{sm_mhz:.0f} MHz (measured SFU/FMA issue costs)"),
+                "traffic": committed_traffic(sha) if args.workload == "mamba1p4b" and plan["launches"] == 1 else None,
+                "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": abytes,
+                "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved_gbs / peaks["hbm_gbs"],
+                        "peak_source": peaks["source"] + " (copy bandwidth)"},
+                "kernel_source_sha": sha},
+            "e2e": e2e,
             "gpu_launches": args.steps * plan["launches"],
             "clocks": clocks,
-        }
+        })
         if world == 1 and not args.no_cpu_baseline:
             v, threads, el, secs = oracle_rate(cfg, budget_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"{el // (cfg.seqlen * cfg.dim)} of {cfg.batch} batch rows "
-                                              f"({el} elements, {secs:.1f} s)"}
+                                    "sample": f"{el} elements of {cfg.name} in blocks of whole channels "
+                                              f"x 2048 steps ({secs:.1f} s)"}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
     return 0
+
+
+def run_decode(args, rank, world, dev):
+    import torch
+    from selective_state_space_36_b200 import binding as lib
+
+    cfg = I.DECODE if rank == 0 else I.DecodeConfig(**{**I.DECODE.__dict__, "seed": I.DECODE.seed + 1000 * rank})
+    A, D, bias = I.decode_params(cfg)
+    st = I.decode_step_inputs(cfg, 0, bias)
+    d = {k: _upload(v, dev) for k, v in st.items()}
+    Ad, Dd = _upload(A, dev), _upload(D, dev)
+    h0 = I.decode_h0(cfg)
+    states = [_upload(h0, dev), _upload(h0, dev)]  # 2 x 84 MB > L2: alternate them
+    out = torch.empty_like(d["x"])
+    stream = torch.cuda.current_stream(dev)
+    k = [0]
+
+    def step():
+        lib.selective_state_update(states[k[0] & 1], d["x"], d["dt"], Ad, d["B"], d["C"], D=Dd, z=d["z"],
+                                   out=out, stream=stream)
+        k[0] += 1
+
+    elapsed_ms, kernel_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
+    ms_per_step = elapsed_ms / args.steps
+    channels = cfg.batch * cfg.dim
+    es = 2
+    abytes = channels * (cfg.dstate * 4 * 2 + 4 * es) + cfg.batch * cfg.dstate * es * 2 + cfg.dim * cfg.dstate * 4
+    host = {kk: v.cpu().pin_memory() for kk, v in d.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for kk in d:
+            d[kk].copy_(host[kk], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+
+    e2e_ms = _e2e(e2e_step, max(3, min(args.steps, 50)), stream, dev, world)
+    if rank == 0:
+        peaks = measured_peaks()
+        achieved = abytes / (kernel_ms * 1e-3) / 1e9
+        line = _base_line(DECODE_METRIC, "steps/s", world * 1e3 / ms_per_step, world, args, ms_per_step)
+        line.update({
+            "config": {"workload": cfg.name, "batch": cfg.batch, "dim": cfg.dim, "dstate": cfg.dstate,
+                       "io": cfg.io, "per_gpu": "one full decode batch per GPU",
+                       "l2": "two 84 MB state buffers alternate (168 MB > 126 MB L2)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel_ms": kernel_ms,
+                         "algorithmic_bytes_per_launch": abytes,
+                         "peak_source": peaks["source"] + " (copy bandwidth)"},
+            "e2e": {"value": world * 1e3 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        })
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            h = h0.astype(np.float64)
+            spent, n = 0.0, 0
+            while spent < args.cpu_budget and n < 50:
+                s_in = I.decode_step_inputs(cfg, n, bias)
+                f = lambda a: I.to_f64(a, cfg.io)
+                t0 = time.perf_counter()
+                _, h = oracle.state_update(h, f(s_in["x"]), f(s_in["dt"]), A, f(s_in["B"]), f(s_in["C"]),
+                                           D=D, z=f(s_in["z"]))
+                spent += time.perf_counter() - t0
+                n += 1
+            line["cpu_baseline"] = {"value": n / spent, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{n} full decode steps ({spent:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> int:
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    try:
+        if args.workload == "decode":
+            return run_decode(args, rank, world, dev)
+        return run_scan(args, rank, world, dev)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
 
 
 def main() -> int:
@@ -377,6 +553,7 @@ def main() -> int:
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seqlen", type=int, default=0, help="override the workload's length (profiling cases)")
     ap.add_argument("--no-e2e", action="store_true", help="device-timed loop only (profiling cases)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mamba1p4b")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -7,8 +7,8 @@
 //     y = sum_n C_n h_n + D u;  out = y * silu(z)
 // with the fp32 state held in registers for the whole sequence, so the
 // expanded (batch, L, dim, N) state is never materialised (the notes'
-// "hardware-aware algorithm": load parameters once, discretise and recur
-// on-chip, write only the outputs).
+// hardware-aware algorithm: parameters are read from HBM once, discretisation
+// and recurrence happen on chip, and only the outputs go back to HBM).
 //
 // Thread layout: a group of G consecutive lanes owns one channel; lane q of
 // the group holds states [q*NS, q*NS + NS).  A block of 128 threads covers
@@ -25,8 +25,9 @@
 //            Delta sum (so that the segment's decay product is exp(A * sum)).
 //  kSegFinal second pass: the carry into segment s is the left fold of
 //            (P_s', h_loc_s') over s' < s with the associative operator
-//            (a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2)  (the notes' "work-efficient
-//            parallel scan"); then the segment is re-scanned with readout.
+//            (a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2), the associative operator
+//            behind the parallel scan the notes cite; then the segment is
+//            re-scanned with readout.
 #include "scan_common.cuh"
 
 namespace ssm {

@@ -6,8 +6,8 @@
 // shared memory: each chunk of T time steps of the block's u, delta, z tiles
 // ([T x channels-per-block]) and of B, C ([T x N]) is brought in with 16-byte
 // cp.async copies, STAGES chunks ahead, so global-memory latency overlaps the
-// recurrence of earlier chunks (the notes' "load from HBM to SRAM, compute on
-// chip, write only the output").  B and C are widened to fp32 once per chunk
+// recurrence of earlier chunks (the notes' hardware-aware algorithm: inputs go
+// from HBM to on-chip memory once and only the outputs are written back).  B and C are widened to fp32 once per chunk
 // and per block, then read by every channel with broadcast 128-bit loads.
 //
 // The waits are cp.async.wait_group (hardware-tracked completion of this
