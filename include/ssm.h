@@ -110,7 +110,7 @@ typedef enum {
     SSM_KERNEL_GENERIC = 1,  /* direct global loads; any size and element alignment */
     SSM_KERNEL_STAGED = 2    /* inputs staged through shared memory with 16-byte async
                                 copies; needs dim and dstate rows of a multiple of 16
-                                bytes and 16-byte aligned u, delta, z, B, C
+                                bytes and 16-byte aligned u, delta, z, B, C, out
                                 (SSM_ERR_UNSUPPORTED otherwise) */
 } ssm_kernel_family;
 
@@ -120,7 +120,9 @@ typedef struct {
     int32_t lanes;    /* lanes sharing one channel: 0 = automatic, else 1, 2 or 4
                          (honoured for 9 <= dstate <= 32) */
     int32_t family;   /* ssm_kernel_family */
-    int32_t reserved[4]; /* must be zero */
+    int32_t channels_per_lane; /* staged kernel: 0 = automatic, 1, or 2 (one B/C load serves two
+                                  adjacent channels) */
+    int32_t reserved[3]; /* must be zero */
 } ssm_scan_opts;
 
 /* ssm_selective_scan_fwd with explicit execution choices (opts may be NULL).
@@ -183,13 +185,13 @@ typedef struct {
     int32_t lanes;           /* lanes per channel */
     int32_t family;          /* ssm_kernel_family chosen: GENERIC or STAGED */
     int32_t launches;        /* kernels the call enqueues (0 for an empty problem) */
-    int32_t reserved0;
+    int32_t channels_per_lane;
     int64_t workspace_bytes; /* device scratch the call allocates (SPLIT), else 0 */
 } ssm_scan_plan_info;
 
 ssm_status ssm_scan_plan(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
-                         const void *B, const void *C, const void *z, const ssm_scan_opts *opts,
-                         ssm_scan_plan_info *info);
+                         const void *B, const void *C, const void *z, const void *out,
+                         const ssm_scan_opts *opts, ssm_scan_plan_info *info);
 
 /*
  * One recurrent (decode) step for every channel: constant time and memory per

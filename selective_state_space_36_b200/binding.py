@@ -35,13 +35,13 @@ class SSMDims(ctypes.Structure):
 class SSMScanOpts(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
                 ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("channels_per_lane", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 class SSMScanPlanInfo(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
                 ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
-                ("launches", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("channels_per_lane", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_int64)]
 
 
@@ -69,7 +69,7 @@ def _load() -> ctypes.CDLL:
     lib.ssm_selective_state_update.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp]
     lib.ssm_selective_state_update.restype = ctypes.c_int
-    lib.ssm_scan_plan.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+    lib.ssm_scan_plan.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                   ctypes.POINTER(SSMScanOpts), ctypes.POINTER(SSMScanPlanInfo)]
     lib.ssm_scan_plan.restype = ctypes.c_int
     lib.ssm_status_string.argtypes = [ctypes.c_int]
@@ -125,7 +125,7 @@ def _stream_handle(stream) -> Optional[int]:
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                        out=None, last_state=None, variant: str = "auto", segments: int = 0,
-                       lanes: int = 0, family: str = "auto", stream=None):
+                       lanes: int = 0, family: str = "auto", cpl: int = 0, stream=None):
     """Selective scan forward on CUDA tensors; returns ``out``.
 
     u, delta, z: (batch, seqlen, dim); B, C: (batch, seqlen, dstate) -- all
@@ -150,10 +150,10 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
         _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate), dev),
     ]
     dims = SSMDims(batch, seqlen, dim, dstate)
-    if variant == "auto" and not segments and not lanes and family == "auto":
+    if variant == "auto" and not segments and not lanes and family == "auto" and not cpl:
         check(lib.ssm_selective_scan_fwd(dims, io, *args, _stream_handle(stream)))
     else:
-        opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
+        opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family], int(cpl))
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
     return out
 
@@ -186,18 +186,19 @@ def selective_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=Non
 
 def scan_plan(batch: int, seqlen: int, dim: int, dstate: int, io: str = "bf16",
               variant: str = "auto", segments: int = 0, lanes: int = 0, family: str = "auto",
-              aligned: bool = True) -> dict:
+              cpl: int = 0, aligned: bool = True) -> dict:
     """What ssm_selective_scan_fwd would do for this shape (no GPU work).
     ``aligned`` describes the data pointers (16-byte aligned or not)."""
     base = 0x100000 if aligned else 0x100002
-    opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family])
+    opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family], int(cpl))
     info = SSMScanPlanInfo()
     check(lib.ssm_scan_plan(SSMDims(batch, seqlen, dim, dstate), SSM_BF16 if io == "bf16" else SSM_F32,
-                            base, base, base, base, base, ctypes.byref(opts), ctypes.byref(info)))
+                            base, base, base, base, base, base, ctypes.byref(opts), ctypes.byref(info)))
     inv_v = {v: k for k, v in VARIANTS.items()}
     inv_f = {v: k for k, v in FAMILIES.items()}
     return {"variant": inv_v.get(info.variant, "none"), "segments": info.segments, "lanes": info.lanes,
             "family": inv_f.get(info.family, "none"), "launches": info.launches,
+            "channels_per_lane": info.channels_per_lane,
             "workspace_bytes": info.workspace_bytes}
 
 

@@ -25,9 +25,21 @@ struct LaneGeom {
     }
 };
 
+// One lane's share of one channel: batch row b, channel d, state slice q.
+struct LaneRef {
+    int64_t b, d;
+    int q;
+    bool active;
+};
+
+template <int G>
+__device__ __forceinline__ LaneRef lane_ref(const LaneGeom<G> &g) {
+    return LaneRef{g.b, g.d, g.q, g.active};
+}
+
 // A (pre-scaled for the decay tier) and the initial state of this lane.
-template <int NS, int G, bool PRECISE, int MODE>
-__device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneGeom<G> &g, int seg,
+template <int NS, bool PRECISE, int MODE>
+__device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneRef &g, int seg,
                                           float (&Aw)[NS], float (&h)[NS]) {
     const int N = a.dstate;
 #pragma unroll
@@ -79,8 +91,8 @@ __device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneGeom<G> &
 }
 
 // Final state (one pass, or the last segment) or the segment aggregate.
-template <int NS, int G, int MODE>
-__device__ __forceinline__ void lane_finish(const ScanArgs &a, const LaneGeom<G> &g, int seg,
+template <int NS, int MODE>
+__device__ __forceinline__ void lane_finish(const ScanArgs &a, const LaneRef &g, int seg,
                                             int64_t t_end, const float (&h)[NS], double dsum) {
     if (!g.active) return;
     const int N = a.dstate;
@@ -166,6 +178,84 @@ __device__ __forceinline__ void recur_block(const float (&dl)[K], const float (&
             }
         }
         y[k] = acc.x + acc.y;
+    }
+}
+
+// The same for a lane that holds NS states of each of CPL channels: step k's
+// B and C values are read once and used for every channel.
+template <int K, int NS, int CPL, bool PRECISE>
+__device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const float (&du)[K][CPL],
+                                                const float *Bs, const float *Cs, int stride,
+                                                const float2 (&A2)[CPL][NS / 2],
+                                                float2 (&h2)[CPL][NS / 2], float (&y)[K][CPL]) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        float2 d2[CPL], u2[CPL], acc[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            d2[c] = make_float2(dl[k][c], dl[k][c]);
+            u2[c] = make_float2(du[k][c], du[k][c]);
+            acc[c] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < NS / 4; ++j) {
+            const float4 bv = *reinterpret_cast<const float4 *>(Bs + k * stride + 4 * j);
+            const float4 cv = *reinterpret_cast<const float4 *>(Cs + k * stride + 4 * j);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                const int p = 2 * j + hlf;
+                const float2 b2 = hlf ? make_float2(bv.z, bv.w) : make_float2(bv.x, bv.y);
+                const float2 c2 = hlf ? make_float2(cv.z, cv.w) : make_float2(cv.x, cv.y);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    if (!PRECISE) {
+                        const float2 x2 = mul2(d2[c], A2[c][p]);
+                        const float2 a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
+                        h2[c][p] = fma2(a2, h2[c][p], mul2(u2[c], b2));
+                        acc[c] = fma2(c2, h2[c][p], acc[c]);
+                    } else {
+                        const float ax = decay_of<PRECISE>(d2[c].x * A2[c][p].x);
+                        const float ay = decay_of<PRECISE>(d2[c].y * A2[c][p].y);
+                        h2[c][p].x = fmaf(ax, h2[c][p].x, u2[c].x * b2.x);
+                        h2[c][p].y = fmaf(ay, h2[c][p].y, u2[c].y * b2.y);
+                        acc[c].x = fmaf(c2.x, h2[c][p].x, acc[c].x);
+                        acc[c].y = fmaf(c2.y, h2[c][p].y, acc[c].y);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) y[k][c] = acc[c].x + acc[c].y;
+    }
+}
+
+// exchange_steps / reduce_scatter_steps for CPL channels per lane.
+template <int K, int G, int CPL>
+__device__ __forceinline__ void exchange_steps_cpl(const float (&dlo)[K / G][CPL],
+                                                   const float (&duo)[K / G][CPL],
+                                                   float (&dl)[K][CPL], float (&du)[K][CPL]) {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        float a[K / G], bo[K / G], x[K], z[K];
+#pragma unroll
+        for (int j = 0; j < K / G; ++j) { a[j] = dlo[j][c]; bo[j] = duo[j][c]; }
+        exchange_steps<K, G>(a, bo, x, z);
+#pragma unroll
+        for (int k = 0; k < K; ++k) { dl[k][c] = x[k]; du[k][c] = z[k]; }
+    }
+}
+
+template <int K, int G, int CPL>
+__device__ __forceinline__ void reduce_scatter_steps_cpl(const float (&y)[K][CPL], float (&yo)[K / G][CPL],
+                                                         int q) {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        float a[K], o[K / G];
+#pragma unroll
+        for (int k = 0; k < K; ++k) a[k] = y[k][c];
+        reduce_scatter_steps<K, G>(a, o, q);
+#pragma unroll
+        for (int j = 0; j < K / G; ++j) yo[j][c] = o[j];
     }
 }
 

@@ -49,7 +49,7 @@ scan_fwd_kernel(const ScanArgs args) {
     const int64_t t_end = t_begin + args.seg_len < L ? t_begin + args.seg_len : L;
 
     float Aw[NS], h[NS];
-    lane_init<NS, G, PRECISE, MODE>(args, g, seg, Aw, h);
+    lane_init<NS, PRECISE, MODE>(args, lane_ref(g), seg, Aw, h);
     const float bias = (g.active && args.bias) ? args.bias[g.d] : 0.f;
     const float dskip = (g.active && args.Dskip) ? args.Dskip[g.d] : 0.f;
 
@@ -96,7 +96,7 @@ scan_fwd_kernel(const ScanArgs args) {
             }
         }
     }
-    lane_finish<NS, G, MODE>(args, g, seg, t_end, h, dsum);
+    lane_finish<NS, MODE>(args, lane_ref(g), seg, t_end, h, dsum);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -105,7 +105,7 @@ scan_fwd_kernel(const ScanArgs args) {
 bool staged_eligible(const ScanArgs &a, int es) {
     auto al = [](const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) % 16) == 0; };
     return (a.dim * es) % 16 == 0 && (a.dstate * es) % 16 == 0 && al(a.u) && al(a.delta) &&
-           al(a.z) && al(a.B) && al(a.C);
+           al(a.z) && al(a.B) && al(a.C) && al(a.out);
 }
 template <typename IO, int NS, int G>
 static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
@@ -140,11 +140,11 @@ static cudaError_t launch_io(const ScanArgs &a, int ns, int g, int variant, cuda
     return cudaErrorInvalidConfiguration;
 }
 
-cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int variant, int family,
-                            cudaStream_t st) {
+cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
+                            int family, cudaStream_t st) {
     const bool eligible = staged_eligible(a, bf16 ? 2 : 4);
     if (family == kFamilyStaged && !eligible) return cudaErrorInvalidValue;
-    if (family != kFamilyGeneric && eligible) return launch_scan_staged(a, bf16, ns, g, variant, st);
+    if (family != kFamilyGeneric && eligible) return launch_scan_staged(a, bf16, ns, g, cpl, variant, st);
     return bf16 ? launch_io<__nv_bfloat16>(a, ns, g, variant, st)
                 : launch_io<float>(a, ns, g, variant, st);
 }

@@ -1,20 +1,30 @@
 // scan_fwd_staged.cu -- selective-scan forward, staged variant (sm_100a).
 //
-// Same arithmetic and thread layout as the generic kernel in scan_fwd.cu
-// (NL-345 Mamba translation, section 2 eq. (2); 【論文要約】Mamba notes, S6
-// Algorithm 2, 数式解説 3), but every input reaches the compute loop through
-// shared memory: each chunk of T time steps of the block's u, delta, z tiles
+// Same arithmetic as the generic kernel in scan_fwd.cu (NL-345 Mamba
+// translation, section 2 eq. (2); 【論文要約】Mamba notes, S6 Algorithm 2,
+// 数式解説 3), but every input reaches the compute loop through shared memory:
+// each chunk of T time steps of the block's u, delta, z tiles
 // ([T x channels-per-block]) and of B, C ([T x N]) is brought in with 16-byte
 // cp.async copies, STAGES chunks ahead, so global-memory latency overlaps the
 // recurrence of earlier chunks (the notes' hardware-aware algorithm: inputs go
-// from HBM to on-chip memory once and only the outputs are written back).  B and C are widened to fp32 once per chunk
-// and per block, then read by every channel with broadcast 128-bit loads.
+// from HBM to on-chip memory once and only the outputs are written back).  B
+// and C are widened to fp32 once per chunk and per block.
+//
+// Thread layout: G lanes share a group of CPL adjacent channels; lane q holds
+// states [q NS, q NS + NS) of each of them.  B_t and C_t are read once per lane
+// and step and serve all CPL channels, so the shared-memory traffic of the
+// broadcast operands (the largest) falls by a factor CPL, and u, delta, z and
+// out move CPL channels per access (one channel per lane is the default: at
+// the benchmark shapes halving the warps costs more than the traffic saved).
+// Tile rows are padded by 32 bytes so that the G rows the lanes of a group
+// read at once fall in different banks.
 //
 // The waits are cp.async.wait_group (hardware-tracked completion of this
 // thread's own copies) followed by a block barrier: there is no polling loop.
 //
 // Eligibility (checked on the host): dim * sizeof(io) and dstate * sizeof(io)
-// are multiples of 16 bytes and u, delta, z, B, C start on 16-byte boundaries.
+// are multiples of 16 bytes and u, delta, z, B, C, out start on 16-byte
+// boundaries.
 #include <atomic>
 
 #include "scan_common.cuh"
@@ -24,17 +34,28 @@ namespace ssm {
 #ifndef SSM_KSTEP
 #define SSM_KSTEP 4
 #endif
-// Time steps processed together: a multiple of 2G (so each lane owns an even
-// number of them) that divides the chunk.
-template <int G>
+// Time steps processed together: a multiple of G that divides the chunk, and
+// with one channel per lane a multiple of 2G, so the per-step scalar work of a
+// lane comes in pairs for the packed softplus.
+template <int G, int CPL>
 struct KStep {
-    static constexpr int value = SSM_KSTEP > 2 * G ? SSM_KSTEP : 2 * G;
+    static constexpr int need = CPL == 2 ? G : 2 * G;
+    static constexpr int value = SSM_KSTEP > need ? SSM_KSTEP : need;
 };
 
+// Two stages: one chunk computes while the next one lands.  A third stage
+// costs enough shared memory to drop a resident block per SM at the 4-lane
+// layout, which at the 1.4B-layer shape turns one wave of blocks into two.
+#ifndef SSM_STAGES
+#define SSM_STAGES 2
+#endif
+#ifndef SSM_CHUNK_BF16
+#define SSM_CHUNK_BF16 32
+#endif
 template <typename IO>
 struct StagedCfg {
-    static constexpr int T = sizeof(IO) == 2 ? 32 : 16;  // time steps per chunk
-    static constexpr int STAGES = 3;
+    static constexpr int T = sizeof(IO) == 2 ? SSM_CHUNK_BF16 : 16;  // time steps per chunk
+    static constexpr int STAGES = SSM_STAGES;
 };
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool full) {
@@ -48,41 +69,84 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-template <typename IO, int NS, int G>
+// Row padding: with G > 1 the lanes of a group read G different rows at once,
+// and 32 bytes of padding put those rows in different banks; with G = 1 all
+// lanes read one row and padding would only cost shared memory.
+#ifndef SSM_ROW_PAD_BYTES
+#define SSM_ROW_PAD_BYTES 32
+#endif
+
+template <typename IO, int NS, int G, int CPL>
 struct StagedLayout {
     static constexpr int T = StagedCfg<IO>::T;
     static constexpr int S = StagedCfg<IO>::STAGES;
-    static constexpr int CPB = kBlock / G;
-    static constexpr int NSP = NS * G;
-    static constexpr int TILE = T * CPB;  // elements of one u/delta/z tile
-    static constexpr int RAW = T * NSP;   // elements reserved for one raw B or C tile
-    static constexpr size_t STAGE_BYTES = (3 * TILE + 2 * RAW) * sizeof(IO);
+    static constexpr int GROUPS = kBlock / G;                 // channel groups per block
+    static constexpr int CPB = GROUPS * CPL;                  // channels per block
+    static constexpr int NSP = NS * G;                        // padded states per channel
+    static constexpr int ROW = CPB + (G > 1 ? SSM_ROW_PAD_BYTES / (int)sizeof(IO) : 0);  // tile row (elements)
+    static constexpr int TILE = T * ROW;                      // elements of one u/delta/z tile
+    static constexpr int RAW = T * NSP;                       // elements reserved for one raw B or C tile
+    static constexpr size_t STAGE_BYTES = (3 * (size_t)TILE + 2 * RAW) * sizeof(IO);
     static constexpr size_t BC_BYTES = 2 * (size_t)T * NSP * sizeof(float);
     static constexpr size_t SMEM = S * STAGE_BYTES + BC_BYTES;
 };
 
-template <typename IO, int NS, int G, bool PRECISE, int MODE>
+// CPL consecutive values from shared memory / to global memory.
+template <typename IO, int CPL>
+__device__ __forceinline__ void load_vals(const IO *p, float (&v)[CPL]) {
+    if (CPL == 2 && sizeof(IO) == 2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+        v[0] = __uint_as_float(w << 16);
+        v[CPL - 1] = __uint_as_float(w & 0xffff0000u);
+    } else if (CPL == 2) {
+        const float2 w = *reinterpret_cast<const float2 *>(p);
+        v[0] = w.x;
+        v[CPL - 1] = w.y;
+    } else {
+        v[0] = io_traits<IO>::load_smem(p);
+    }
+}
+
+template <typename IO, int CPL>
+__device__ __forceinline__ void store_vals(IO *p, const float (&v)[CPL]) {
+    if (CPL == 2 && sizeof(IO) == 2) {
+        const __nv_bfloat162 w = __floats2bfloat162_rn(v[0], v[CPL - 1]);
+        __stcs(reinterpret_cast<unsigned int *>(p), *reinterpret_cast<const unsigned int *>(&w));
+    } else if (CPL == 2) {
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(v[0], v[CPL - 1]));
+    } else {
+        io_traits<IO>::store(p, v[0]);
+    }
+}
+
+template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE>
 __global__ void __launch_bounds__(kBlock)
 scan_fwd_staged_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
-    using Lay = StagedLayout<IO, NS, G>;
-    constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP;
+    using Lay = StagedLayout<IO, NS, G, CPL>;
+    constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP, ROW = Lay::ROW;
     constexpr int EPV = 16 / sizeof(IO);  // elements per 16-byte piece
     constexpr int ROWV = CPB / EPV;       // pieces per tile row
-    constexpr int KSTEP = KStep<G>::value;
+    constexpr int KSTEP = KStep<G, CPL>::value;
     constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
+    static_assert(T % KSTEP == 0, "a chunk holds whole step blocks");
     extern __shared__ __align__(16) unsigned char smem[];
     float *fB = reinterpret_cast<float *>(smem + S * Lay::STAGE_BYTES);
     float *fC = fB + T * NSP;
 
-    const LaneGeom<G> g(args);
     const int64_t L = args.seqlen, Dm = args.dim;
     const int N = args.dstate;
     const int tid = threadIdx.x;
+    const int q = tid % G;
+    const int grp = tid / G;
+    const int64_t tiles = (Dm + CPB - 1) / CPB;
+    const int64_t b = blockIdx.x / tiles;
+    const int64_t d0 = (blockIdx.x % tiles) * CPB;
+    const int64_t dfirst = d0 + (int64_t)grp * CPL;  // first channel of this group
+    const bool active = dfirst < Dm;                  // dim is a multiple of CPL here
     const int seg = blockIdx.y;
     const int64_t t_begin = (int64_t)seg * args.seg_len;
     const int64_t t_end = t_begin + args.seg_len < L ? t_begin + args.seg_len : L;
-    const int64_t d0 = (blockIdx.x % ((Dm + CPB - 1) / CPB)) * CPB;
 
     const IO *pu = static_cast<const IO *>(args.u);
     const IO *pd = static_cast<const IO *>(args.delta);
@@ -105,31 +169,38 @@ scan_fwd_staged_kernel(const ScanArgs args) {
             const int r = p / ROWV, v = p % ROWV;
             const int64_t col = d0 + v * EPV;
             const bool ok = r < rows && col < Dm;
-            const int64_t go = ok ? (g.b * L + tc + r) * Dm + col : 0;
-            const int so = r * CPB + v * EPV;
+            const int64_t go = ok ? (b * L + tc + r) * Dm + col : 0;
+            const int so = r * ROW + v * EPV;
             cp_async16(su + so, pu + go, ok);
             cp_async16(sd + so, pd + go, ok);
             if (pz) cp_async16(sz + so, pz + go, ok);
         }
         const int pieces = rows * N / EPV;  // B/C rows of this chunk are contiguous
-        const int64_t gbc = (g.b * L + tc) * N;
+        const int64_t gbc = (b * L + tc) * N;
         for (int p = tid; p < pieces; p += kBlock) {
             cp_async16(rb + p * EPV, pB + gbc + p * EPV, true);
             cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
         }
     };
 
-    float Aw[NS], h[NS];
-    lane_init<NS, G, PRECISE, MODE>(args, g, seg, Aw, h);
-    float2 A2[NS / 2], h2[NS / 2];
+    // per-channel constants and state
+    float2 A2[CPL][NS / 2], h2[CPL][NS / 2];
+    float bias[CPL], dskip[CPL];
+    double dsum[CPL];
 #pragma unroll
-    for (int p = 0; p < NS / 2; ++p) {
-        A2[p] = make_float2(Aw[2 * p], Aw[2 * p + 1]);
-        h2[p] = make_float2(h[2 * p], h[2 * p + 1]);
+    for (int c = 0; c < CPL; ++c) {
+        const LaneRef lr{b, dfirst + c, q, active};
+        float Aw[NS], h[NS];
+        lane_init<NS, PRECISE, MODE>(args, lr, seg, Aw, h);
+#pragma unroll
+        for (int p = 0; p < NS / 2; ++p) {
+            A2[c][p] = make_float2(Aw[2 * p], Aw[2 * p + 1]);
+            h2[c][p] = make_float2(h[2 * p], h[2 * p + 1]);
+        }
+        bias[c] = (active && args.bias) ? args.bias[dfirst + c] : 0.f;
+        dskip[c] = (active && args.Dskip) ? args.Dskip[dfirst + c] : 0.f;
+        dsum[c] = 0.0;
     }
-    const float bias = (g.active && args.bias) ? args.bias[g.d] : 0.f;
-    const float dskip = (g.active && args.Dskip) ? args.Dskip[g.d] : 0.f;
-    double dsum = 0.0;
 
 #pragma unroll
     for (int c = 0; c < S - 1; ++c) {
@@ -152,58 +223,82 @@ scan_fwd_staged_kernel(const ScanArgs args) {
             fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
         }
         __syncthreads();
-        if (g.active) {
-            const IO *su = st + g.ch, *sd = st + Lay::TILE + g.ch, *sz = st + 2 * Lay::TILE + g.ch;
-            const int64_t off0 = (g.b * L + tc) * Dm + g.d;
-            // KSTEP steps at a time.  The G lanes of a channel split its states;
-            // the per-step scalar work (softplus, Delta u, skip, gate, store) of
-            // step r0 + j G + q is done once, by lane q, and Delta, Delta u and
-            // the partial readouts travel between the lanes by shuffles.  Rows
-            // past the end of the sequence were zero-filled by the copy and get
+        if (active) {
+            const int col = grp * CPL;
+            const IO *su = st + col, *sd = st + Lay::TILE + col, *sz = st + 2 * Lay::TILE + col;
+            const int64_t off0 = (b * L + tc) * Dm + dfirst;
+            // KSTEP steps at a time.  The per-step scalar work (softplus,
+            // Delta u, skip, gate, store) of step r0 + j G + q is done once, by
+            // lane q, for the group's CPL channels; Delta, Delta u and the
+            // partial readouts travel between the lanes by shuffles.  Rows past
+            // the end of the sequence were zero-filled by the copy and get
             // Delta = 0 (decay 1, no input): the state passes through them.
             for (int r0 = 0; r0 < rows; r0 += KSTEP) {
-                float uvo[KG], dlo[KG], duo[KG];
+                float uvo[KG][CPL], dlo[KG][CPL], duo[KG][CPL];
 #pragma unroll
                 for (int j = 0; j < KG; ++j) {
-                    const int r = r0 + j * G + g.q;
-                    uvo[j] = io::load_smem(su + r * CPB);
-                    dlo[j] = io::load_smem(sd + r * CPB) + bias;
+                    const int r = r0 + j * G + q;
+                    load_vals<IO, CPL>(su + r * ROW, uvo[j]);
+                    load_vals<IO, CPL>(sd + r * ROW, dlo[j]);
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) dlo[j][cc] += bias[cc];
                 }
                 if (args.softplus) {
-                    if (!PRECISE && KG % 2 == 0) {
+                    if (!PRECISE && CPL == 2) {
+#pragma unroll
+                        for (int j = 0; j < KG; ++j) {
+                            const float2 sp = softplus2_fast(make_float2(dlo[j][0], dlo[j][CPL - 1]));
+                            dlo[j][0] = sp.x;
+                            dlo[j][CPL - 1] = sp.y;
+                        }
+                    } else if (!PRECISE && KG % 2 == 0) {
 #pragma unroll
                         for (int j = 0; j < KG; j += 2) {
-                            const float2 sp = softplus2_fast(make_float2(dlo[j], dlo[j + 1]));
-                            dlo[j] = sp.x;
-                            dlo[j + 1] = sp.y;
+                            const float2 sp = softplus2_fast(make_float2(dlo[j][0], dlo[j + 1][0]));
+                            dlo[j][0] = sp.x;
+                            dlo[j + 1][0] = sp.y;
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < KG; ++j) dlo[j] = softplus<PRECISE>(dlo[j]);
+                        for (int j = 0; j < KG; ++j)
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) dlo[j][cc] = softplus<PRECISE>(dlo[j][cc]);
                     }
                 }
 #pragma unroll
                 for (int j = 0; j < KG; ++j) {
-                    if (r0 + j * G + g.q >= rows) dlo[j] = 0.f;
-                    duo[j] = dlo[j] * uvo[j];
+                    const bool ok = r0 + j * G + q < rows;
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) {
+                        if (!ok) dlo[j][cc] = 0.f;
+                        duo[j][cc] = dlo[j][cc] * uvo[j][cc];
+                    }
                 }
-                float dl[KSTEP], du[KSTEP], y[KSTEP];
-                exchange_steps<KSTEP, G>(dlo, duo, dl, du);
-                recur_block<KSTEP, NS, PRECISE>(dl, du, fB + r0 * NSP + g.q * NS, fC + r0 * NSP + g.q * NS,
-                                                NSP, A2, h2, y);
+                float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
+                exchange_steps_cpl<KSTEP, G, CPL>(dlo, duo, dl, du);
+                recur_block_cpl<KSTEP, NS, CPL, PRECISE>(dl, du, fB + r0 * NSP + q * NS,
+                                                         fC + r0 * NSP + q * NS, NSP, A2, h2, y);
                 if (MODE == kSegAgg) {
 #pragma unroll
-                    for (int j = 0; j < KG; ++j) dsum += (double)dlo[j];
+                    for (int j = 0; j < KG; ++j)
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) dsum[cc] += (double)dlo[j][cc];
                 } else {
-                    float yo[KG];
-                    reduce_scatter_steps<KSTEP, G>(y, yo, g.q);
+                    float yo[KG][CPL];
+                    reduce_scatter_steps_cpl<KSTEP, G, CPL>(y, yo, q);
 #pragma unroll
                     for (int j = 0; j < KG; ++j) {
-                        const int r = r0 + j * G + g.q;
+                        const int r = r0 + j * G + q;
                         if (r < rows) {
-                            float yy = fmaf(dskip, uvo[j], yo[j]);
-                            if (pz) yy *= silu<PRECISE>(io::load_smem(sz + r * CPB));
-                            io::store(po + off0 + (int64_t)r * Dm, yy);
+                            float yy[CPL], zz[CPL];
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) yy[cc] = fmaf(dskip[cc], uvo[j][cc], yo[j][cc]);
+                            if (pz) {
+                                load_vals<IO, CPL>(sz + r * ROW, zz);
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) yy[cc] *= silu<PRECISE>(zz[cc]);
+                            }
+                            store_vals<IO, CPL>(po + off0 + (int64_t)r * Dm, yy);
                         }
                     }
                 }
@@ -212,20 +307,24 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         __syncthreads();  // stage c % S and the fp32 B/C buffers are free again
     }
     cp_async_wait<0>();
-    if (MODE == kSegAgg) dsum = group_sum_d<G>(dsum);
 #pragma unroll
-    for (int p = 0; p < NS / 2; ++p) {
-        h[2 * p] = h2[p].x;
-        h[2 * p + 1] = h2[p].y;
+    for (int c = 0; c < CPL; ++c) {
+        const double ds = MODE == kSegAgg ? group_sum_d<G>(dsum[c]) : 0.0;
+        float h[NS];
+#pragma unroll
+        for (int p = 0; p < NS / 2; ++p) {
+            h[2 * p] = h2[c][p].x;
+            h[2 * p + 1] = h2[c][p].y;
+        }
+        lane_finish<NS, MODE>(args, LaneRef{b, dfirst + c, q, active}, seg, t_end, h, ds);
     }
-    lane_finish<NS, G, MODE>(args, g, seg, t_end, h, dsum);
 }
 
-template <typename IO, int NS, int G, int MODE>
+template <typename IO, int NS, int G, int CPL, int MODE>
 static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
     constexpr bool P = std::is_same<IO, float>::value;
-    using Lay = StagedLayout<IO, NS, G>;
-    auto kern = scan_fwd_staged_kernel<IO, NS, G, P, MODE>;
+    using Lay = StagedLayout<IO, NS, G, CPL>;
+    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE>;
     // the shared-memory opt-in is a per-device function attribute: set it once per device
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -234,38 +333,64 @@ static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_relaxed) & bit)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return e;
+        }
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
     kern<<<grid, kBlock, Lay::SMEM, st>>>(a);
     return cudaGetLastError();
 }
 
-template <typename IO, int NS, int G>
+template <typename IO, int NS, int G, int CPL>
 static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
-    constexpr int CPB = kBlock / G;
+    constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
     const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
-    if (variant == kVariantSlab) return launch_mode<IO, NS, G, kFull>(a, dim3(bx, 1), st);
-    cudaError_t e = launch_mode<IO, NS, G, kSegAgg>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
+    if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull>(a, dim3(bx, 1), st);
+    cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
     if (e != cudaSuccess) return e;
-    return launch_mode<IO, NS, G, kSegFinal>(a, dim3(bx, (unsigned)a.nseg), st);
+    return launch_mode<IO, NS, G, CPL, kSegFinal>(a, dim3(bx, (unsigned)a.nseg), st);
 }
 
-template <typename IO>
-static cudaError_t launch_io(const ScanArgs &a, int ns, int g, int variant, cudaStream_t st) {
-    if (ns == 4 && g == 1) return launch_t<IO, 4, 1>(a, variant, st);
-    if (ns == 8 && g == 1) return launch_t<IO, 8, 1>(a, variant, st);
-    if (ns == 16 && g == 1) return launch_t<IO, 16, 1>(a, variant, st);
-    if (ns == 8 && g == 2) return launch_t<IO, 8, 2>(a, variant, st);
-    if (ns == 4 && g == 4) return launch_t<IO, 4, 4>(a, variant, st);
-    if (ns == 16 && g == 2) return launch_t<IO, 16, 2>(a, variant, st);
-    if (ns == 8 && g == 4) return launch_t<IO, 8, 4>(a, variant, st);
-    if (ns == 16 && g == 4) return launch_t<IO, 16, 4>(a, variant, st);
+template <typename IO, int CPL>
+static cudaError_t launch_cpl(const ScanArgs &a, int ns, int g, int variant, cudaStream_t st) {
+    if (ns == 4 && g == 1) return launch_t<IO, 4, 1, CPL>(a, variant, st);
+    if (ns == 8 && g == 1) return launch_t<IO, 8, 1, CPL>(a, variant, st);
+    if (ns == 16 && g == 1) return launch_t<IO, 16, 1, CPL>(a, variant, st);
+    if (ns == 8 && g == 2) return launch_t<IO, 8, 2, CPL>(a, variant, st);
+    if (ns == 4 && g == 4) return launch_t<IO, 4, 4, CPL>(a, variant, st);
+    if (ns == 16 && g == 2) return launch_t<IO, 16, 2, CPL>(a, variant, st);
+    if (ns == 8 && g == 4) return launch_t<IO, 8, 4, CPL>(a, variant, st);
+    if (ns == 16 && g == 4) return launch_t<IO, 16, 4, CPL>(a, variant, st);
     return cudaErrorInvalidConfiguration;
 }
 
-cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int variant, cudaStream_t st) {
-    return bf16 ? launch_io<__nv_bfloat16>(a, ns, g, variant, st) : launch_io<float>(a, ns, g, variant, st);
+template <typename IO, int CPL>
+static size_t smem_of(int ns, int g) {
+    if (ns == 4 && g == 1) return StagedLayout<IO, 4, 1, CPL>::SMEM;
+    if (ns == 8 && g == 1) return StagedLayout<IO, 8, 1, CPL>::SMEM;
+    if (ns == 16 && g == 1) return StagedLayout<IO, 16, 1, CPL>::SMEM;
+    if (ns == 8 && g == 2) return StagedLayout<IO, 8, 2, CPL>::SMEM;
+    if (ns == 4 && g == 4) return StagedLayout<IO, 4, 4, CPL>::SMEM;
+    if (ns == 16 && g == 2) return StagedLayout<IO, 16, 2, CPL>::SMEM;
+    if (ns == 8 && g == 4) return StagedLayout<IO, 8, 4, CPL>::SMEM;
+    if (ns == 16 && g == 4) return StagedLayout<IO, 16, 4, CPL>::SMEM;
+    return ~(size_t)0;
+}
+
+size_t staged_smem_bytes(bool bf16, int ns, int g, int cpl) {
+    if (cpl == 2) return bf16 ? smem_of<__nv_bfloat16, 2>(ns, g) : smem_of<float, 2>(ns, g);
+    return bf16 ? smem_of<__nv_bfloat16, 1>(ns, g) : smem_of<float, 1>(ns, g);
+}
+
+cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
+                               cudaStream_t st) {
+    if (cpl == 2)
+        return bf16 ? launch_cpl<__nv_bfloat16, 2>(a, ns, g, variant, st)
+                    : launch_cpl<float, 2>(a, ns, g, variant, st);
+    return bf16 ? launch_cpl<__nv_bfloat16, 1>(a, ns, g, variant, st)
+                : launch_cpl<float, 1>(a, ns, g, variant, st);
 }
 
 }  // namespace ssm

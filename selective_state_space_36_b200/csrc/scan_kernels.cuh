@@ -44,11 +44,12 @@ struct DecodeArgs {
     int dstate;
 };
 
-cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int variant, int family,
-                            cudaStream_t st);
-cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int variant,
+cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
+                            int family, cudaStream_t st);
+cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
                                cudaStream_t st);
 bool staged_eligible(const ScanArgs &a, int es);
+size_t staged_smem_bytes(bool bf16, int ns, int g, int cpl);
 bool scan_shape_supported(int ns, int g);
 cudaError_t launch_state_update(const DecodeArgs &a, bool bf16, int ns, int g, cudaStream_t st);
 

@@ -23,6 +23,9 @@ ssm_status fail(ssm_status s, const char *fmt, ...) {
 }
 
 ssm_status cuda_fail(cudaError_t e, const char *what) {
+    // The CUDA runtime is shared with the caller (torch, for instance): leave
+    // no error of ours behind for its next status check to trip over.
+    (void)cudaGetLastError();
     return fail(SSM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
@@ -34,8 +37,15 @@ constexpr int64_t kMaxGridX = 2147483647LL;
 // 128-thread blocks per SM the sequence split aims for.
 constexpr int kTargetBlocksPerSm = 8;
 
+// Channels per lane of the staged kernel when the caller does not choose.
+#ifndef SSM_DEFAULT_CPL
+#define SSM_DEFAULT_CPL 1
+#endif
+constexpr int kDefaultStagedCpl = SSM_DEFAULT_CPL;
+
 struct DeviceInfo {
     int sms = 148;
+    int smem_optin = 227 * 1024;  // dynamic shared memory a block may opt in to
 };
 
 DeviceInfo device_info() {
@@ -45,7 +55,10 @@ DeviceInfo device_info() {
         int v = 0;
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
             di.sms = v;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && v > 0)
+            di.smem_optin = v;
     }
+    (void)cudaGetLastError();  // no device here is not an error of the caller's
     return di;
 }
 
@@ -106,7 +119,7 @@ namespace {
 // Everything a scan call decides before launching.
 struct ScanPlan {
     int variant = SSM_VARIANT_SLAB;
-    int ns = 16, g = 1;
+    int ns = 16, g = 1, cpl = 1;
     int family = ssm::kFamilyGeneric;
     int nseg = 1;
     int64_t seg_len = 0;
@@ -117,8 +130,8 @@ struct ScanPlan {
 // Validates sizes and options (not data pointers, which may be absent when
 // only planning) and decides variant, layout, kernel family and segments.
 ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *delta, const void *B,
-                     const void *C, const void *z, int delta_softplus, const ssm_scan_opts *opts,
-                     ScanPlan *plan) {
+                     const void *C, const void *z, const void *out, int delta_softplus,
+                     const ssm_scan_opts *opts, ScanPlan *plan) {
     size_t es = 0;
     if (ssm_status s = check_io(io, &es)) return s;
     if (dims.batch < 0 || dims.seqlen < 0 || dims.dim < 0 || dims.dstate < 0)
@@ -135,8 +148,11 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
         return fail(SSM_ERR_INVALID_ARG, "unknown variant %d", variant);
     const int lanes_req = opts ? opts->lanes : 0;
     int family = opts ? opts->family : 0;
-    if (opts && (opts->reserved[0] || opts->reserved[1] || opts->reserved[2] || opts->reserved[3]))
+    const int cpl_req = opts ? opts->channels_per_lane : 0;
+    if (opts && (opts->reserved[0] || opts->reserved[1] || opts->reserved[2]))
         return fail(SSM_ERR_INVALID_ARG, "ssm_scan_opts.reserved must be zero");
+    if (cpl_req != 0 && cpl_req != 1 && cpl_req != 2)
+        return fail(SSM_ERR_INVALID_ARG, "channels per lane must be 0, 1 or 2");
     if (family < ssm::kFamilyAuto || family > ssm::kFamilyStaged)
         return fail(SSM_ERR_INVALID_ARG, "kernel family must be 0 (auto), 1 (generic) or 2 (staged)");
     if (lanes_req != 0 && lanes_req != 1 && lanes_req != 2 && lanes_req != 4)
@@ -156,15 +172,23 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
     if (!ssm::scan_shape_supported(plan->ns, plan->g))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for %d states x %d lanes", plan->ns, plan->g);
     ssm::ScanArgs probe{};
-    probe.u = u; probe.delta = delta; probe.z = z; probe.B = B; probe.C = C;
+    probe.u = u; probe.delta = delta; probe.z = z; probe.B = B; probe.C = C; probe.out = const_cast<void *>(out);
     probe.dim = dims.dim; probe.dstate = (int)dims.dstate;
     const bool eligible = ssm::staged_eligible(probe, (int)es);
     if (family == ssm::kFamilyStaged && !eligible)
         return fail(SSM_ERR_UNSUPPORTED, "staged kernel needs 16-byte aligned rows (dim and dstate "
-                    "multiples of %d, 16-byte aligned u, delta, z, B, C)", (int)(16 / es));
-    if (family == ssm::kFamilyAuto) family = eligible ? ssm::kFamilyStaged : ssm::kFamilyGeneric;
+                    "multiples of %d, 16-byte aligned u, delta, z, B, C, out)", (int)(16 / es));
+    const int cpl_try = cpl_req ? cpl_req : kDefaultStagedCpl;
+    const bool fits = ssm::staged_smem_bytes(io == SSM_BF16, plan->ns, plan->g, cpl_try) <= (size_t)di.smem_optin;
+    if (family == ssm::kFamilyStaged && !fits)
+        return fail(SSM_ERR_UNSUPPORTED, "the staged kernel's shared memory for %d lanes x %d channels "
+                    "exceeds the device's %d bytes", plan->g, cpl_try, di.smem_optin);
+    if (family == ssm::kFamilyAuto) family = (eligible && fits) ? ssm::kFamilyStaged : ssm::kFamilyGeneric;
     plan->family = family;
-    const int64_t cpb = ssm::kBlock / plan->g;
+    if (cpl_req == 2 && family != ssm::kFamilyStaged)
+        return fail(SSM_ERR_UNSUPPORTED, "two channels per lane needs the staged kernel");
+    plan->cpl = family == ssm::kFamilyStaged ? cpl_try : 1;
+    const int64_t cpb = ssm::kBlock / plan->g * plan->cpl;
     const int64_t blocks = dims.batch * ((dims.dim + cpb - 1) / cpb);
     if (blocks > kMaxGridX) return fail(SSM_ERR_UNSUPPORTED, "grid too large");
 
@@ -174,7 +198,7 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
     const int64_t full = (int64_t)di.sms * kTargetBlocksPerSm;
     int64_t blocks_now = blocks;
     if (variant == SSM_VARIANT_AUTO) {
-        const int64_t blocks1 = dims.batch * ((dims.dim + ssm::kBlock - 1) / ssm::kBlock);
+        const int64_t blocks1 = dims.batch * ((dims.dim + ssm::kBlock * plan->cpl - 1) / (ssm::kBlock * plan->cpl));
         variant = (blocks1 < di.sms && dims.seqlen >= 4 * 1024) ? SSM_VARIANT_SPLIT : SSM_VARIANT_SLAB;
         // segments, not extra lanes per channel, supply the parallelism of a split
         if (variant == SSM_VARIANT_SPLIT && lanes_req == 0 && dims.dstate > 8 && dims.dstate <= 16) {
@@ -216,18 +240,19 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
 extern "C" {
 
 ssm_status ssm_scan_plan(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
-                         const void *B, const void *C, const void *z, const ssm_scan_opts *opts,
-                         ssm_scan_plan_info *info) {
+                         const void *B, const void *C, const void *z, const void *out,
+                         const ssm_scan_opts *opts, ssm_scan_plan_info *info) {
     g_last_error[0] = 0;
     if (!info) return fail(SSM_ERR_INVALID_ARG, "info is required");
     ScanPlan p;
-    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, 0, opts, &p)) return s;
+    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, 0, opts, &p)) return s;
     memset(info, 0, sizeof(*info));
     info->variant = p.variant;
     info->segments = p.nseg;
     info->lanes = p.g;
     info->family = p.family;
     info->launches = p.launches;
+    info->channels_per_lane = p.cpl;
     info->workspace_bytes = (int64_t)p.ws_bytes;
     return SSM_OK;
 }
@@ -239,7 +264,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
                                      ssm_stream stream) {
     g_last_error[0] = 0;
     ScanPlan p;
-    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, delta_softplus, opts, &p)) return s;
+    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, opts, &p)) return s;
     if (p.launches == 0) return SSM_OK;  // empty problem
     const size_t es = io == SSM_BF16 ? 2 : 4;
     if (!u || !delta || !A || !B || !C || !out)
@@ -261,7 +286,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     if (p.variant == SSM_VARIANT_SLAB) {
-        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSlab, p.family, st);
+        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, p.cpl, ssm::kVariantSlab, p.family, st);
         if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
         return SSM_OK;
     }
@@ -272,7 +297,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     a.seg_h0 = static_cast<float *>(ws);
     a.seg_h = a.seg_h0 + n_h0;
     a.seg_dsum = a.seg_h + n_h0 * p.nseg;
-    e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSplit, p.family, st);
+    e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, p.cpl, ssm::kVariantSplit, p.family, st);
     cudaError_t ef = cudaFreeAsync(ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "split scan launch");
     if (ef != cudaSuccess) return cuda_fail(ef, "workspace release");
@@ -330,7 +355,7 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
     o.variant = SSM_VARIANT_SPLIT;
     o.segments = segments;
     ScanPlan p;
-    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, delta_softplus, &o, &p)) return s;
+    if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &p)) return s;
     if (p.launches == 0) return SSM_OK;  // empty problem
     if (p.ws_bytes > kNoAllocScratchBytes && segments == 0) {
         // automatic segment count: take the largest that fits the scratch
@@ -339,7 +364,7 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
         const size_t fit = kNoAllocScratchBytes > fixed ? (kNoAllocScratchBytes - fixed) / per_seg : 0;
         if (fit >= 2) {
             o.segments = (int)(fit > 65535 ? 65535 : fit);
-            if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, delta_softplus, &o, &p)) return s;
+            if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &p)) return s;
         }
     }
     if (p.ws_bytes > kNoAllocScratchBytes)
@@ -365,7 +390,7 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
     a.nseg = p.nseg;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (p.variant == SSM_VARIANT_SLAB) {  // too short to split: one pass, no scratch
-        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSlab, p.family, st);
+        cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, p.cpl, ssm::kVariantSlab, p.family, st);
         if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
         return SSM_OK;
     }
@@ -378,7 +403,7 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
     a.seg_h0 = static_cast<float *>(ws);
     a.seg_h = a.seg_h0 + n_h0;
     a.seg_dsum = a.seg_h + n_h0 * p.nseg;
-    cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, ssm::kVariantSplit, p.family, st);
+    cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, p.cpl, ssm::kVariantSplit, p.family, st);
     if (e != cudaSuccess) return cuda_fail(e, "split scan launch");
     return SSM_OK;
 }

@@ -71,13 +71,17 @@ LAYOUTS = [dict(variant="slab", lanes=1), dict(variant="slab", lanes=2), dict(va
            dict(variant="split", segments=7, lanes=4)]
 
 
-@pytest.mark.parametrize("family", ["generic", "staged"])
+FAMILIES = {"generic": dict(family="generic"), "staged": dict(family="staged", cpl=1),
+            "staged_cpl2": dict(family="staged", cpl=2)}
+
+
+@pytest.mark.parametrize("family", sorted(FAMILIES))
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("layout", range(len(LAYOUTS)))
 def test_layouts_ragged(io, layout, family):
-    # dim 200: one full 128-channel tile + a ragged one; L 333 = several chunks + a tail
+    # dim 200: full channel tiles + a ragged one; L 333 = several chunks + a tail
     _, x = _case(io, 3, 333, 200, 16, seed=10 + layout, h0_sigma=0.3, d_skip="uniform")
-    _check(x, io, family=family, **LAYOUTS[layout])
+    _check(x, io, **FAMILIES[family], **LAYOUTS[layout])
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -91,9 +95,10 @@ def test_state_sizes(io, N):
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("N", [8, 16, 24, 32, 64])
 @pytest.mark.parametrize("lanes", [1, 2, 4])
-def test_state_sizes_staged(io, N, lanes):
+@pytest.mark.parametrize("cpl", [1, 2])
+def test_state_sizes_staged(io, N, lanes, cpl):
     _, x = _case(io, 2, 130, 40, N, seed=N + lanes, h0_sigma=0.2)
-    _check(x, io, family="staged", lanes=lanes, variant="slab")
+    _check(x, io, family="staged", lanes=lanes, variant="slab", cpl=cpl)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -122,9 +127,9 @@ def test_split_equals_slab_long(io):
     """Sequence split vs one pass at many segment counts, both vs the oracle."""
     _, x = _case(io, 1, 4 * 1024 + 77, 24, 16, seed=7, h0_sigma=0.3)
     ref_out, ref_state = T.oracle_scan(x, io)
-    for family in ("generic", "staged"):
+    for fam in ("generic", "staged", "staged_cpl2"):
         for seg in (2, 3, 16, 65):
-            out, st = T.gpu_scan(x, io, variant="split", segments=seg, family=family)
+            out, st = T.gpu_scan(x, io, variant="split", segments=seg, **FAMILIES[fam])
             T.check_out(T.from_dev(out), ref_out, io)
             T.check_state(T.from_dev(st), ref_state, io)
 
@@ -172,3 +177,20 @@ def test_empty_inputs_leave_state_untouched(lib):
         out = lib.selective_scan_fwd(u, u, A, Bm, Bm, last_state=st)
         torch.cuda.synchronize()
         assert out.shape == (batch, L, dim) and torch.equal(st, st0)
+
+
+def test_failed_call_leaves_no_cuda_error_behind(lib):
+    """A call that fails inside a CUDA runtime call returns SSM_ERR_CUDA and
+    leaves the runtime's error state clean for the caller (torch shares it).
+    Here the sequence split asks cudaMallocAsync for ~1 TB of carries, which
+    fails before anything is launched; the data pointers are never used."""
+    import ctypes
+    dims = lib.SSMDims(1, 65536, 1 << 24, 16)
+    opts = lib.SSMScanOpts(2, 1024, 1, 1, 0)  # split, 1024 segments, 1 lane, generic
+    fake = 0x100000
+    rc = lib.lib.ssm_selective_scan_fwd_ex(dims, lib.SSM_BF16, fake, fake, fake, fake, fake, None, None,
+                                           None, 1, fake, None, ctypes.byref(opts), None)
+    assert rc == lib.SSM_ERR_CUDA
+    assert b"workspace" in lib.lib.ssm_last_error()
+    torch.cuda.synchronize()
+    assert torch.ones(8, device="cuda").sum().item() == 8.0
