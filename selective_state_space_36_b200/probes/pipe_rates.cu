@@ -37,11 +37,12 @@ __device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsign
 }
 
 // KIND: 0 ex2 + K ffma, 1 tanh + K ffma, 2 ex2.f16x2 + K ffma, 3 ex2 + K ffma2,
-//       4 K ffma only, 5 K ffma2 only
+//       4 K ffma only, 5 K ffma2 only, 6 ex2 + K/2 ffma + K/2 integer xor-add,
+//       7 K/2 ffma + K/2 integer xor-add (no transcendental)
 template <int K, int KIND>
 __global__ void chains(float *out, long long *cyc, float s) {
     float a[4], b[4];
-    unsigned hh[4];
+    unsigned hh[4], iv[4];
     unsigned long long b2[4], s2, c2;
     {
         float2 v = make_float2(s, s);
@@ -53,6 +54,7 @@ __global__ void chains(float *out, long long *cyc, float s) {
         a[i] = -(threadIdx.x * 1e-4f + i * 0.01f);
         b[i] = i;
         hh[i] = 0x3c003c00u ^ threadIdx.x;
+        iv[i] = threadIdx.x * 7u + i;
         float2 v = make_float2(i, i + 1);
         b2[i] = *reinterpret_cast<unsigned long long *>(&v);
     }
@@ -60,12 +62,13 @@ __global__ void chains(float *out, long long *cyc, float s) {
     for (int it = 0; it < ITERS; ++it) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if (KIND == 0 || KIND == 3) a[i] = ex2(a[i]);
+            if (KIND == 0 || KIND == 3 || KIND == 6) a[i] = ex2(a[i]);
             if (KIND == 1) a[i] = th(a[i]);
             if (KIND == 2) hh[i] = ex2h2(hh[i]);
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 if (KIND == 3 || KIND == 5) b2[i] = ffma2(b2[i], s2, c2);
+                else if ((KIND == 6 || KIND == 7) && (k & 1)) iv[i] = (iv[i] ^ 0x9e3779b9u) + (unsigned)k;
                 else b[i] = fmaf(b[i], s, 0.25f);
             }
         }
@@ -74,7 +77,7 @@ __global__ void chains(float *out, long long *cyc, float s) {
     float r = 0;
     for (int i = 0; i < 4; ++i) {
         float2 v = *reinterpret_cast<float2 *>(&b2[i]);
-        r += a[i] + b[i] + (float)hh[i] + v.x + v.y;
+        r += a[i] + b[i] + (float)hh[i] + (float)iv[i] + v.x + v.y;
     }
     out[blockIdx.x * blockDim.x + threadIdx.x] = r;
     if (threadIdx.x == 0) cyc[blockIdx.x] = t1 - t0;
@@ -125,6 +128,9 @@ int main() {
     run("tanh + ffma", chains<8, 1>, 8, 1, 1, sms);
     run("ex2.f16x2", chains<0, 2>, 0, 1, 1, sms);
     run("ex2.f16x2 + ffma", chains<8, 2>, 8, 1, 1, sms);
+    run("ffma/int mix only", chains<8, 7>, 8, 1, 0, sms);
+    run("ex2 + ffma/int mix", chains<8, 6>, 8, 1, 1, sms);
+    run("ex2 + ffma/int mix", chains<16, 6>, 16, 1, 1, sms);
 
     const size_t n = (size_t)1 << 30;
     void *a, *b;
