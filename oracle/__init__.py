@@ -18,6 +18,8 @@ Parity status of each function (what pins it lives in tests/test_oracle_pins.py)
   scan(..., zoh_b=True)   pinned: brute force (ZOH form), Theorem 1.
   state_update            pinned: 1000 decode steps == scan over 1000 steps,
                           one-step brute force.
+  scan_bwd                pinned: central finite differences of scan (every
+                          input), torch autograd of an independent fp64 loop.
 """
 from __future__ import annotations
 
@@ -60,6 +62,8 @@ def _bind(path: str):
                                         _dp, _dp, _dp, _dp, _dp]
     lib.oracle_default_threads.restype = ctypes.c_int
     lib.oracle_default_threads.argtypes = []
+    lib.oracle_selective_scan_bwd.restype = ctypes.c_int
+    lib.oracle_selective_scan_bwd.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [ctypes.c_int] + [_dp] * 11
     return lib
 
 
@@ -124,6 +128,43 @@ def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True
     return out, state
 
 
+def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, delta_softplus=True,
+             h0=None, _lib_handle=None):
+    """Gradients of sum(dout * out) of the scan (Euler Bbar) in fp64.
+
+    Returns a dict: du, ddelta, dz (batch, seqlen, dim) [dz None without z],
+    dA (dim, dstate), dB, dC (batch, seqlen, dstate), dD, ddelta_bias (dim,),
+    dh0 (batch, dim, dstate).
+    """
+    u = np.asarray(u)
+    batch, seqlen, dim = u.shape
+    dstate = np.asarray(A).shape[1]
+    keep = []
+
+    def p(a, shape, name):
+        arr, ptr = _c64(a, shape, name)
+        keep.append(arr)
+        return ptr
+
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate)
+    ins = [p(u, seq, "u"), p(delta, seq, "delta"), p(A, (dim, dstate), "A"), p(B, bc, "B"),
+           p(C, bc, "C"), p(D, (dim,), "D"), p(z, seq, "z"), p(delta_bias, (dim,), "delta_bias")]
+    ph0 = p(h0, (batch, dim, dstate), "h0")
+    pdo = p(dout, seq, "dout")
+    out = {"du": np.zeros(seq), "ddelta": np.zeros(seq), "dA": np.zeros((dim, dstate)),
+           "dB": np.zeros(bc), "dC": np.zeros(bc), "dD": np.zeros(dim),
+           "dz": np.zeros(seq) if z is not None else None, "ddelta_bias": np.zeros(dim),
+           "dh0": np.zeros((batch, dim, dstate))}
+    ptr = lambda k: out[k].ctypes.data_as(_dp) if out[k] is not None else None
+    rc = (_lib_handle or _load()).oracle_selective_scan_bwd(
+        batch, seqlen, dim, dstate, *ins, int(bool(delta_softplus)), ph0, pdo,
+        ptr("du"), ptr("ddelta"), ptr("dA"), ptr("dB"), ptr("dC"), ptr("dD"), ptr("dz"),
+        ptr("ddelta_bias"), ptr("dh0"))
+    if rc != 0:
+        raise RuntimeError(f"oracle_selective_scan_bwd failed with code {rc}")
+    return out
+
+
 def state_update(state, x, dt, A, B, C, D=None, z=None, _lib_handle=None):
     """One decode step in fp64.  Returns (out (batch, dim), new_state)."""
     st = np.array(state, dtype=np.float64, order="C", copy=True)
@@ -162,6 +203,9 @@ class Variant:
 
     def state_update(self, *a, **kw):
         return state_update(*a, _lib_handle=self._h, **kw)
+
+    def scan_bwd(self, *a, **kw):
+        return scan_bwd(*a, _lib_handle=self._h, **kw)
 
 
 def compile_variant(source: str, path: str) -> "Variant":

@@ -181,6 +181,100 @@ int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t ds
 }
 
 /*
+ * Gradient of the selective scan (Euler Bbar) for upstream gradients dout of
+ * the output: the chain rule applied to the forward loop of
+ * oracle_selective_scan, in reverse time.  Per channel the forward states
+ * h_{-1..L-1} are first stored (this is a reference; the library recomputes
+ * them instead), then with lambda_t = dL/dh_t:
+ *     dy_t      = dout_t silu(z_t)        (dout_t without a gate)
+ *     dz_t      = dout_t y_t silu'(z_t),  silu'(z) = s (1 + z (1 - s)), s = sigmoid(z)
+ *     lambda_t  = dy_t C_t + Abar_{t+1} lambda_{t+1}
+ *     dC_t     += dy_t h_t                (summed over channels)
+ *     dDelta_t  = sum_n lambda_t,n (h_{t-1},n Abar_t,n A_n + B_t,n u_t)
+ *     dA_n     += lambda_t,n h_{t-1},n Abar_t,n Delta_t
+ *     dB_t,n   += lambda_t,n Delta_t u_t  (summed over channels)
+ *     du_t      = dy_t D + Delta_t sum_n lambda_t,n B_t,n
+ *     dD       += dy_t u_t
+ *     ddelta_t  = dDelta_t sigmoid(delta_t + bias) (softplus on) or dDelta_t
+ *     dbias    += ddelta_t;   dh0 = Abar_0 lambda_0
+ * Every gradient array is overwritten.  dz may be NULL when z is NULL; dh0 may
+ * be NULL.  Single-threaded (the channel-shared gradients are plain sums).
+ */
+int oracle_selective_scan_bwd(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                              const double *u, const double *delta, const double *A,
+                              const double *B, const double *C, const double *Dskip,
+                              const double *z, const double *delta_bias, int delta_softplus,
+                              const double *h0, const double *dout, double *du, double *ddelta,
+                              double *dA, double *dB, double *dC, double *dD, double *dz,
+                              double *ddelta_bias, double *dh0)
+{
+    const int64_t L = seqlen, Dm = dim, N = dstate;
+    if (batch < 0 || L < 0 || Dm < 0 || N < 0) return ORACLE_BAD_ARG;
+    if (!du || !ddelta || !dA || !dB || !dC || !dD || !ddelta_bias || (z && !dz)) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < Dm * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < batch * L * N; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    for (int64_t i = 0; i < Dm; ++i) { dD[i] = 0.0; ddelta_bias[i] = 0.0; }
+    double *hs = (double *)malloc((size_t)((L + 1) * (N > 0 ? N : 1)) * sizeof(double));
+    double *dl = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    double *yv = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    double *lam = (double *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+    if (!hs || !dl || !yv || !lam) { free(hs); free(dl); free(yv); free(lam); return ORACLE_NO_MEM; }
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < Dm; ++d) {
+            /* forward, keeping every state: hs[(t + 1) N + n] = h_t[n] */
+            for (int64_t n = 0; n < N; ++n) hs[n] = h0 ? h0[(b * Dm + d) * N + n] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t td = (b * L + t) * Dm + d, tn = (b * L + t) * N;
+                const double s = delta[td] + (delta_bias ? delta_bias[d] : 0.0);
+                dl[t] = delta_softplus ? oracle_softplus(s) : s;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double h = exp(dl[t] * A[d * N + n]) * hs[t * N + n] + dl[t] * B[tn + n] * u[td];
+                    hs[(t + 1) * N + n] = h;
+                    acc += C[tn + n] * h;
+                }
+                yv[t] = acc + (Dskip ? Dskip[d] * u[td] : 0.0);
+            }
+            /* reverse */
+            for (int64_t n = 0; n < N; ++n) lam[n] = 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const int64_t td = (b * L + t) * Dm + d, tn = (b * L + t) * N;
+                double dy = dout[td];
+                if (z) {
+                    const double sg = 1.0 / (1.0 + exp(-z[td]));
+                    dy = dout[td] * z[td] * sg;
+                    dz[td] = dout[td] * yv[t] * sg * (1.0 + z[td] * (1.0 - sg));
+                }
+                if (Dskip) dD[d] += dy * u[td];
+                double dut = Dskip ? dy * Dskip[d] : 0.0;
+                double ddl = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double an = A[d * N + n];
+                    const double abar = exp(dl[t] * an);
+                    const double hprev = hs[t * N + n];
+                    lam[n] += dy * C[tn + n];
+                    dC[tn + n] += dy * hs[(t + 1) * N + n];
+                    ddl += lam[n] * (hprev * abar * an + B[tn + n] * u[td]);
+                    dA[d * N + n] += lam[n] * hprev * abar * dl[t];
+                    dB[tn + n] += lam[n] * dl[t] * u[td];
+                    dut += lam[n] * dl[t] * B[tn + n];
+                    lam[n] *= abar;
+                }
+                du[td] = dut;
+                double sv = delta[td] + (delta_bias ? delta_bias[d] : 0.0);
+                const double dd = delta_softplus ? ddl / (1.0 + exp(-sv)) : ddl;
+                ddelta[td] = dd;
+                ddelta_bias[d] += dd;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n) dh0[(b * Dm + d) * N + n] = lam[n];
+        }
+    }
+    free(hs); free(dl); free(yv); free(lam);
+    return ORACLE_OK;
+}
+
+/*
  * One recurrent (decode) step for every channel (NL-345 section 1: constant
  * time per generated step; section 2 eq. (2) for one t).  dt is the time step
  * itself (already positive: no bias, no softplus).  state (batch, dim, dstate)

@@ -39,6 +39,15 @@ MUTANTS = {
     "decode_without_dt": ("h[n] = abar * h[n] + dlt * B[b * dstate + n] * xv;",
                           "h[n] = abar * h[n] + B[b * dstate + n] * xv;"),
     "h0_ignored": ("h[n] = j->state ? j->state[(b * Dm + d) * N + n] : 0.0;", "h[n] = 0.0;"),
+    # backward
+    "bwd_adjoint_not_decayed": ("lam[n] *= abar;", "(void)0;"),
+    "bwd_dA_without_decay": ("dA[d * N + n] += lam[n] * hprev * abar * dl[t];",
+                             "dA[d * N + n] += lam[n] * hprev * dl[t];"),
+    "bwd_dC_with_previous_state": ("dC[tn + n] += dy * hs[(t + 1) * N + n];", "dC[tn + n] += dy * hprev;"),
+    "bwd_silu_derivative": ("dz[td] = dout[td] * yv[t] * sg * (1.0 + z[td] * (1.0 - sg));",
+                            "dz[td] = dout[td] * yv[t] * sg;"),
+    "bwd_softplus_derivative": ("const double dd = delta_softplus ? ddl / (1.0 + exp(-sv)) : ddl;",
+                                "const double dd = ddl;"),
 }
 
 

@@ -341,3 +341,70 @@ def test_empty_and_degenerate_shapes(oracle_mod):
     out, last = oracle_mod.scan(u, rng.standard_normal((1, 5, 2)), np.zeros((2, 0)),
                                 np.zeros((1, 5, 0)), np.zeros((1, 5, 0)), D=np.array([2.0, -1.0]), z=z)
     _close(out, np.array([2.0, -1.0]) * u * z * expit(z), 1e-15)
+
+
+# ------------------------------------------------------------------ backward
+def _bwd_case(seed, softplus=True, gate=True):
+    rng = np.random.default_rng(seed)
+    case = _rand_case(rng, batch=2, L=6, dim=3, N=3, softplus=softplus, gate=gate)
+    if not softplus:
+        case["delta"] = np.abs(case["delta"]) + 0.1
+    dout = rng.standard_normal(case["u"].shape)
+    return case, dout
+
+
+_GRAD_OF = {"u": "du", "delta": "ddelta", "z": "dz", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+            "delta_bias": "ddelta_bias", "h0": "dh0"}
+
+
+def _loss(oracle_mod, case, dout):
+    out, _ = _run(oracle_mod, case)
+    return float(np.sum(out * dout))
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+@pytest.mark.parametrize("gate", [True, False])
+def test_bwd_matches_central_differences(oracle_mod, softplus, gate):
+    """Every gradient of sum(dout * out) against central differences of the
+    (separately pinned) forward oracle, eps = 1e-6."""
+    case, dout = _bwd_case(60 + 2 * softplus + gate, softplus, gate)
+    g = oracle_mod.scan_bwd(case["u"], case["delta"], case["A"], case["B"], case["C"], dout,
+                            D=case["D"], z=case["z"], delta_bias=case["delta_bias"],
+                            delta_softplus=softplus, h0=case["h0"])
+    eps = 1e-6
+    for name, gname in _GRAD_OF.items():
+        if case[name] is None:
+            continue
+        base = case[name]
+        for idx in np.ndindex(base.shape):
+            plus, minus = dict(case), dict(case)
+            plus[name] = base.copy(); plus[name][idx] += eps
+            minus[name] = base.copy(); minus[name][idx] -= eps
+            fd = (_loss(oracle_mod, plus, dout) - _loss(oracle_mod, minus, dout)) / (2 * eps)
+            assert abs(fd - g[gname][idx]) <= 2e-7 * (1 + abs(fd)), (name, idx, fd, g[gname][idx])
+
+
+def test_bwd_matches_torch_autograd(oracle_mod):
+    """Gradients from torch autograd of an independent plain fp64 loop."""
+    import torch
+    case, dout = _bwd_case(70)
+    t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True)
+         for k, v in case.items() if isinstance(v, np.ndarray)}
+    batch, L, dim = case["u"].shape
+    N = case["A"].shape[1]
+    outs = []
+    for b in range(batch):
+        h = t["h0"][b]                                            # (dim, N)
+        rows = []
+        for s in range(L):
+            dlt = torch.nn.functional.softplus(t["delta"][b, s] + t["delta_bias"])   # (dim,)
+            h = torch.exp(dlt[:, None] * t["A"]) * h + (dlt * t["u"][b, s])[:, None] * t["B"][b, s][None, :]
+            y = h @ t["C"][b, s] + t["D"] * t["u"][b, s]
+            rows.append(y * torch.nn.functional.silu(t["z"][b, s]))
+        outs.append(torch.stack(rows))
+    loss = (torch.stack(outs) * torch.tensor(dout)).sum()
+    loss.backward()
+    g = oracle_mod.scan_bwd(case["u"], case["delta"], case["A"], case["B"], case["C"], dout,
+                            D=case["D"], z=case["z"], delta_bias=case["delta_bias"], h0=case["h0"])
+    for name, gname in _GRAD_OF.items():
+        _close(g[gname], t[name].grad.numpy(), 1e-12)
