@@ -79,6 +79,8 @@ typedef struct CUstream_st *ssm_stream;
  *   z              : (batch, seqlen, dim) io or NULL (no gate).
  *   delta_bias     : (dim) float32 or NULL (zero bias).
  *   delta_softplus : 1 => Delta = softplus(delta + bias); 0 => delta + bias.
+ *                    (Bbar is the Euler form Delta B; ssm_selective_scan_fwd_ex can select
+ *                    the exact zero-order hold instead.)
  *   out            : (batch, seqlen, dim) io, written.
  *   last_state     : (batch, dim, dstate) float32 or NULL.  In: h_0 (the scan
  *                    resumes from it).  Out: h_L.  NULL => h_0 = 0, h_L not
@@ -114,6 +116,14 @@ typedef enum {
                                 (SSM_ERR_UNSUPPORTED otherwise) */
 } ssm_kernel_family;
 
+/* How B is discretised (A always uses the zero-order hold, Abar = exp(Delta A)). */
+typedef enum {
+    SSM_DISCRETIZE_EULER_B = 0, /* Bbar = Delta B (the default) */
+    SSM_DISCRETIZE_ZOH = 1      /* exact zero-order hold: Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B
+                                   = expm1(Delta A) / A * B, and Delta B where Delta A = 0
+                                   (【論文要約】Mamba notes, 数式解説 3); one channel per lane only */
+} ssm_discretization;
+
 typedef struct {
     int32_t variant;  /* ssm_variant */
     int32_t segments; /* SPLIT only: number of sequence segments, 0 = automatic */
@@ -122,7 +132,8 @@ typedef struct {
     int32_t family;   /* ssm_kernel_family */
     int32_t channels_per_lane; /* staged kernel: 0 = automatic, 1, or 2 (one B/C load serves two
                                   adjacent channels) */
-    int32_t reserved[3]; /* must be zero */
+    int32_t discretization;    /* ssm_discretization of B */
+    int32_t reserved[2];       /* must be zero */
 } ssm_scan_opts;
 
 /* ssm_selective_scan_fwd with explicit execution choices (opts may be NULL).

@@ -35,7 +35,8 @@ class SSMDims(ctypes.Structure):
 class SSMScanOpts(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("segments", ctypes.c_int32),
                 ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
-                ("channels_per_lane", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("channels_per_lane", ctypes.c_int32), ("discretization", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class SSMScanPlanInfo(ctypes.Structure):
@@ -125,14 +126,17 @@ def _stream_handle(stream) -> Optional[int]:
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                        out=None, last_state=None, variant: str = "auto", segments: int = 0,
-                       lanes: int = 0, family: str = "auto", cpl: int = 0, stream=None):
+                       lanes: int = 0, family: str = "auto", cpl: int = 0, zoh_b: bool = False,
+                       stream=None):
     """Selective scan forward on CUDA tensors; returns ``out``.
 
     u, delta, z: (batch, seqlen, dim); B, C: (batch, seqlen, dstate) -- all
     float32 or all bfloat16.  A (dim, dstate), D and delta_bias (dim,) float32.
     last_state (batch, dim, dstate) float32 is read as h_0 and overwritten with
-    h_L.  ``variant``/``segments``/``lanes``/``family`` force an execution
-    choice (sequence split, lanes per channel, generic or staged kernel).
+    h_L.  ``variant``/``segments``/``lanes``/``family``/``cpl`` force an
+    execution choice (sequence split, lanes per channel, generic or staged
+    kernel, channels per lane); ``zoh_b`` selects the exact zero-order hold
+    for B instead of the Euler form.
     """
     io = _io_of(u)
     batch, seqlen, dim = u.shape
@@ -150,10 +154,11 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
         _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate), dev),
     ]
     dims = SSMDims(batch, seqlen, dim, dstate)
-    if variant == "auto" and not segments and not lanes and family == "auto" and not cpl:
+    if variant == "auto" and not segments and not lanes and family == "auto" and not cpl and not zoh_b:
         check(lib.ssm_selective_scan_fwd(dims, io, *args, _stream_handle(stream)))
     else:
-        opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family], int(cpl))
+        opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family], int(cpl),
+                           int(bool(zoh_b)))
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
     return out
 

@@ -116,7 +116,7 @@ __device__ __forceinline__ void lane_finish(const ScanArgs &a, const LaneRef &g,
 
 // One time step of one channel: discretise, recur, read out.  Returns this
 // lane's partial y (its states only).  du = Delta * u.
-template <int NS, bool PRECISE>
+template <int NS, bool PRECISE, bool ZOH = false>
 __device__ __forceinline__ float lane_step(float dl, float du, const float *Bs, const float *Cs,
                                            const float (&Aw)[NS], float (&h)[NS]) {
     float y0 = 0.f, y1 = 0.f;
@@ -129,7 +129,16 @@ __device__ __forceinline__ float lane_step(float dl, float du, const float *Bs, 
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float a = decay<PRECISE>(dl, Aw[i + k]);
-            h[i + k] = fmaf(a, h[i + k], du * bb[k]);
+            float bu = du * bb[k];
+            if (ZOH) {
+                // Aw is A (precise tier) or A log2(e) (fast tier)
+                const float z = PRECISE ? dl * Aw[i + k] : dl * Aw[i + k] * kLn2;
+                bu *= PRECISE ? zoh_phi_precise(z)
+                              : (fabsf(z) < 0.0625f
+                                     ? fmaf(fmaf(fmaf(fmaf(1.f / 120.f, z, 1.f / 24.f), z, 1.f / 6.f), z, 0.5f), z, 1.f)
+                                     : (a - 1.f) / z);
+            }
+            h[i + k] = fmaf(a, h[i + k], bu);
             if (k & 1) y1 = fmaf(cc[k], h[i + k], y1);
             else y0 = fmaf(cc[k], h[i + k], y0);
         }
@@ -183,19 +192,24 @@ __device__ __forceinline__ void recur_block(const float (&dl)[K], const float (&
 
 // The same for a lane that holds NS states of each of CPL channels: step k's
 // B and C values are read once and used for every channel.
-template <int K, int NS, int CPL, bool PRECISE>
+template <int K, int NS, int CPL, bool PRECISE, bool ZOH = false>
 __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const float (&du)[K][CPL],
                                                 const float *Bs, const float *Cs, int stride,
                                                 const float2 (&A2)[CPL][NS / 2],
-                                                float2 (&h2)[CPL][NS / 2], float (&y)[K][CPL]) {
+                                                float2 (&h2)[CPL][NS / 2], float (&y)[K][CPL],
+                                                const float2 (*invA2)[NS / 2] = nullptr) {
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-        float2 d2[CPL], u2[CPL], acc[CPL];
+        float2 d2[CPL], u2[CPL], acc[CPL], id2[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             d2[c] = make_float2(dl[k][c], dl[k][c]);
             u2[c] = make_float2(du[k][c], du[k][c]);
             acc[c] = make_float2(0.f, 0.f);
+            if (ZOH && !PRECISE) {
+                const float inv = rcp_approx(dl[k][c]);
+                id2[c] = make_float2(inv, inv);
+            }
         }
 #pragma unroll
         for (int j = 0; j < NS / 4; ++j) {
@@ -211,13 +225,21 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
                     if (!PRECISE) {
                         const float2 x2 = mul2(d2[c], A2[c][p]);
                         const float2 a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
-                        h2[c][p] = fma2(a2, h2[c][p], mul2(u2[c], b2));
+                        float2 bu = mul2(u2[c], b2);
+                        if (ZOH)
+                            bu = mul2(bu, zoh_phi2(mul2(x2, make_float2(kLn2, kLn2)), a2, invA2[c][p], id2[c]));
+                        h2[c][p] = fma2(a2, h2[c][p], bu);
                         acc[c] = fma2(c2, h2[c][p], acc[c]);
                     } else {
-                        const float ax = decay_of<PRECISE>(d2[c].x * A2[c][p].x);
-                        const float ay = decay_of<PRECISE>(d2[c].y * A2[c][p].y);
-                        h2[c][p].x = fmaf(ax, h2[c][p].x, u2[c].x * b2.x);
-                        h2[c][p].y = fmaf(ay, h2[c][p].y, u2[c].y * b2.y);
+                        const float zx = d2[c].x * A2[c][p].x, zy = d2[c].y * A2[c][p].y;
+                        const float ax = decay_of<PRECISE>(zx), ay = decay_of<PRECISE>(zy);
+                        float bx = u2[c].x * b2.x, by = u2[c].y * b2.y;
+                        if (ZOH) {
+                            bx *= zoh_phi_precise(zx);
+                            by *= zoh_phi_precise(zy);
+                        }
+                        h2[c][p].x = fmaf(ax, h2[c][p].x, bx);
+                        h2[c][p].y = fmaf(ay, h2[c][p].y, by);
                         acc[c].x = fmaf(c2.x, h2[c][p].x, acc[c].x);
                         acc[c].y = fmaf(c2.y, h2[c][p].y, acc[c].y);
                     }

@@ -32,7 +32,7 @@
 
 namespace ssm {
 
-template <typename IO, int NS, int G, bool PRECISE, int MODE>
+template <typename IO, int NS, int G, bool PRECISE, int MODE, bool ZOH>
 __global__ void __launch_bounds__(kBlock)
 scan_fwd_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
@@ -83,7 +83,7 @@ scan_fwd_kernel(const ScanArgs args) {
             const float uv = io::load_stream(pu + off);
             const float s = io::load_stream(pd + off) + bias;
             const float dl = args.softplus ? softplus<PRECISE>(s) : s;
-            const float yl = lane_step<NS, PRECISE>(dl, dl * uv, &sB[r][g.q * NS], &sC[r][g.q * NS], Aw, h);
+            const float yl = lane_step<NS, PRECISE, ZOH>(dl, dl * uv, &sB[r][g.q * NS], &sC[r][g.q * NS], Aw, h);
             if (MODE == kSegAgg) {
                 dsum += (double)dl;
             } else {
@@ -107,24 +107,29 @@ bool staged_eligible(const ScanArgs &a, int es) {
     return (a.dim * es) % 16 == 0 && (a.dstate * es) % 16 == 0 && al(a.u) && al(a.delta) &&
            al(a.z) && al(a.B) && al(a.C) && al(a.out);
 }
-template <typename IO, int NS, int G>
-static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
+template <typename IO, int NS, int G, bool ZOH>
+static cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
     constexpr bool P = std::is_same<IO, float>::value;
     constexpr int CPB = kBlock / G;
     const int64_t tiles = (a.dim + CPB - 1) / CPB;
     const dim3 block(kBlock);
     if (variant == kVariantSlab) {
-        scan_fwd_kernel<IO, NS, G, P, kFull><<<dim3((unsigned)(a.batch * tiles), 1), block, 0, st>>>(a);
+        scan_fwd_kernel<IO, NS, G, P, kFull, ZOH><<<dim3((unsigned)(a.batch * tiles), 1), block, 0, st>>>(a);
         return cudaGetLastError();
     }
     if (a.nseg > 1)
-        scan_fwd_kernel<IO, NS, G, P, kSegAgg>
+        scan_fwd_kernel<IO, NS, G, P, kSegAgg, ZOH>
             <<<dim3((unsigned)(a.batch * tiles), (unsigned)(a.nseg - 1)), block, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    scan_fwd_kernel<IO, NS, G, P, kSegFinal>
+    scan_fwd_kernel<IO, NS, G, P, kSegFinal, ZOH>
         <<<dim3((unsigned)(a.batch * tiles), (unsigned)a.nseg), block, 0, st>>>(a);
     return cudaGetLastError();
+}
+
+template <typename IO, int NS, int G>
+static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
+    return a.zoh_b ? launch_z<IO, NS, G, true>(a, variant, st) : launch_z<IO, NS, G, false>(a, variant, st);
 }
 
 template <typename IO>

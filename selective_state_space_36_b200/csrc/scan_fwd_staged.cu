@@ -119,7 +119,7 @@ __device__ __forceinline__ void store_vals(IO *p, const float (&v)[CPL]) {
     }
 }
 
-template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE>
+template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH>
 __global__ void __launch_bounds__(kBlock)
 scan_fwd_staged_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
@@ -184,7 +184,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     };
 
     // per-channel constants and state
-    float2 A2[CPL][NS / 2], h2[CPL][NS / 2];
+    float2 A2[CPL][NS / 2], h2[CPL][NS / 2], invA2[CPL][NS / 2];
     float bias[CPL], dskip[CPL];
     double dsum[CPL];
 #pragma unroll
@@ -196,6 +196,10 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         for (int p = 0; p < NS / 2; ++p) {
             A2[c][p] = make_float2(Aw[2 * p], Aw[2 * p + 1]);
             h2[c][p] = make_float2(h[2 * p], h[2 * p + 1]);
+            if (ZOH) {  // 1 / A in natural units (Aw carries log2(e) in the fast tier)
+                const float s0 = PRECISE ? 1.f : kLn2;
+                invA2[c][p] = make_float2(1.f / (Aw[2 * p] * s0), 1.f / (Aw[2 * p + 1] * s0));
+            }
         }
         bias[c] = (active && args.bias) ? args.bias[dfirst + c] : 0.f;
         dskip[c] = (active && args.Dskip) ? args.Dskip[dfirst + c] : 0.f;
@@ -276,8 +280,8 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 }
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
                 exchange_steps_cpl<KSTEP, G, CPL>(dlo, duo, dl, du);
-                recur_block_cpl<KSTEP, NS, CPL, PRECISE>(dl, du, fB + r0 * NSP + q * NS,
-                                                         fC + r0 * NSP + q * NS, NSP, A2, h2, y);
+                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH>(dl, du, fB + r0 * NSP + q * NS,
+                                                              fC + r0 * NSP + q * NS, NSP, A2, h2, y, invA2);
                 if (MODE == kSegAgg) {
 #pragma unroll
                     for (int j = 0; j < KG; ++j)
@@ -320,11 +324,11 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     }
 }
 
-template <typename IO, int NS, int G, int CPL, int MODE>
+template <typename IO, int NS, int G, int CPL, int MODE, bool ZOH>
 static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
     constexpr bool P = std::is_same<IO, float>::value;
     using Lay = StagedLayout<IO, NS, G, CPL>;
-    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE>;
+    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE, ZOH>;
     // the shared-memory opt-in is a per-device function attribute: set it once per device
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -343,14 +347,22 @@ static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <typename IO, int NS, int G, int CPL>
-static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
+template <typename IO, int NS, int G, int CPL, bool ZOH>
+static cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
     constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
     const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
-    if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull>(a, dim3(bx, 1), st);
-    cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
+    if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull, ZOH>(a, dim3(bx, 1), st);
+    cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg, ZOH>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
     if (e != cudaSuccess) return e;
-    return launch_mode<IO, NS, G, CPL, kSegFinal>(a, dim3(bx, (unsigned)a.nseg), st);
+    return launch_mode<IO, NS, G, CPL, kSegFinal, ZOH>(a, dim3(bx, (unsigned)a.nseg), st);
+}
+
+// Exact ZOH on B is built for one channel per lane only.
+template <typename IO, int NS, int G, int CPL>
+static cudaError_t launch_t(const ScanArgs &a, int variant, cudaStream_t st) {
+    if (!a.zoh_b) return launch_z<IO, NS, G, CPL, false>(a, variant, st);
+    if (CPL != 1) return cudaErrorInvalidConfiguration;
+    return launch_z<IO, NS, G, 1, true>(a, variant, st);
 }
 
 template <typename IO, int CPL>

@@ -31,6 +31,7 @@ struct ScanArgs {
     int64_t batch, seqlen, dim;
     int dstate;
     int softplus;
+    int zoh_b;        // 1: exact zero-order hold on B (Bbar = expm1(Delta A)/A B); 0: Euler (Delta B)
     int64_t seg_len;  // time steps per segment (== seqlen for one pass)
     int nseg;
 };

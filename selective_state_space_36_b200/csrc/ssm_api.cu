@@ -120,6 +120,7 @@ namespace {
 struct ScanPlan {
     int variant = SSM_VARIANT_SLAB;
     int ns = 16, g = 1, cpl = 1;
+    int zoh_b = 0;
     int family = ssm::kFamilyGeneric;
     int nseg = 1;
     int64_t seg_len = 0;
@@ -149,8 +150,13 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
     const int lanes_req = opts ? opts->lanes : 0;
     int family = opts ? opts->family : 0;
     const int cpl_req = opts ? opts->channels_per_lane : 0;
-    if (opts && (opts->reserved[0] || opts->reserved[1] || opts->reserved[2]))
+    const int disc = opts ? opts->discretization : SSM_DISCRETIZE_EULER_B;
+    if (opts && (opts->reserved[0] || opts->reserved[1]))
         return fail(SSM_ERR_INVALID_ARG, "ssm_scan_opts.reserved must be zero");
+    if (disc != SSM_DISCRETIZE_EULER_B && disc != SSM_DISCRETIZE_ZOH)
+        return fail(SSM_ERR_INVALID_ARG, "discretization must be SSM_DISCRETIZE_EULER_B or SSM_DISCRETIZE_ZOH");
+    if (disc == SSM_DISCRETIZE_ZOH && cpl_req == 2)
+        return fail(SSM_ERR_UNSUPPORTED, "exact ZOH on B is built for one channel per lane");
     if (cpl_req != 0 && cpl_req != 1 && cpl_req != 2)
         return fail(SSM_ERR_INVALID_ARG, "channels per lane must be 0, 1 or 2");
     if (family < ssm::kFamilyAuto || family > ssm::kFamilyStaged)
@@ -178,7 +184,7 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
     if (family == ssm::kFamilyStaged && !eligible)
         return fail(SSM_ERR_UNSUPPORTED, "staged kernel needs 16-byte aligned rows (dim and dstate "
                     "multiples of %d, 16-byte aligned u, delta, z, B, C, out)", (int)(16 / es));
-    const int cpl_try = cpl_req ? cpl_req : kDefaultStagedCpl;
+    const int cpl_try = cpl_req ? cpl_req : (disc == SSM_DISCRETIZE_ZOH ? 1 : kDefaultStagedCpl);
     const bool fits = ssm::staged_smem_bytes(io == SSM_BF16, plan->ns, plan->g, cpl_try) <= (size_t)di.smem_optin;
     if (family == ssm::kFamilyStaged && !fits)
         return fail(SSM_ERR_UNSUPPORTED, "the staged kernel's shared memory for %d lanes x %d channels "
@@ -188,6 +194,7 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
     if (cpl_req == 2 && family != ssm::kFamilyStaged)
         return fail(SSM_ERR_UNSUPPORTED, "two channels per lane needs the staged kernel");
     plan->cpl = family == ssm::kFamilyStaged ? cpl_try : 1;
+    plan->zoh_b = disc == SSM_DISCRETIZE_ZOH;
     const int64_t cpb = ssm::kBlock / plan->g * plan->cpl;
     const int64_t blocks = dims.batch * ((dims.dim + cpb - 1) / cpb);
     if (blocks > kMaxGridX) return fail(SSM_ERR_UNSUPPORTED, "grid too large");
@@ -281,6 +288,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     a.batch = dims.batch; a.seqlen = dims.seqlen; a.dim = dims.dim;
     a.dstate = (int)dims.dstate;
     a.softplus = delta_softplus;
+    a.zoh_b = p.zoh_b;
     a.seg_len = p.seg_len;
     a.nseg = p.nseg;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

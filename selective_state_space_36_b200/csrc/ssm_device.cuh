@@ -186,6 +186,22 @@ __device__ __forceinline__ float2 softplus2_fast(float2 s) {
     return add2(make_float2(fmaxf(s.x, 0.f), fmaxf(s.y, 0.f)), mul2(p, e));
 }
 
+// Exact zero-order hold on B: Bbar = (exp(z) - 1) / z * Delta B with
+// z = Delta A, i.e. phi(z) = expm1(z) / z multiplies the Euler input term.
+// Near z = 0 the quotient cancels, so |z| < 1/16 uses the Taylor series of
+// phi to z^4 (remainder < z^5 / 720 < 1.4e-9); elsewhere (a - 1) * (1/A) * (1/Delta)
+// with a = exp(z) already computed for the decay.  Two lanes at once.
+__device__ __forceinline__ float2 zoh_phi2(float2 z, float2 a, float2 inv_a, float2 inv_dl) {
+    float2 s = make_float2(1.f / 120.f, 1.f / 120.f);
+    s = fma2(s, z, make_float2(1.f / 24.f, 1.f / 24.f));
+    s = fma2(s, z, make_float2(1.f / 6.f, 1.f / 6.f));
+    s = fma2(s, z, make_float2(0.5f, 0.5f));
+    s = fma2(s, z, make_float2(1.f, 1.f));
+    const float2 d = mul2(mul2(add2(a, make_float2(-1.f, -1.f)), inv_a), inv_dl);
+    return make_float2(fabsf(z.x) < 0.0625f ? s.x : d.x, fabsf(z.y) < 0.0625f ? s.y : d.y);
+}
+__device__ __forceinline__ float zoh_phi_precise(float z) { return z == 0.f ? 1.f : expm1f(z) / z; }
+
 template <int G>
 __device__ __forceinline__ double group_sum_d(double v) {
     if (G > 1) {

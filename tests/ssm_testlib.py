@@ -69,12 +69,12 @@ def check_state(got, ref, io, what="last_state"):
     return e
 
 
-def oracle_scan(x: dict, io: str, nthreads: int = 0):
+def oracle_scan(x: dict, io: str, nthreads: int = 0, zoh_b: bool = False):
     """Oracle on the exact fp64 values of a scan_inputs() dictionary."""
     return oracle.scan(f64(x["u"], io), f64(x["delta"], io), f64(x["A"], "f32"), f64(x["B"], io),
                        f64(x["C"], io), D=f64(x["D"], "f32"), z=f64(x["z"], io),
                        delta_bias=f64(x["delta_bias"], "f32"), delta_softplus=x["delta_softplus"],
-                       h0=f64(x["h0"], "f32"), nthreads=nthreads)
+                       h0=f64(x["h0"], "f32"), nthreads=nthreads, zoh_b=zoh_b)
 
 
 def gpu_scan(x: dict, io: str, with_state=True, **kw):

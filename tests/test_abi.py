@@ -74,7 +74,13 @@ def test_scan_argument_validation(b):
     opts = b.SSMScanOpts(1, 0, 0, 5)
     assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
     opts = b.SSMScanOpts(1, 0, 0, 0)
-    opts.reserved[2] = 1
+    opts.reserved[1] = 1
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(1, 0, 0, 0, 0, 7)  # unknown discretization
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
+    opts = b.SSMScanOpts(1, 0, 0, 2, 2, 1)  # exact ZOH with two channels per lane
+    assert _scan(b, ok, opts=opts) == b.SSM_ERR_UNSUPPORTED
+    opts = b.SSMScanOpts(1, 0, 0, 0, 3)  # channels per lane must be 0, 1 or 2
     assert _scan(b, ok, opts=opts) == b.SSM_ERR_INVALID_ARG
     # staged kernel on rows that are not 16-byte multiples: refused before launch
     opts = b.SSMScanOpts(1, 0, 0, 2)

@@ -194,3 +194,43 @@ def test_failed_call_leaves_no_cuda_error_behind(lib):
     assert b"workspace" in lib.lib.ssm_last_error()
     torch.cuda.synchronize()
     assert torch.ones(8, device="cuda").sum().item() == 8.0
+
+
+# ----------------------------------------------- exact zero-order hold on B
+@pytest.mark.parametrize("family", ["generic", "staged"])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("layout", [dict(variant="slab", lanes=1), dict(variant="slab", lanes=4),
+                                    dict(variant="split", segments=3)])
+def test_zoh_b_matches_oracle(io, family, layout):
+    """Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B (【論文要約】Mamba notes,
+    数式解説 3) against the oracle's ZOH mode, including Delta A near 0 (series
+    branch) and larger Delta A (direct branch)."""
+    _, x = _case(io, 2, 300, 96, 16, seed=41, h0_sigma=0.3, d_skip="uniform", dt_max=0.5)
+    out, st = T.gpu_scan(x, io, family=family, zoh_b=True, **layout)
+    ref_out, ref_st = T.oracle_scan(x, io, zoh_b=True)
+    T.check_out(T.from_dev(out), ref_out, io)
+    T.check_state(T.from_dev(st), ref_st, io)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_theorem1_gated_rnn_on_gpu(io):
+    """N = 1, A = -1, B = C = 1, no skip, no gate, Delta = softplus(raw + bias),
+    exact ZOH: the scan is the gated RNN h_t = (1 - g_t) h_{t-1} + g_t x_t with
+    g_t = sigmoid(raw_t + bias) (【論文要約】Mamba notes, 数式解説 4, Theorem 1),
+    computed here in fp64 from the rounded inputs, independently of the oracle."""
+    from scipy.special import expit
+    cfg, x = _case(io, 2, 200, 40, 1, seed=43, h0_sigma=0.5, has_z=False, has_d=False)
+    x["A"] = -np.ones_like(x["A"])
+    ones = np.ones_like(I.to_f64(x["B"], io))
+    x["B"] = x["C"] = (I.f32_to_bf16_bits(ones.astype(np.float32)) if io == "bf16"
+                       else ones.astype(np.float32))
+    out, st = T.gpu_scan(x, io, zoh_b=True)
+    u, raw = I.to_f64(x["u"], io), I.to_f64(x["delta"], io)
+    g = expit(raw + x["delta_bias"].astype(np.float64)[None, None, :])
+    h = x["h0"][:, :, 0].astype(np.float64)
+    ref = np.zeros_like(u)
+    for t in range(cfg.seqlen):
+        h = (1.0 - g[:, t]) * h + g[:, t] * u[:, t]
+        ref[:, t] = h
+    T.check_out(T.from_dev(out), ref, io)
+    T.check_state(T.from_dev(st)[:, :, 0:1], h[:, :, None], io)
