@@ -17,7 +17,8 @@
  * (recurrence, readout after the update); 【論文要約】Mamba notes, 数式解説 3
  * (ZOH for Abar) and the "S6" section, Algorithm 2 (B, C per token, Delta =
  * softplus(parameter + projection)).  The pages give the exact ZOH form for
- * Bbar; this library uses the Euler form Delta * B.  The D skip and the silu(z)
+ * Bbar; this library uses the Euler form Delta * B by default and offers the
+ * exact form through ssm_selective_scan_fwd_ex.  The D skip and the silu(z)
  * gate are the Mamba block's epilogue fused into the scan.
  *
  * Conventions for every entry point
@@ -203,6 +204,59 @@ typedef struct {
 ssm_status ssm_scan_plan(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
                          const void *B, const void *C, const void *z, const void *out,
                          const ssm_scan_opts *opts, ssm_scan_plan_info *info);
+
+/*
+ * Selective scan, backward: the gradients of the scalar loss sum(dout * out)
+ * of one ssm_selective_scan_fwd pass (Euler Bbar) with respect to every input.
+ * The states are recomputed from checkpoints instead of being kept by the
+ * forward pass (【論文要約】Mamba notes, "3.ハードウェアを考慮した効率的な
+ * アルゴリズム": recomputation keeps the stored intermediate states small;
+ * NL-345 section 1, "Fast training and inference").
+ *
+ * Inputs are those of the forward call (same layouts and dtypes; h0 is the
+ * state the forward pass started from, (batch, dim, dstate) float32, or NULL
+ * for zero) plus
+ *   dout           : (batch, seqlen, dim) io, the gradient of out.
+ * Outputs (all written, none accumulated into):
+ *   du, ddelta     : (batch, seqlen, dim) io.  ddelta is d/d(raw delta).
+ *   dz             : (batch, seqlen, dim) io; required iff z is given.
+ *   dA             : (dim, dstate) float32.
+ *   dB, dC         : (batch, seqlen, dstate) float32.
+ *   dD             : (dim) float32; required iff D is given.
+ *   ddelta_bias    : (dim) float32 or NULL (not computed).
+ *   dh0            : (batch, dim, dstate) float32 or NULL (not computed).
+ * The float32 sums (dA, dB, dC, dD, ddelta_bias) are accumulated with
+ * atomics, so their last bits depend on the order blocks finish in.
+ * Workspace: (batch, ceil(seqlen / K), dim, dstate) float32 state checkpoints
+ * (K = 8 on the staged path; 16, 8 or 4 on the generic one for dstate <= 16,
+ * 32, 64), taken with cudaMallocAsync and released with cudaFreeAsync on
+ * "stream".  Output buffers must not overlap each other or any input.
+ */
+ssm_status ssm_selective_scan_bwd(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                  const float *A, const void *B, const void *C, const float *D,
+                                  const void *z, const float *delta_bias, int delta_softplus,
+                                  const float *h0, const void *dout, void *du, void *ddelta,
+                                  void *dz, float *dA, float *dB, float *dC, float *dD,
+                                  float *ddelta_bias, float *dh0, ssm_stream stream);
+
+/*
+ * ssm_selective_scan_bwd with a forced kernel family (tests, tuning).  Only
+ * opts->family is read; every other field of opts must be zero (the backward
+ * has no sequence split and no lane choices, and implements the Euler Bbar
+ * only).  SSM_KERNEL_STAGED -- a checkpointing pass of the staged forward
+ * kernel (a state every 8 steps) and a staged reverse pass -- needs
+ * dstate <= 16 and the staged forward kernel's row alignment (for du, ddelta,
+ * dz and dout as well); SSM_KERNEL_GENERIC is one kernel with direct global
+ * loads and a checkpoint every 64 / ceil(dstate / 4) steps.  opts may be NULL
+ * (automatic: staged where eligible).
+ */
+ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, const float *delta_bias, int delta_softplus,
+                                     const float *h0, const void *dout, void *du, void *ddelta,
+                                     void *dz, float *dA, float *dB, float *dC, float *dD,
+                                     float *ddelta_bias, float *dh0, const ssm_scan_opts *opts,
+                                     ssm_stream stream);
 
 /*
  * One recurrent (decode) step for every channel: constant time and memory per

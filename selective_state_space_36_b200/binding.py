@@ -22,7 +22,7 @@ FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
 
 # every symbol include/ssm.h declares
 EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
-            "ssm_selective_state_update", "ssm_scan_plan", "ssm_status_string", "ssm_last_error",
+            "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ex", "ssm_selective_state_update", "ssm_scan_plan", "ssm_status_string", "ssm_last_error",
             "ssm_version")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -67,6 +67,12 @@ def _load() -> ctypes.CDLL:
     lib.ssm_selective_scan_fwd_ex.restype = ctypes.c_int
     lib.ssm_selective_scan_fwd_noalloc.argtypes = scan_args + [ctypes.c_int, _vp]
     lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssm_selective_scan_bwd.argtypes = ([SSMDims, ctypes.c_int] + [_vp] * 8 + [ctypes.c_int] +
+                                           [_vp] * 11 + [_vp])
+    lib.ssm_selective_scan_bwd.restype = ctypes.c_int
+    lib.ssm_selective_scan_bwd_ex.argtypes = ([SSMDims, ctypes.c_int] + [_vp] * 8 + [ctypes.c_int] +
+                                              [_vp] * 11 + [ctypes.POINTER(SSMScanOpts), _vp])
+    lib.ssm_selective_scan_bwd_ex.restype = ctypes.c_int
     lib.ssm_selective_state_update.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp]
     lib.ssm_selective_state_update.restype = ctypes.c_int
@@ -161,6 +167,49 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
                            int(bool(zoh_b)))
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
     return out
+
+
+def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, h0=None, want_dh0=False, family: str = "auto",
+                       stream=None):
+    """Gradients of sum(dout * out) of one forward scan (Euler Bbar).
+
+    Arguments as for ``selective_scan_fwd``; ``h0`` (batch, dim, dstate)
+    float32 is the state that forward pass started from (None: zero).  Returns
+    a dict: du, ddelta, dz (io dtype, dz None without z); dA (dim, dstate), dB,
+    dC (batch, seqlen, dstate), dD (None without D), ddelta_bias (None without
+    delta_bias) float32; dh0 (batch, dim, dstate) float32 if ``want_dh0`` (or
+    h0 is given), else None.  ``family`` forces the generic or the staged
+    kernels.
+    """
+    io = _io_of(u)
+    batch, seqlen, dim = u.shape
+    dstate = A.shape[1]
+    dev = u.device
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+         "dz": torch.empty_like(u) if z is not None else None,
+         "dA": torch.empty((dim, dstate), **f32), "dB": torch.empty(bc, **f32),
+         "dC": torch.empty(bc, **f32),
+         "dD": torch.empty((dim,), **f32) if D is not None else None,
+         "ddelta_bias": torch.empty((dim,), **f32) if delta_bias is not None else None,
+         "dh0": torch.empty((batch, dim, dstate), **f32) if (want_dh0 or h0 is not None) else None}
+    args = [
+        _ptr(u, "u", u.dtype, seq, dev), _ptr(delta, "delta", u.dtype, seq, dev),
+        _ptr(A, "A", torch.float32, (dim, dstate), dev), _ptr(B, "B", u.dtype, bc, dev),
+        _ptr(C, "C", u.dtype, bc, dev), _ptr(D, "D", torch.float32, (dim,), dev),
+        _ptr(z, "z", u.dtype, seq, dev), _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev),
+        int(bool(delta_softplus)),
+        _ptr(h0, "h0", torch.float32, (batch, dim, dstate), dev), _ptr(dout, "dout", u.dtype, seq, dev),
+    ] + [_ptr(g[k], k) for k in ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dh0")]
+    dims = SSMDims(batch, seqlen, dim, dstate)
+    if family == "auto":
+        check(lib.ssm_selective_scan_bwd(dims, io, *args, _stream_handle(stream)))
+    else:
+        opts = SSMScanOpts(0, 0, 0, FAMILIES[family])
+        check(lib.ssm_selective_scan_bwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
+    return g
 
 
 def selective_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None,

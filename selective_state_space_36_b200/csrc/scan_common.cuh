@@ -51,7 +51,7 @@ __device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneRef &g, i
     }
     if (!g.active) return;
     const int64_t soff = (g.b * a.dim + g.d) * N;
-    if (MODE == kFull && a.last_state) {
+    if ((MODE == kFull || MODE == kCkpt) && a.last_state) {
 #pragma unroll
         for (int i = 0; i < NS; ++i) {
             const int n = g.q * NS + i;
@@ -94,7 +94,7 @@ __device__ __forceinline__ void lane_init(const ScanArgs &a, const LaneRef &g, i
 template <int NS, int MODE>
 __device__ __forceinline__ void lane_finish(const ScanArgs &a, const LaneRef &g, int seg,
                                             int64_t t_end, const float (&h)[NS], double dsum) {
-    if (!g.active) return;
+    if (!g.active || MODE == kCkpt) return;
     const int N = a.dstate;
     if (MODE == kSegAgg) {
         const int64_t agg = (g.b * a.nseg + seg) * a.dim + g.d;
@@ -192,7 +192,7 @@ __device__ __forceinline__ void recur_block(const float (&dl)[K], const float (&
 
 // The same for a lane that holds NS states of each of CPL channels: step k's
 // B and C values are read once and used for every channel.
-template <int K, int NS, int CPL, bool PRECISE, bool ZOH = false>
+template <int K, int NS, int CPL, bool PRECISE, bool ZOH = false, bool READOUT = true>
 __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const float (&du)[K][CPL],
                                                 const float *Bs, const float *Cs, int stride,
                                                 const float2 (&A2)[CPL][NS / 2],
@@ -214,7 +214,8 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
 #pragma unroll
         for (int j = 0; j < NS / 4; ++j) {
             const float4 bv = *reinterpret_cast<const float4 *>(Bs + k * stride + 4 * j);
-            const float4 cv = *reinterpret_cast<const float4 *>(Cs + k * stride + 4 * j);
+            const float4 cv = READOUT ? *reinterpret_cast<const float4 *>(Cs + k * stride + 4 * j)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int hlf = 0; hlf < 2; ++hlf) {
                 const int p = 2 * j + hlf;
@@ -229,7 +230,7 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
                         if (ZOH)
                             bu = mul2(bu, zoh_phi2(mul2(x2, make_float2(kLn2, kLn2)), a2, invA2[c][p], id2[c]));
                         h2[c][p] = fma2(a2, h2[c][p], bu);
-                        acc[c] = fma2(c2, h2[c][p], acc[c]);
+                        if (READOUT) acc[c] = fma2(c2, h2[c][p], acc[c]);
                     } else {
                         const float zx = d2[c].x * A2[c][p].x, zy = d2[c].y * A2[c][p].y;
                         const float ax = decay_of<PRECISE>(zx), ay = decay_of<PRECISE>(zy);
@@ -240,8 +241,10 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
                         }
                         h2[c][p].x = fmaf(ax, h2[c][p].x, bx);
                         h2[c][p].y = fmaf(ay, h2[c][p].y, by);
-                        acc[c].x = fmaf(c2.x, h2[c][p].x, acc[c].x);
-                        acc[c].y = fmaf(c2.y, h2[c][p].y, acc[c].y);
+                        if (READOUT) {
+                            acc[c].x = fmaf(c2.x, h2[c][p].x, acc[c].x);
+                            acc[c].y = fmaf(c2.y, h2[c][p].y, acc[c].y);
+                        }
                     }
                 }
             }

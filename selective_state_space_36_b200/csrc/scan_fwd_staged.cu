@@ -27,6 +27,7 @@
 // boundaries.
 #include <atomic>
 
+#include "cp_async.cuh"
 #include "scan_common.cuh"
 
 namespace ssm {
@@ -57,17 +58,6 @@ struct StagedCfg {
     static constexpr int T = sizeof(IO) == 2 ? SSM_CHUNK_BF16 : 16;  // time steps per chunk
     static constexpr int STAGES = SSM_STAGES;
 };
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool full) {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    const int n = full ? 16 : 0;  // 0: no global read, destination zero-filled
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
 
 // Row padding: with G > 1 the lanes of a group read G different rows at once,
 // and 32 bytes of padding put those rows in different banks; with G = 1 all
@@ -150,7 +140,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
 
     const IO *pu = static_cast<const IO *>(args.u);
     const IO *pd = static_cast<const IO *>(args.delta);
-    const IO *pz = MODE == kSegAgg ? nullptr : static_cast<const IO *>(args.z);
+    const IO *pz = (MODE == kSegAgg || MODE == kCkpt) ? nullptr : static_cast<const IO *>(args.z);
     const IO *pB = static_cast<const IO *>(args.B);
     const IO *pC = static_cast<const IO *>(args.C);
     IO *po = static_cast<IO *>(args.out);
@@ -179,7 +169,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         const int64_t gbc = (b * L + tc) * N;
         for (int p = tid; p < pieces; p += kBlock) {
             cp_async16(rb + p * EPV, pB + gbc + p * EPV, true);
-            cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
+            if (MODE != kCkpt) cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
         }
     };
 
@@ -224,7 +214,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
             const int r = i / NSP, n = i % NSP;
             const bool ok = r < rows && n < N;
             fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
-            fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+            if (MODE != kCkpt) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
         }
         __syncthreads();
         if (active) {
@@ -278,11 +268,23 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                         duo[j][cc] = dlo[j][cc] * uvo[j][cc];
                     }
                 }
+                if (MODE == kCkpt && (tc + r0) % args.ckpt_every == 0) {
+                    // the state entering step tc + r0 (ckpt_every is a multiple of KSTEP)
+                    const int64_t nck = (L + args.ckpt_every - 1) / args.ckpt_every;
+                    float *cp = args.ckpt + ((b * nck + (tc + r0) / args.ckpt_every) * Dm + dfirst) * N + q * NS;
+#pragma unroll
+                    for (int p = 0; p < NS / 2; ++p) {
+                        if (q * NS + 2 * p < N) cp[2 * p] = h2[0][p].x;
+                        if (q * NS + 2 * p + 1 < N) cp[2 * p + 1] = h2[0][p].y;
+                    }
+                }
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
                 exchange_steps_cpl<KSTEP, G, CPL>(dlo, duo, dl, du);
-                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH>(dl, du, fB + r0 * NSP + q * NS,
-                                                              fC + r0 * NSP + q * NS, NSP, A2, h2, y, invA2);
-                if (MODE == kSegAgg) {
+                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, MODE != kCkpt>(
+                    dl, du, fB + r0 * NSP + q * NS, fC + r0 * NSP + q * NS, NSP, A2, h2, y, invA2);
+                if (MODE == kCkpt) {
+                    // no readout
+                } else if (MODE == kSegAgg) {
 #pragma unroll
                     for (int j = 0; j < KG; ++j)
 #pragma unroll
@@ -352,6 +354,10 @@ static cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
     constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
     const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
     if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull, ZOH>(a, dim3(bx, 1), st);
+    if (variant == kVariantCkpt) {
+        if (CPL != 1 || ZOH) return cudaErrorInvalidConfiguration;
+        return launch_mode<IO, NS, G, 1, kCkpt, false>(a, dim3(bx, 1), st);
+    }
     cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg, ZOH>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
     if (e != cudaSuccess) return e;
     return launch_mode<IO, NS, G, CPL, kSegFinal, ZOH>(a, dim3(bx, (unsigned)a.nseg), st);

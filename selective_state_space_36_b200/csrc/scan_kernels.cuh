@@ -14,8 +14,10 @@ namespace ssm {
 constexpr int kBlock = 128;  // threads per block
 constexpr int kChunk = 64;   // time steps of B/C staged in shared memory at once
 
-enum ScanMode { kFull = 0, kSegAgg = 1, kSegFinal = 2 };
-enum { kVariantSlab = 1, kVariantSplit = 2 };
+// kCkpt: forward recurrence only (no readout), storing the state entering
+// every ckpt_every-th step -- the first pass of the backward scan.
+enum ScanMode { kFull = 0, kSegAgg = 1, kSegFinal = 2, kCkpt = 3 };
+enum { kVariantSlab = 1, kVariantSplit = 2, kVariantCkpt = 3 };
 // kernel family: generic (direct global loads, any alignment) or staged
 // (cp.async pipeline through shared memory, 16-byte aligned rows)
 enum { kFamilyAuto = 0, kFamilyGeneric = 1, kFamilyStaged = 2 };
@@ -34,6 +36,10 @@ struct ScanArgs {
     int zoh_b;        // 1: exact zero-order hold on B (Bbar = expm1(Delta A)/A B); 0: Euler (Delta B)
     int64_t seg_len;  // time steps per segment (== seqlen for one pass)
     int nseg;
+    // kCkpt: states (batch, ceil(seqlen / ckpt_every), dim, dstate); h_0 is
+    // read from last_state, which is not written
+    float *ckpt;
+    int ckpt_every;
 };
 
 struct DecodeArgs {
@@ -45,6 +51,20 @@ struct DecodeArgs {
     int dstate;
 };
 
+// Gradient of the scan (Euler Bbar): inputs as in ScanArgs plus dout; the
+// accumulated gradients (dA, dB, dC, dD, dbias) must be zero on entry.
+struct ScanBwdArgs {
+    const void *u, *delta, *B, *C, *z, *dout;
+    const float *A, *Dskip, *bias, *h0;
+    void *du, *ddelta, *dz;
+    float *dA, *dB, *dC, *dD, *dbias, *dh0;
+    float *ckpt;  // workspace: (batch, ceil(seqlen / chunk), dim, dstate) states
+    int64_t batch, seqlen, dim;
+    int dstate;
+    int softplus;
+    int vec_red;  // dB / dC rows take 16-byte vector atomics
+};
+
 cudaError_t launch_scan_fwd(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
                             int family, cudaStream_t st);
 cudaError_t launch_scan_staged(const ScanArgs &a, bool bf16, int ns, int g, int cpl, int variant,
@@ -53,5 +73,13 @@ bool staged_eligible(const ScanArgs &a, int es);
 size_t staged_smem_bytes(bool bf16, int ns, int g, int cpl);
 bool scan_shape_supported(int ns, int g);
 cudaError_t launch_state_update(const DecodeArgs &a, bool bf16, int ns, int g, cudaStream_t st);
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
+// staged second pass (checkpoints every scan_bwd_staged_chunk() steps, from
+// the staged forward kernel in kCkpt mode)
+bool scan_bwd_staged_eligible(const ScanBwdArgs &a, int es);
+int scan_bwd_staged_chunk();
+cudaError_t launch_scan_bwd_staged(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
+int64_t scan_bwd_chunk(int dstate);              // time steps between checkpoints
+int64_t scan_bwd_channels_per_block();
 
 }  // namespace ssm

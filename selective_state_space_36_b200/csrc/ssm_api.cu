@@ -424,6 +424,151 @@ ssm_status ssm_selective_scan_fwd(ssm_dims dims, ssm_dtype io, const void *u, co
                                      out, last_state, nullptr, stream);
 }
 
+ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, const float *delta_bias, int delta_softplus,
+                                     const float *h0, const void *dout, void *du, void *ddelta,
+                                     void *dz, float *dA, float *dB, float *dC, float *dD,
+                                     float *ddelta_bias, float *dh0, const ssm_scan_opts *opts,
+                                     ssm_stream stream) {
+    g_last_error[0] = 0;
+    size_t es = 0;
+    if (ssm_status s = check_io(io, &es)) return s;
+    if (dims.batch < 0 || dims.seqlen < 0 || dims.dim < 0 || dims.dstate < 0)
+        return fail(SSM_ERR_INVALID_ARG, "negative size (batch %lld, seqlen %lld, dim %lld, dstate %lld)",
+                    (long long)dims.batch, (long long)dims.seqlen, (long long)dims.dim,
+                    (long long)dims.dstate);
+    if (dims.dstate < 1) return fail(SSM_ERR_INVALID_ARG, "dstate must be >= 1");
+    if (dims.dstate > kMaxDstate)
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %lld > %lld", (long long)dims.dstate, (long long)kMaxDstate);
+    if (delta_softplus != 0 && delta_softplus != 1)
+        return fail(SSM_ERR_INVALID_ARG, "delta_softplus must be 0 or 1");
+    int family = ssm::kFamilyAuto;
+    if (opts) {
+        if (opts->variant != SSM_VARIANT_AUTO || opts->segments != 0 || opts->lanes != 0 ||
+            opts->channels_per_lane != 0 || opts->reserved[0] != 0 || opts->reserved[1] != 0)
+            return fail(SSM_ERR_INVALID_ARG, "the backward scan takes only opts.family (other fields must be 0)");
+        if (opts->discretization != SSM_DISCRETIZE_EULER_B)
+            return fail(SSM_ERR_UNSUPPORTED, "the backward scan implements the Euler Bbar only");
+        if (opts->family != SSM_KERNEL_AUTO && opts->family != SSM_KERNEL_GENERIC &&
+            opts->family != SSM_KERNEL_STAGED)
+            return fail(SSM_ERR_INVALID_ARG, "unknown kernel family %d", opts->family);
+        family = opts->family;
+    }
+    const int64_t channels = dims.batch * dims.dim;
+    if (dims.batch != 0 && channels / dims.batch != dims.dim)
+        return fail(SSM_ERR_INVALID_ARG, "batch * dim overflows");
+    if (dims.dim != 0 && dims.dstate != 0 && dims.dim > INT64_MAX / dims.dstate)
+        return fail(SSM_ERR_INVALID_ARG, "dim * dstate overflows");
+    if (channels != 0 && dims.seqlen > INT64_MAX / channels / dims.dstate)
+        return fail(SSM_ERR_INVALID_ARG, "batch * seqlen * dim * dstate overflows");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool has_work = channels != 0 && dims.seqlen != 0;
+    // Parameter gradients are sums: with no work they are zero.  dh0 of an
+    // empty sequence is zero as well (the loss does not depend on h0).
+    if (!has_work) {
+        const size_t dn = (size_t)dims.dim * dims.dstate;
+        const size_t hn = (size_t)channels * dims.dstate;
+        struct Z { void *p; size_t n; } zs[] = {{dA, dn}, {dD, (size_t)dims.dim},
+                                               {ddelta_bias, (size_t)dims.dim}, {dh0, hn}};
+        for (const Z &zz : zs)
+            if (zz.p && zz.n && misaligned(zz.p, 4))
+                return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+        for (const Z &zz : zs) {
+            if (!zz.p || zz.n == 0) continue;
+            cudaError_t e = cudaMemsetAsync(zz.p, 0, zz.n * sizeof(float), st);
+            if (e != cudaSuccess) return cuda_fail(e, "zeroing gradients");
+        }
+        return SSM_OK;
+    }
+    if (!u || !delta || !A || !B || !C || !dout || !du || !ddelta || !dA || !dB || !dC)
+        return fail(SSM_ERR_INVALID_ARG, "u, delta, A, B, C, dout, du, ddelta, dA, dB and dC are required");
+    if ((z != nullptr) != (dz != nullptr)) return fail(SSM_ERR_INVALID_ARG, "dz is required iff z is given");
+    if ((D != nullptr) != (dD != nullptr)) return fail(SSM_ERR_INVALID_ARG, "dD is required iff D is given");
+    if (misaligned(u, es) || misaligned(delta, es) || misaligned(B, es) || misaligned(C, es) ||
+        misaligned(z, es) || misaligned(dout, es) || misaligned(du, es) || misaligned(ddelta, es) ||
+        misaligned(dz, es) || misaligned(A, 4) || misaligned(D, 4) || misaligned(delta_bias, 4) ||
+        misaligned(h0, 4) || misaligned(dA, 4) || misaligned(dB, 4) || misaligned(dC, 4) ||
+        misaligned(dD, 4) || misaligned(ddelta_bias, 4) || misaligned(dh0, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+    const int64_t cpb = ssm::scan_bwd_channels_per_block();
+    if (dims.batch * ((dims.dim + cpb - 1) / cpb) > kMaxGridX)
+        return fail(SSM_ERR_UNSUPPORTED, "grid too large");
+
+    ssm::ScanBwdArgs a{};
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z; a.dout = dout;
+    a.A = A; a.Dskip = D; a.bias = delta_bias; a.h0 = h0;
+    a.du = du; a.ddelta = ddelta; a.dz = dz;
+    a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.dbias = ddelta_bias; a.dh0 = dh0;
+    a.batch = dims.batch; a.seqlen = dims.seqlen; a.dim = dims.dim;
+    a.dstate = (int)dims.dstate;
+    a.softplus = delta_softplus;
+    a.vec_red = dims.dstate % 4 == 0 && !misaligned(dB, 16) && !misaligned(dC, 16);
+
+    // staged pair (checkpointing forward pass + staged reverse pass) where
+    // the rows allow it, else the generic single kernel
+    const bool eligible = ssm::scan_bwd_staged_eligible(a, (int)es);
+    if (family == ssm::kFamilyStaged && !eligible)
+        return fail(SSM_ERR_UNSUPPORTED, "staged backward needs dstate <= 16 and 16-byte aligned rows "
+                    "(dim and dstate times the element size multiples of 16, pointers 16-byte aligned)");
+    const bool staged = eligible && family != ssm::kFamilyGeneric;
+    int ns = 0, g = 0;
+    if (staged) {
+        const DeviceInfo di = device_info();
+        scan_layout(dims.dstate, channels, di.sms, 0, &ns, &g);
+        if (ssm::staged_smem_bytes(io == SSM_BF16, ns, g, 1) > (size_t)di.smem_optin)
+            return fail(SSM_ERR_UNSUPPORTED, "staged backward needs more shared memory than the device has");
+    }
+
+    const size_t bln = (size_t)dims.batch * dims.seqlen * dims.dstate;
+    struct Z { void *p; size_t n; } zs[] = {{dA, (size_t)dims.dim * dims.dstate}, {dB, bln}, {dC, bln},
+                                           {dD, (size_t)dims.dim}, {ddelta_bias, (size_t)dims.dim}};
+    for (const Z &zz : zs) {
+        if (!zz.p) continue;
+        cudaError_t e = cudaMemsetAsync(zz.p, 0, zz.n * sizeof(float), st);
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing gradients");
+    }
+    const int64_t kc = staged ? ssm::scan_bwd_staged_chunk() : ssm::scan_bwd_chunk((int)dims.dstate);
+    const size_t ws_bytes = (size_t)channels * ((dims.seqlen + kc - 1) / kc) * dims.dstate * sizeof(float);
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, ws_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "checkpoint workspace allocation");
+    a.ckpt = static_cast<float *>(ws);
+    if (staged) {
+        ssm::ScanArgs f{};
+        f.u = u; f.delta = delta; f.B = B; f.C = C; f.z = nullptr;
+        f.A = A; f.Dskip = nullptr; f.bias = delta_bias;
+        f.out = nullptr;
+        f.last_state = const_cast<float *>(h0);  // read as h_0, not written in checkpoint mode
+        f.batch = dims.batch; f.seqlen = dims.seqlen; f.dim = dims.dim;
+        f.dstate = (int)dims.dstate;
+        f.softplus = delta_softplus;
+        f.seg_len = dims.seqlen;
+        f.nseg = 1;
+        f.ckpt = a.ckpt;
+        f.ckpt_every = (int)kc;
+        e = ssm::launch_scan_staged(f, io == SSM_BF16, ns, g, 1, ssm::kVariantCkpt, st);
+        if (e == cudaSuccess) e = ssm::launch_scan_bwd_staged(a, io == SSM_BF16, st);
+    } else {
+        e = ssm::launch_scan_bwd(a, io == SSM_BF16, st);
+    }
+    cudaError_t ef = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward scan launch");
+    if (ef != cudaSuccess) return cuda_fail(ef, "workspace release");
+    return SSM_OK;
+}
+
+ssm_status ssm_selective_scan_bwd(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                  const float *A, const void *B, const void *C, const float *D,
+                                  const void *z, const float *delta_bias, int delta_softplus,
+                                  const float *h0, const void *dout, void *du, void *ddelta,
+                                  void *dz, float *dA, float *dB, float *dC, float *dD,
+                                  float *ddelta_bias, float *dh0, ssm_stream stream) {
+    return ssm_selective_scan_bwd_ex(dims, io, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0,
+                                     dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0, nullptr,
+                                     stream);
+}
+
 ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state, const void *x,
                                       const void *dt, const float *A, const void *B, const void *C,
                                       const float *D, const void *z, void *out, ssm_stream stream) {

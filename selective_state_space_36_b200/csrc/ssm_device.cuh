@@ -32,6 +32,7 @@ template <> struct io_traits<float> {
         v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
     }
     static __device__ __forceinline__ void store(float *p, float v) { __stcs(p, v); }
+    static __device__ __forceinline__ void store_smem(float *p, float v) { *p = v; }
 };
 
 template <> struct io_traits<__nv_bfloat16> {
@@ -55,6 +56,7 @@ template <> struct io_traits<__nv_bfloat16> {
         __nv_bfloat16 b = __float2bfloat16_rn(v);
         __stcs(reinterpret_cast<unsigned short *>(p), *reinterpret_cast<unsigned short *>(&b));
     }
+    static __device__ __forceinline__ void store_smem(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
 };
 
 // ------------------------------------------------------------- SFU wrappers

@@ -43,7 +43,7 @@ CHUNK_ROWS = 4096
 
 # stream identifiers: one independent PCG64 family per drawn quantity
 _TID = {"param": 0, "u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "h0": 6,
-        "x": 7, "dt": 8, "dB": 9, "dC": 10, "dz": 11}
+        "x": 7, "dt": 8, "dB": 9, "dC": 10, "dz": 11, "dout": 12}
 
 SEQ_NAMES = ("u", "delta", "z", "B", "C")
 
@@ -265,6 +265,13 @@ def scan_inputs(cfg: ScanConfig, t0: int = 0, t1: Optional[int] = None,
                  if cfg.h0_sigma is not None else None)
     res["delta_softplus"] = cfg.softplus
     return res
+
+
+def draw_dout(cfg: ScanConfig, t0: int = 0, t1: Optional[int] = None,
+              threads: int = 0) -> np.ndarray:
+    """Upstream gradient of the scan output: (batch, t1 - t0, dim) ~ N(0, 1)
+    in I/O representation, from its own stream (the loss is sum(dout * out))."""
+    return draw_tensor(cfg, "dout", t0, t1, threads)
 
 
 # --------------------------------------------------------------------------

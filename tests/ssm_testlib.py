@@ -116,3 +116,73 @@ def channel_subset(x: dict, dims_idx, batch_idx=None) -> dict:
         else:
             sub[k] = v
     return sub
+
+
+# ------------------------------------------------------------------ backward
+# Gradients are compared row by row (rows = every index but the last axis)
+# with a norm-wise bound, max_j |g - g_ref| <= tol * max_j |g_ref|, for the
+# same reason as the bf16 state: single entries of a gradient cross zero.
+# The bounds (derivation with the backward kernel's description):
+#   io outputs du, ddelta, dz: bf16 rounding of the result (2^-9 relative)
+#   dominates, so 1e-2 for bf16; float32 sums (dA, dB, dC, dD, ddelta_bias,
+#   dh0) and every fp32-I/O output carry only fp32 arithmetic, whose error in
+#   the adjoint grows at most linearly with the decay's memory 1/(Delta |A|)
+#   (<= ~1e3 steps at these inputs, i.e. <= ~6e-5 relative): 1e-4.
+TOL_GRAD = {"io": {"f32": 1e-4, "bf16": 1e-2}, "f32": {"f32": 1e-4, "bf16": 1e-4}}
+GRAD_IO = ("du", "ddelta", "dz")
+GRAD_F32 = ("dA", "dB", "dC", "dD", "ddelta_bias", "dh0")
+
+
+def grad_err(got, ref) -> float:
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    if got.size == 0:
+        return 0.0
+    g2 = got.reshape(-1, got.shape[-1]) if got.ndim > 1 else got.reshape(1, -1)
+    r2 = ref.reshape(-1, ref.shape[-1]) if ref.ndim > 1 else ref.reshape(1, -1)
+    floor = 1e-6 * float(np.max(np.abs(r2))) + 1e-30
+    num = np.max(np.abs(g2 - r2), axis=1)
+    den = np.max(np.abs(r2), axis=1) + floor
+    return float(np.max(num / den))
+
+
+def grad_keys(x: dict):
+    """The gradients a call with these inputs returns (dh0 requested)."""
+    ks = ["du", "ddelta", "dA", "dB", "dC", "dh0"]
+    ks += ["dz"] if x.get("z") is not None else []
+    ks += ["dD"] if x.get("D") is not None else []
+    ks += ["ddelta_bias"] if x.get("delta_bias") is not None else []
+    return ks
+
+
+def check_grads(got: dict, ref: dict, io: str, keys) -> dict:
+    errs = {}
+    for k in keys:
+        assert got.get(k) is not None, f"{k}: not returned"
+        g = from_dev(got[k])
+        assert g.shape == ref[k].shape, f"{k}: shape {g.shape} != {ref[k].shape}"
+        assert np.all(np.isfinite(g)), f"{k}: non-finite values"
+        tol = TOL_GRAD["io" if k in GRAD_IO else "f32"][io]
+        e = grad_err(g, ref[k])
+        assert e <= tol, f"{k}: max row-wise rel err {e:.3e} > {tol:.0e}"
+        errs[k] = e
+    return errs
+
+
+def oracle_bwd(x: dict, io: str, dout):
+    """Oracle gradients on the exact fp64 values of scan_inputs() + dout."""
+    return oracle.scan_bwd(f64(x["u"], io), f64(x["delta"], io), f64(x["A"], "f32"), f64(x["B"], io),
+                           f64(x["C"], io), f64(dout, io), D=f64(x["D"], "f32"), z=f64(x["z"], io),
+                           delta_bias=f64(x["delta_bias"], "f32"), delta_softplus=x["delta_softplus"],
+                           h0=f64(x["h0"], "f32"))
+
+
+def gpu_bwd(x: dict, io: str, dout, want_dh0=True, family="auto"):
+    """Library backward on device copies of scan_inputs() + dout."""
+    from selective_state_space_36_b200 import binding
+    d = {k: to_dev(v, io) for k, v in x.items() if isinstance(v, np.ndarray)}
+    g = binding.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], to_dev(dout, io),
+                                   D=d.get("D"), z=d.get("z"), delta_bias=d.get("delta_bias"),
+                                   delta_softplus=x["delta_softplus"], h0=d.get("h0"),
+                                   want_dh0=want_dh0, family=family)
+    torch.cuda.synchronize()
+    return g

@@ -119,3 +119,51 @@ def test_python_binding_rejects_bad_tensors(b):
         b.selective_scan_fwd(u.double(), u.double(), A, torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
     with pytest.raises(ValueError):
         b.selective_scan_fwd(u, u[:, :2], A, torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
+
+
+def _bwd(b, dims, io=1, opts=None, softplus=1, **kw):
+    # inputs u, delta, A, B, C, D, z, bias; h0, dout; outputs du, ddelta, dz,
+    # dA, dB, dC, dD, ddelta_bias, dh0 -- distinct fake, 256-byte aligned addresses
+    names = ["u", "delta", "A", "B", "C", "D", "z", "bias", "h0", "dout", "du", "ddelta", "dz",
+             "dA", "dB", "dC", "dD", "dbias", "dh0"]
+    p = {n: 0x100000 * (i + 1) for i, n in enumerate(names)}
+    for n in ("D", "z", "bias", "h0", "dz", "dD", "dbias", "dh0"):
+        p[n] = None
+    p.update(kw)
+    args = [b.SSMDims(*dims), io] + [p[n] for n in names[:8]] + [softplus] + [p[n] for n in names[8:]]
+    if opts is None:
+        return b.lib.ssm_selective_scan_bwd(*args, None)
+    return b.lib.ssm_selective_scan_bwd_ex(*args, ctypes.byref(opts), None)
+
+
+def test_bwd_argument_validation(b):
+    ok = (2, 16, 64, 16)
+    assert _bwd(b, ok, io=3) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, (2, 16, 64, 65)) == b.SSM_ERR_UNSUPPORTED
+    assert _bwd(b, (2, -16, 64, 16)) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, softplus=5) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, dout=None) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, dB=None) == b.SSM_ERR_INVALID_ARG
+    # dz exactly when z, dD exactly when D
+    assert _bwd(b, ok, z=0x7000000) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, dz=0x7000000) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, D=0x7000000) == b.SSM_ERR_INVALID_ARG
+    assert b"dD" in b.lib.ssm_last_error()
+    assert _bwd(b, ok, du=0x7000001) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, dA=0x7000002) == b.SSM_ERR_INVALID_ARG
+    assert b"aligned" in b.lib.ssm_last_error()
+    # options: only the kernel family may be set; ZOH has no backward
+    assert _bwd(b, ok, opts=b.SSMScanOpts(1)) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, opts=b.SSMScanOpts(0, 0, 0, 9)) == b.SSM_ERR_INVALID_ARG
+    assert _bwd(b, ok, opts=b.SSMScanOpts(0, 0, 0, 0, 0, 1)) == b.SSM_ERR_UNSUPPORTED
+    # the staged family on rows that are not 16-byte multiples, or N > 16
+    assert _bwd(b, (2, 16, 37, 16), opts=b.SSMScanOpts(0, 0, 0, 2)) == b.SSM_ERR_UNSUPPORTED
+    assert _bwd(b, (2, 16, 64, 32), opts=b.SSMScanOpts(0, 0, 0, 2)) == b.SSM_ERR_UNSUPPORTED
+    assert b"staged backward" in b.lib.ssm_last_error()
+
+
+def test_bwd_empty_sizes_without_outputs_are_noops(b):
+    none = dict(u=None, delta=None, A=None, B=None, C=None, dout=None, du=None, ddelta=None,
+                dA=None, dB=None, dC=None)
+    for dims in [(0, 16, 8, 16), (2, 0, 8, 16), (2, 16, 0, 16)]:
+        assert _bwd(b, dims, **none) == b.SSM_OK

@@ -1,0 +1,145 @@
+"""GPU parity of ssm_selective_scan_bwd against the fp64 oracle backward.
+
+The oracle's backward is pinned on the CPU (central differences of the oracle
+scan, torch autograd on an fp64 restatement, planted mistakes); here every
+gradient the library returns is compared with it on the same seeded inputs,
+for both kernel families -- the generic single kernel and the staged pair
+(checkpointing forward pass + staged reverse pass): shapes spanning several
+checkpoint chunks, staged chunks, 32-channel blocks and ragged tails, every
+state-size layout, each optional input absent or present, and the Mamba-1.4B
+workload's launch configuration on a channel subset.
+"""
+import numpy as np
+import pytest
+import torch
+
+from selective_state_space_36_b200 import inputs as I
+from tests import ssm_testlib as T
+
+pytestmark = pytest.mark.gpu
+FAMILIES = ["generic", "staged"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from selective_state_space_36_b200 import binding
+    return binding
+
+
+def _case(io, batch, L, dim, N, seed, **kw):
+    cfg = I.ScanConfig("bwd", batch, L, dim, N, io=io, seed=seed, **kw)
+    return cfg, I.scan_inputs(cfg), I.draw_dout(cfg)
+
+
+def _check(io, batch, L, dim, N, seed, family="auto", positive_bias=False, **kw):
+    cfg, x, dout = _case(io, batch, L, dim, N, seed, **kw)
+    if positive_bias:
+        # without softplus Delta = raw + bias: keep it small and positive
+        x["delta_bias"] = np.abs(x["delta_bias"]).astype(np.float32) * 0.01
+    got = T.gpu_bwd(x, io, dout, family=family)
+    ref = T.oracle_bwd(x, io, dout)
+    errs = T.check_grads(got, ref, io, T.grad_keys(x))
+    print(f"[bwd {family} {io} B{batch} L{L} D{dim} N{N} {kw}] "
+          + " ".join(f"{k}={v:.1e}" for k, v in errs.items()))
+    return errs
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_bwd_small_all_inputs(io, family):
+    # L = 100: several checkpoint and staged chunks and a ragged one; dim = 40:
+    # one full 32-channel block and a ragged one
+    _check(io, 2, 100, 40, 16, 11, family=family, h0_sigma=0.5)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [1, 3, 4, 7, 8, 12, 16, 17, 24, 32, 33, 48, 64])
+def test_bwd_state_sizes_generic(io, N):
+    _check(io, 1, 37, 33, N, 100 + N, family="generic", h0_sigma=0.3)
+
+
+@pytest.mark.parametrize("io,N", [("f32", 4), ("f32", 8), ("f32", 12), ("f32", 16),
+                                  ("bf16", 8), ("bf16", 16)])
+def test_bwd_state_sizes_staged(io, N):
+    # every staged-eligible state size; L = 77 ends mid-chunk and mid-sub-chunk
+    _check(io, 2, 77, 72, N, 200 + N, family="staged", h0_sigma=0.3)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("opt", [dict(has_z=False), dict(has_d=False), dict(has_bias=False),
+                                 dict(softplus=False, delta_sigma=0.02, positive_bias=True),
+                                 dict(h0_sigma=None), dict(has_z=False, has_d=False, has_bias=False)])
+def test_bwd_optional_inputs(io, opt, family):
+    _check(io, 2, 45, 40, 16, 7, family=family, **opt)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("L", [1, 2, 7, 8, 9, 15, 16, 17, 32, 33, 64, 65])
+def test_bwd_lengths(L, family):
+    _check("f32", 1, L, 32, 16, 300 + L, family=family, h0_sigma=0.5)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+def test_bwd_long_memory_fp32(family):
+    # small Delta: the adjoint carries over ~1e3 steps
+    _check("f32", 1, 1500, 64, 16, 21, family=family, dt_min=1e-3, dt_max=2e-3, h0_sigma=0.5)
+
+
+@pytest.mark.slow
+def test_bwd_mamba1p4b_launch_shape_subset():
+    # the Mamba-1.4B workload's launch configuration (batch 8, L 2048, bf16,
+    # N 16) on 256 of its channels, all gradients against the oracle
+    cfg = I.MAMBA1P4B.with_(dim=256)
+    x, dout = I.scan_inputs(cfg), I.draw_dout(cfg)
+    got = T.gpu_bwd(x, "bf16", dout)
+    ref = T.oracle_bwd(x, "bf16", dout)
+    errs = T.check_grads(got, ref, "bf16", T.grad_keys(x))
+    print("[bwd 1.4B subset] " + " ".join(f"{k}={v:.1e}" for k, v in errs.items()))
+
+
+def test_bwd_families_agree_mid_size():
+    # the two families on a shape too large for the oracle to take quickly
+    cfg, x, dout = _case("bf16", 4, 1000, 512, 16, 9, h0_sigma=0.5)
+    g = T.gpu_bwd(x, "bf16", dout, family="generic")
+    s = T.gpu_bwd(x, "bf16", dout, family="staged")
+    for k in T.grad_keys(x):
+        e = T.grad_err(T.from_dev(s[k]), T.from_dev(g[k]))
+        tol = T.TOL_GRAD["io" if k in T.GRAD_IO else "f32"]["bf16"]
+        assert e <= tol, (k, e)
+
+
+def test_bwd_staged_rejects_ineligible_rows(lib):
+    cfg, x, dout = _case("bf16", 1, 10, 33, 16, 1)
+    with pytest.raises(lib.SSMError) as ei:
+        T.gpu_bwd(x, "bf16", dout, family="staged")
+    assert ei.value.status == lib.SSM_ERR_UNSUPPORTED
+
+
+def test_bwd_empty_shapes(lib):
+    for (b, L, d) in [(0, 5, 8), (2, 0, 8), (2, 5, 0)]:
+        dev = "cuda"
+        u = torch.zeros((b, L, d), device=dev)
+        A = -torch.ones((d, 4), device=dev)
+        Bm = torch.zeros((b, L, 4), device=dev)
+        D = torch.ones(d, device=dev)
+        g = lib.selective_scan_bwd(u, u, A, Bm, Bm, u, D=D, z=u, delta_bias=torch.zeros(d, device=dev),
+                                   want_dh0=True)
+        torch.cuda.synchronize()
+        for k in ("dA", "dD", "ddelta_bias", "dh0"):
+            assert torch.all(g[k] == 0), k
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+def test_bwd_is_linear_in_dout(family):
+    # the gradients are linear in dout: g(dout1 + dout2) = g(dout1) + g(dout2),
+    # up to fp32 rounding, on a shape the oracle would take long on
+    cfg, x, d1 = _case("f32", 2, 700, 200, 16, 5, h0_sigma=0.5)
+    d2 = I.draw_dout(cfg.with_(seed=6))
+    g1, g2, g12 = (T.gpu_bwd(x, "f32", d, family=family) for d in (d1, d2, d1 + d2))
+    for k in ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias"):
+        ref = T.from_dev(g1[k]) + T.from_dev(g2[k])
+        e = T.grad_err(T.from_dev(g12[k]), ref)
+        assert e <= 1e-4, (k, e)
