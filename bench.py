@@ -6,13 +6,14 @@ softplus(Delta), discretisation, recurrence, readout, D skip, silu(z) gate, the
 fp32 state in and out.  Inputs are seeded synthetic data of that shape.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload mamba1p4b|mamba130m|longseq|decode]
+                  [--workload mamba1p4b|mamba130m|longseq|decode|mamba1p4b_bwd]
 
 The other workloads measure the remaining hot-path kernels the same way:
 mamba130m (batch 8, L 2048, dim 1536), longseq (batch 1, L 1,048,576, dim 1536:
 the sequence-split variant) and decode (one ssm_selective_state_update step at
 batch 256, dim 5120, N 16; two state buffers alternate so that the 84 MB state
-cannot simply stay in the 126 MB L2).
+cannot simply stay in the 126 MB L2) and mamba1p4b_bwd (one
+ssm_selective_scan_bwd call on the 1.4B-layer workload with a seeded dout).
 
 Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of
 the workload on its GPU (independent batches, no collective on the data path:
@@ -45,13 +46,35 @@ UNIT = "Gelem/s"
 WORKLOAD = I.MAMBA1P4B
 L2_BYTES = 126 * 1024 * 1024
 WORKLOADS = {"mamba1p4b": I.MAMBA1P4B, "mamba130m": I.MAMBA130M, "longseq": I.LONGSEQ,
-             "decode": I.DECODE}
+             "decode": I.DECODE, "mamba1p4b_bwd": I.MAMBA1P4B}
 SCAN_METRICS = {
     "mamba1p4b": METRIC,
     "mamba130m": "selective-scan fwd Gelem/s (B·L·D) at 130M-layer shape; % of HBM roofline",
     "longseq": "selective-scan fwd Gelem/s (B·L·D) at L=1,048,576 (sequence split); % of HBM roofline",
 }
 DECODE_METRIC = "decode state-update steps/s at batch 256, dim 5120, N 16; % of HBM roofline"
+BWD_METRIC = "selective-scan bwd Gelem/s (B·L·D) at 1.4B-layer shape"
+
+
+def bwd_sfu_ceiling_per_sm_clock(dstate: int = 16) -> float:
+    """Elements per SM clock the backward's SFU work allows (the SFU delivers
+    16 results per SM clock): the checkpointing forward pass needs dstate
+    decays and the softplus exponential per element, the reverse pass the
+    dstate decays again (recomputed), the softplus exponential, and an
+    exponential and a reciprocal for each of sigmoid(z) and sigmoid(delta +
+    bias).  An upper bound: it ignores the issue slots the rest takes."""
+    return 16.0 / ((dstate + 1) + (dstate + 1 + 4))
+
+
+def bwd_algorithmic_bytes(cfg: I.ScanConfig, ckpt_every: int = 8) -> int:
+    """Bytes the backward must move: u, delta read twice (both passes), z,
+    dout, B, C read and du, ddelta, dz written once, dB, dC written in fp32,
+    and the state checkpoints written and read once."""
+    es = 2 if cfg.io == "bf16" else 4
+    seq = cfg.elements * es * (2 * 2 + 2 + 3)
+    bc = cfg.batch * cfg.seqlen * cfg.dstate * (es * 3 + 4 * 2)
+    ck = cfg.batch * cfg.dim * ((cfg.seqlen + ckpt_every - 1) // ckpt_every) * cfg.dstate * 4 * 2
+    return seq + bc + ck
 
 
 def alu_ceiling_per_sm_clock(dstate: int = 16) -> float:
@@ -532,6 +555,72 @@ def run_decode(args, rank, world, dev):
     return 0
 
 
+def run_bwd(args, rank, world, dev):
+    """One step = one ssm_selective_scan_bwd over the 1.4B-layer workload with a
+    seeded upstream gradient dout (both kernels, the zeroing of the summed
+    gradients and the checkpoint workspace are inside the step)."""
+    import torch
+    from selective_state_space_36_b200 import binding as lib
+
+    cfg = WORKLOADS[args.workload]
+    if rank:
+        cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
+    if args.batch or args.seqlen:
+        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
+        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"{args.workload}_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
+    d = _scan_device_inputs(cfg, dev)
+    dout = torch.empty_like(d["u"])
+    for b in range(cfg.batch):
+        for t0, t1 in I.iter_time_blocks(cfg.seqlen, 1 << 16):
+            dout[b, t0:t1].copy_(_upload(I.draw_rows(cfg, "dout", b, t0, t1), dev))
+    h0 = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lib.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], dout, D=d["D"], z=d["z"],
+                               delta_bias=d["delta_bias"], h0=h0, stream=stream)
+
+    elapsed_ms, call_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
+    ms_per_step = elapsed_ms / args.steps
+    value = whole_job_rate(world, cfg.elements, ms_per_step)
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"metric": BWD_METRIC, "value": value, "unit": UNIT, "kernel_ms": call_ms,
+                              "config": {"workload": cfg.name},
+                              "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
+        return 0
+    if rank == 0:
+        peaks = measured_peaks()
+        sm_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sfu_peak = bwd_sfu_ceiling_per_sm_clock(cfg.dstate) * sms * sm_mhz * 1e6 / 1e9
+        call_gelem = cfg.elements / (call_ms * 1e-3) / 1e9
+        abytes = bwd_algorithmic_bytes(cfg)
+        line = _base_line(BWD_METRIC, UNIT, value, world, args, ms_per_step)
+        line.update({
+            "config": {"workload": cfg.name + "_bwd", "batch": cfg.batch, "seqlen": cfg.seqlen,
+                       "dim": cfg.dim, "dstate": cfg.dstate, "io": cfg.io,
+                       "per_gpu": "one full workload per GPU",
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"inputs {abytes / 1e6:.0f} MB moved per call > {L2_BYTES >> 20} MB L2; no flush"},
+            "roofline": {
+                "bound": "alu", "achieved": call_gelem, "peak": sfu_peak, "unit": "Gelem/s",
+                "frac": call_gelem / sfu_peak, "traffic": None, "kernel_ms": call_ms,
+                "scope": "the whole backward call (checkpointing forward pass + reverse pass)",
+                "peak_source": (f"derived SFU bound: {bwd_sfu_ceiling_per_sm_clock(cfg.dstate):.3f} elem/clk/SM"
+                                f" x {sms} SMs x {sm_mhz:.0f} MHz"),
+                "hbm": {"achieved": abytes / (call_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": abytes / (call_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "algorithmic_bytes_per_call": abytes,
+                        "peak_source": peaks["source"] + " (copy bandwidth)"}},
+            "e2e": None,
+            "gpu_launches": args.steps * 2,
+            "clocks": clocks,
+        })
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> int:
     import torch
     import torch.distributed as dist
@@ -542,6 +631,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
     try:
         if args.workload == "decode":
             return run_decode(args, rank, world, dev)
+        if args.workload == "mamba1p4b_bwd":
+            return run_bwd(args, rank, world, dev)
         return run_scan(args, rank, world, dev)
     finally:
         if world > 1:

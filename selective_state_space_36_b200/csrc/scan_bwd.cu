@@ -310,7 +310,11 @@ struct BwdStagedLayout {
     static constexpr int RAW = T * NSP;                   // raw B or C rows (elements)
     static constexpr size_t STAGE_BYTES = (4 * (size_t)TILE + 2 * RAW) * sizeof(IO);
     static constexpr size_t BC_BYTES = 2 * (size_t)T * NSP * sizeof(float);
-    static constexpr size_t RED_BYTES = 2 * (size_t)KC * CPB * NSP * sizeof(float);
+    // reduction tile [2 (dC, dB)][KC][CPB][NSP]; each step's slab is padded by
+    // 16 floats so that the reading threads of a quarter-warp (4 state
+    // columns x 2 steps) fall in different banks
+    static constexpr int KSTRIDE = CPB * NSP + 16;
+    static constexpr size_t RED_BYTES = 2 * (size_t)KC * KSTRIDE * sizeof(float);
     static constexpr size_t SMEM = S * STAGE_BYTES + BC_BYTES + RED_BYTES;
     static_assert(T % KC == 0 && KC % G == 0, "chunks hold whole sub-chunks of whole step groups");
 };
@@ -338,7 +342,8 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
     extern __shared__ __align__(16) unsigned char smem[];
     float *fB = reinterpret_cast<float *>(smem + S * Lay::STAGE_BYTES);
     float *fC = fB + T * NSP;
-    float *sred = fC + T * NSP;            // [2 (dC, dB)][KC][CPB][NSP]
+    float *sred = fC + T * NSP;            // [2 (dC, dB)][KC] slabs of [CPB][NSP], KSTRIDE apart
+    constexpr int KSTRIDE = Lay::KSTRIDE;
 
     const int64_t L = args.seqlen, Dm = args.dim;
     const int N = args.dstate;
@@ -409,6 +414,16 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) { lam2[p] = make_float2(0.f, 0.f); dA2[p] = make_float2(0.f, 0.f); }
     float dD_acc = 0.f, dbias_acc = 0.f;
+    // the checkpoint of the first sub-chunk processed (the last one in time)
+    float2 hc_next[NS / 2];
+    {
+        const float *cp = ck_lane + (nck - 1) * Dm * N;
+#pragma unroll
+        for (int p = 0; p < NS / 2; ++p) {
+            const int n = q * NS + 2 * p;
+            hc_next[p] = make_float2((active && n < N) ? cp[2 * p] : 0.f, (active && n + 1 < N) ? cp[2 * p + 1] : 0.f);
+        }
+    }
 
 #pragma unroll
     for (int o = 0; o < S - 1; ++o) {
@@ -425,39 +440,55 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
         IO *st = stage_ptr(o % S);
         {
             const IO *rb = st + 4 * TILE, *rc = rb + Lay::RAW;
-            for (int i = tid; i < T * NSP; i += kBlock) {
-                const int r = i / NSP, n = i % NSP;
-                const bool ok = r < rows && n < N;
-                fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
-                fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+            if (rows == T && N == NSP) {
+                for (int i = 4 * tid; i < T * NSP; i += 4 * kBlock) {
+                    float v[4];
+                    io::load4_smem(rb + i, v);
+                    *reinterpret_cast<float4 *>(fB + i) = make_float4(v[0], v[1], v[2], v[3]);
+                    io::load4_smem(rc + i, v);
+                    *reinterpret_cast<float4 *>(fC + i) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            } else {
+                for (int i = tid; i < T * NSP; i += kBlock) {
+                    const int r = i / NSP, n = i % NSP;
+                    const bool ok = r < rows && n < N;
+                    fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
+                    fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+                }
             }
         }
         __syncthreads();
-        IO *su = st + grp, *sd = st + TILE + grp, *sz = st + 2 * TILE + grp, *sg = st + 3 * TILE + grp;
-        const int nsub = (rows + KC - 1) / KC;
-        for (int sc = nsub - 1; sc >= 0; --sc) {
-            const int k0 = sc * KC;
+        // this lane's rows of the tiles start at step q
+        IO *su = st + grp + q * ROW, *sd = st + TILE + grp + q * ROW;
+        IO *sz = st + 2 * TILE + grp + q * ROW, *sg = st + 3 * TILE + grp + q * ROW;
+        const float *fBq = fB + q * NS, *fCq = fC + q * NS;
+        float *sredq = sred + grp * NSP + q * NS;
+
+        // One sub-chunk of KC steps starting at chunk row k0 (nrows: the rows
+        // of this chunk; the constant T for full chunks).
+        auto sub_chunk = [&](const int k0, const int nrows) {
             const int64_t t0 = tc + k0;
-            // state entering step t0
             float2 hc[NS / 2];
-            {
-                const float *cp = ck_lane + (t0 / KC) * Dm * N;
+#pragma unroll
+            for (int p = 0; p < NS / 2; ++p) hc[p] = hc_next[p];
+            if (t0 >= KC) {  // prefetch the checkpoint of the sub-chunk processed next
+                const float *cp = ck_lane + (t0 / KC - 1) * Dm * N;
 #pragma unroll
                 for (int p = 0; p < NS / 2; ++p) {
                     const int n = q * NS + 2 * p;
-                    hc[p] = make_float2((active && n < N) ? cp[2 * p] : 0.f,
-                                        (active && n + 1 < N) ? cp[2 * p + 1] : 0.f);
+                    hc_next[p] = make_float2((active && n < N) ? cp[2 * p] : 0.f,
+                                             (active && n + 1 < N) ? cp[2 * p + 1] : 0.f);
                 }
             }
-            // ---- per-step scalars of the owned steps r = k0 + j G + q
+            // ---- per-step scalars of the owned steps k0 + j G + q
             float uo[KG], so[KG], zo[KG], go[KG], szo[KG], dlo[KG], duo[KG], dyo[KG];
 #pragma unroll
             for (int j = 0; j < KG; ++j) {
-                const int r = k0 + j * G + q;
-                uo[j] = io::load_smem(su + r * ROW);
-                so[j] = io::load_smem(sd + r * ROW) + bias;
-                zo[j] = pz ? io::load_smem(sz + r * ROW) : 0.f;
-                go[j] = io::load_smem(sg + r * ROW);
+                const int rr = k0 + j * G;
+                uo[j] = io::load_smem(su + rr * ROW);
+                so[j] = io::load_smem(sd + rr * ROW) + bias;
+                zo[j] = pz ? io::load_smem(sz + rr * ROW) : 0.f;
+                go[j] = io::load_smem(sg + rr * ROW);
             }
             if (args.softplus) {
                 if (!PRECISE && KG % 2 == 0) {
@@ -477,7 +508,7 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             }
 #pragma unroll
             for (int j = 0; j < KG; ++j) {
-                if (k0 + j * G + q >= rows || !active) { dlo[j] = 0.f; go[j] = 0.f; }
+                if (k0 + j * G + q >= nrows || !active) { dlo[j] = 0.f; go[j] = 0.f; }
                 duo[j] = dlo[j] * uo[j];
                 if (pz) {
                     szo[j] = sigmoid_of<PRECISE>(zo[j]);
@@ -499,7 +530,7 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                 for (int p = 0; p < NS / 2; ++p) h2[p] = hc[p];
 #pragma unroll
                 for (int k = 0; k < KC; ++k) {
-                    const float4 bv = *reinterpret_cast<const float4 *>(fB + (k0 + k) * NSP + q * NS);
+                    const float4 bv = *reinterpret_cast<const float4 *>(fBq + (k0 + k) * NSP);
                     const float2 d2 = make_float2(dl[k], dl[k]), u2 = make_float2(du[k], du[k]);
 #pragma unroll
                     for (int p = 0; p < NS / 2; ++p) {
@@ -517,8 +548,8 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             float ddl_p[KC], dub_p[KC], y_p[KC];
 #pragma unroll
             for (int k = KC - 1; k >= 0; --k) {
-                const float4 bv = *reinterpret_cast<const float4 *>(fB + (k0 + k) * NSP + q * NS);
-                const float4 cv = *reinterpret_cast<const float4 *>(fC + (k0 + k) * NSP + q * NS);
+                const float4 bv = *reinterpret_cast<const float4 *>(fBq + (k0 + k) * NSP);
+                const float4 cv = *reinterpret_cast<const float4 *>(fCq + (k0 + k) * NSP);
                 const float2 dy2 = make_float2(dy[k], dy[k]), dl2 = make_float2(dl[k], dl[k]);
                 const float2 du2 = make_float2(du[k], du[k]);
                 float2 accy = make_float2(0.f, 0.f), accd = accy, accb = accy, pc[NS / 2], pb[NS / 2];
@@ -538,10 +569,9 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                     dA2[p] = fma2(ga, dl2, dA2[p]);
                     lam2[p] = la;
                 }
-                float *rc = sred + ((size_t)(0 * KC + k) * CPB + grp) * NSP + q * NS;
-                float *rbp = sred + ((size_t)(1 * KC + k) * CPB + grp) * NSP + q * NS;
-                *reinterpret_cast<float4 *>(rc) = make_float4(pc[0].x, pc[0].y, pc[1].x, pc[1].y);
-                *reinterpret_cast<float4 *>(rbp) = make_float4(pb[0].x, pb[0].y, pb[1].x, pb[1].y);
+                *reinterpret_cast<float4 *>(sredq + k * KSTRIDE) = make_float4(pc[0].x, pc[0].y, pc[1].x, pc[1].y);
+                *reinterpret_cast<float4 *>(sredq + (KC + k) * KSTRIDE) =
+                    make_float4(pb[0].x, pb[0].y, pb[1].x, pb[1].y);
                 ddl_p[k] = accd.x + accd.y;
                 dub_p[k] = accb.x + accb.y;
                 y_p[k] = accy.x + accy.y;
@@ -552,16 +582,16 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             reduce_scatter_steps<KC, G>(y_p, y_o, q);
 #pragma unroll
             for (int j = 0; j < KG; ++j) {
-                const int r = k0 + j * G + q;
-                if (r < rows && active) {
+                const int rr = k0 + j * G;
+                if (rr + q < nrows && active) {
                     const float dub = dub_o[j];
                     const float ddl = fmaf(uo[j], dub, ddl_o[j]);
                     const float dd = args.softplus ? ddl * sigmoid_of<PRECISE>(so[j]) : ddl;
-                    io::store_smem(su + r * ROW, fmaf(dyo[j], dskip, dlo[j] * dub));
-                    io::store_smem(sd + r * ROW, dd);
+                    io::store_smem(su + rr * ROW, fmaf(dyo[j], dskip, dlo[j] * dub));
+                    io::store_smem(sd + rr * ROW, dd);
                     if (pz) {
                         const float y = fmaf(dskip, uo[j], y_o[j]);
-                        io::store_smem(sz + r * ROW, go[j] * y * szo[j] * (1.f + zo[j] * (1.f - szo[j])));
+                        io::store_smem(sz + rr * ROW, go[j] * y * szo[j] * (1.f + zo[j] * (1.f - szo[j])));
                     }
                     dbias_acc += dd;
                     dD_acc = fmaf(dyo[j], uo[j], dD_acc);
@@ -573,19 +603,21 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                 const int nq = tid % NQ;
                 const int kk = (tid / NQ) % KC;
                 const int which = tid / (NQ * KC);  // 0: dC, 1: dB
-                const float4 *col = reinterpret_cast<const float4 *>(sred) + (size_t)(which * KC + kk) * CPB * NQ + nq;
-                float2 a01 = make_float2(0.f, 0.f), a23 = a01;
-#pragma unroll 8
-                for (int cc = 0; cc < CPB; ++cc) {
-                    // rows of a quarter-warp start at different channels: no bank conflicts
-                    const float4 v = col[(size_t)((cc + kk) & (CPB - 1)) * NQ];
+                const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) + nq;
+                float2 a01 = make_float2(0.f, 0.f), a23 = a01, b01 = a01, b23 = a01;
+#pragma unroll
+                for (int cc = 0; cc < CPB; cc += 2) {
+                    const float4 v = col[cc * NQ], w = col[(cc + 1) * NQ];
                     a01 = add2(a01, make_float2(v.x, v.y));
                     a23 = add2(a23, make_float2(v.z, v.w));
+                    b01 = add2(b01, make_float2(w.x, w.y));
+                    b23 = add2(b23, make_float2(w.z, w.w));
                 }
-                const int64_t tt = t0 + kk;
+                a01 = add2(a01, b01);
+                a23 = add2(a23, b23);
                 const int n = nq * 4;
-                if (kk < rows - k0 && n < N) {
-                    float *dst = (which ? args.dB : args.dC) + (b * L + tt) * N + n;
+                if (k0 + kk < nrows && n < N) {
+                    float *dst = (which ? args.dB : args.dC) + (b * L + t0 + kk) * N + n;
                     if (args.vec_red) {
                         atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(a01.x, a01.y, a23.x, a23.y));
                     } else {
@@ -597,6 +629,12 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                 }
             }
             __syncthreads();
+        };
+        if (rows == T) {
+#pragma unroll
+            for (int sc = T / KC - 1; sc >= 0; --sc) sub_chunk(sc * KC, T);
+        } else {
+            for (int sc = (rows + KC - 1) / KC - 1; sc >= 0; --sc) sub_chunk(sc * KC, rows);
         }
         // ---- the chunk's du, ddelta, dz leave in 16-byte pieces
         for (int p = tid; p < T * ROWV; p += kBlock) {

@@ -53,6 +53,13 @@ struct KStep {
 #ifndef SSM_CHUNK_BF16
 #define SSM_CHUNK_BF16 32
 #endif
+// Step blocks of a full chunk unrolled together (1 = no unrolling).
+#ifndef SSM_R0_UNROLL
+#define SSM_R0_UNROLL 4
+#endif
+#define SSM_PRAGMA_(x) _Pragma(#x)
+#define SSM_UNROLL_N(n) SSM_PRAGMA_(unroll n)
+
 template <typename IO>
 struct StagedCfg {
     static constexpr int T = sizeof(IO) == 2 ? SSM_CHUNK_BF16 : 16;  // time steps per chunk
@@ -210,30 +217,48 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         const int rows = (int)(t_end - tc < T ? t_end - tc : T);
         const IO *st = stage_ptr(c % S);
         const IO *rb = st + 3 * Lay::TILE, *rc = rb + Lay::RAW;
-        for (int i = tid; i < T * NSP; i += kBlock) {
-            const int r = i / NSP, n = i % NSP;
-            const bool ok = r < rows && n < N;
-            fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
-            if (MODE != kCkpt) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+        if (rows == T && N == NSP) {
+            // whole chunk, no padded states: four values per thread and copy
+            for (int i = 4 * tid; i < T * NSP; i += 4 * kBlock) {
+                float v[4];
+                io::load4_smem(rb + i, v);
+                *reinterpret_cast<float4 *>(fB + i) = make_float4(v[0], v[1], v[2], v[3]);
+                if (MODE != kCkpt) {
+                    io::load4_smem(rc + i, v);
+                    *reinterpret_cast<float4 *>(fC + i) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            }
+        } else {
+            for (int i = tid; i < T * NSP; i += kBlock) {
+                const int r = i / NSP, n = i % NSP;
+                const bool ok = r < rows && n < N;
+                fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
+                if (MODE != kCkpt) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+            }
         }
         __syncthreads();
         if (active) {
             const int col = grp * CPL;
-            const IO *su = st + col, *sd = st + Lay::TILE + col, *sz = st + 2 * Lay::TILE + col;
-            const int64_t off0 = (b * L + tc) * Dm + dfirst;
+            // this lane's rows of the tiles start at step q, its B/C slice at state q NS
+            const IO *su = st + col + q * ROW, *sd = st + Lay::TILE + col + q * ROW;
+            const IO *sz = st + 2 * Lay::TILE + col + q * ROW;
+            const float *fBq = fB + q * NS, *fCq = fC + q * NS;
+            IO *poq = po ? po + (b * L + tc + q) * Dm + dfirst : nullptr;
             // KSTEP steps at a time.  The per-step scalar work (softplus,
             // Delta u, skip, gate, store) of step r0 + j G + q is done once, by
             // lane q, for the group's CPL channels; Delta, Delta u and the
             // partial readouts travel between the lanes by shuffles.  Rows past
             // the end of the sequence were zero-filled by the copy and get
             // Delta = 0 (decay 1, no input): the state passes through them.
-            for (int r0 = 0; r0 < rows; r0 += KSTEP) {
+            // Full chunks take an unrolled copy of the block in which nrows is
+            // the constant T (no row tests, immediate shared-memory offsets).
+            auto step_block = [&](const int r0, const int nrows) {
                 float uvo[KG][CPL], dlo[KG][CPL], duo[KG][CPL];
 #pragma unroll
                 for (int j = 0; j < KG; ++j) {
-                    const int r = r0 + j * G + q;
-                    load_vals<IO, CPL>(su + r * ROW, uvo[j]);
-                    load_vals<IO, CPL>(sd + r * ROW, dlo[j]);
+                    const int rr = r0 + j * G;  // this lane's step is rr + q
+                    load_vals<IO, CPL>(su + rr * ROW, uvo[j]);
+                    load_vals<IO, CPL>(sd + rr * ROW, dlo[j]);
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) dlo[j][cc] += bias[cc];
                 }
@@ -261,7 +286,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 }
 #pragma unroll
                 for (int j = 0; j < KG; ++j) {
-                    const bool ok = r0 + j * G + q < rows;
+                    const bool ok = r0 + j * G + q < nrows;
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) {
                         if (!ok) dlo[j][cc] = 0.f;
@@ -281,7 +306,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
                 exchange_steps_cpl<KSTEP, G, CPL>(dlo, duo, dl, du);
                 recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, MODE != kCkpt>(
-                    dl, du, fB + r0 * NSP + q * NS, fC + r0 * NSP + q * NS, NSP, A2, h2, y, invA2);
+                    dl, du, fBq + r0 * NSP, fCq + r0 * NSP, NSP, A2, h2, y, invA2);
                 if (MODE == kCkpt) {
                     // no readout
                 } else if (MODE == kSegAgg) {
@@ -294,20 +319,26 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                     reduce_scatter_steps_cpl<KSTEP, G, CPL>(y, yo, q);
 #pragma unroll
                     for (int j = 0; j < KG; ++j) {
-                        const int r = r0 + j * G + q;
-                        if (r < rows) {
+                        const int rr = r0 + j * G;
+                        if (rr + q < nrows) {
                             float yy[CPL], zz[CPL];
 #pragma unroll
                             for (int cc = 0; cc < CPL; ++cc) yy[cc] = fmaf(dskip[cc], uvo[j][cc], yo[j][cc]);
                             if (pz) {
-                                load_vals<IO, CPL>(sz + r * ROW, zz);
+                                load_vals<IO, CPL>(sz + rr * ROW, zz);
 #pragma unroll
                                 for (int cc = 0; cc < CPL; ++cc) yy[cc] *= silu<PRECISE>(zz[cc]);
                             }
-                            store_vals<IO, CPL>(po + off0 + (int64_t)r * Dm, yy);
+                            store_vals<IO, CPL>(poq + (int64_t)rr * Dm, yy);
                         }
                     }
                 }
+            };
+            if (rows == T) {
+                SSM_UNROLL_N(SSM_R0_UNROLL)
+                for (int r0 = 0; r0 < T; r0 += KSTEP) step_block(r0, T);
+            } else {
+                for (int r0 = 0; r0 < rows; r0 += KSTEP) step_block(r0, rows);
             }
         }
         __syncthreads();  // stage c % S and the fp32 B/C buffers are free again

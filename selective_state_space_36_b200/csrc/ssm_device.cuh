@@ -26,6 +26,11 @@ template <> struct io_traits<float> {
     static __device__ __forceinline__ float load(const float *p) { return __ldg(p); }
     static __device__ __forceinline__ float load_stream(const float *p) { return __ldcs(p); }
     static __device__ __forceinline__ float load_smem(const float *p) { return *p; }
+    // four consecutive values from a 16-byte aligned shared-memory address
+    static __device__ __forceinline__ void load4_smem(const float *p, float *v) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    }
     // four consecutive values from a 16-byte aligned address
     static __device__ __forceinline__ void load4(const float *p, float *v) {
         const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
@@ -45,6 +50,12 @@ template <> struct io_traits<__nv_bfloat16> {
     }
     static __device__ __forceinline__ float load_smem(const __nv_bfloat16 *p) {
         return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(p)) << 16);
+    }
+    // four consecutive values from an 8-byte aligned shared-memory address
+    static __device__ __forceinline__ void load4_smem(const __nv_bfloat16 *p, float *v) {
+        const uint2 t = *reinterpret_cast<const uint2 *>(p);
+        v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
+        v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
     }
     // four consecutive values from an 8-byte aligned address
     static __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float *v) {
