@@ -269,12 +269,35 @@ ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
  *   A     : (dim, dstate) float32.     B, C : (batch, dstate) io.
  *   D     : (dim) float32 or NULL.     z    : (batch, dim) io or NULL.
  *   out   : (batch, dim) io.
- * dims.seqlen is ignored.
+ * dims.seqlen is ignored.  With dstate 4, 8, 16, 32 or 64, a 16-byte aligned
+ * state and A, and B, C aligned to four elements, the state moves through
+ * shared memory in 16 KB units by TMA bulk copies (a persistent kernel whose
+ * waits are bounded, see ssm_get_device_status); otherwise each thread loads
+ * its 4-state slice directly.
  */
 ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
                                       const void *x, const void *dt, const float *A,
                                       const void *B, const void *C, const float *D,
                                       const void *z, void *out, ssm_stream stream);
+
+/*
+ * Reads and clears the device status word of the current device, after
+ * synchronising "stream".  Bit 0: a bounded wait inside the decode kernel
+ * (its state copies, see ssm_selective_state_update) gave up; the outputs of
+ * the launches since the last read are then not valid.  The word is shared by
+ * every launch on the device.  Returns SSM_ERR_CUDA if the copies or the
+ * synchronisation fail.
+ */
+ssm_status ssm_get_device_status(ssm_stream stream, uint32_t *flags);
+
+/*
+ * Test hook (no counterpart in the method): while enabled, every decode
+ * launch that moves its state with bulk copies waits for 16 bytes per unit
+ * that never arrive, so each of its waits runs out (200 ms) and sets bit 0 of
+ * the device status word; the copies themselves complete normally.  Used to
+ * test the bounded waits without a GPU fault.  Process-wide; 0 disables.
+ */
+void ssm_test_inject_decode_wait_timeout(int32_t enable);
 
 /* Static description of a status code. */
 const char *ssm_status_string(ssm_status status);

@@ -22,8 +22,9 @@ FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
 
 # every symbol include/ssm.h declares
 EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
-            "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ex", "ssm_selective_state_update", "ssm_scan_plan", "ssm_status_string", "ssm_last_error",
-            "ssm_version")
+            "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ex", "ssm_selective_state_update",
+            "ssm_scan_plan", "ssm_get_device_status", "ssm_test_inject_decode_wait_timeout",
+            "ssm_status_string", "ssm_last_error", "ssm_version")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -79,6 +80,10 @@ def _load() -> ctypes.CDLL:
     lib.ssm_scan_plan.argtypes = [SSMDims, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                   ctypes.POINTER(SSMScanOpts), ctypes.POINTER(SSMScanPlanInfo)]
     lib.ssm_scan_plan.restype = ctypes.c_int
+    lib.ssm_get_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.ssm_get_device_status.restype = ctypes.c_int
+    lib.ssm_test_inject_decode_wait_timeout.argtypes = [ctypes.c_int32]
+    lib.ssm_test_inject_decode_wait_timeout.restype = None
     lib.ssm_status_string.argtypes = [ctypes.c_int]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_last_error.argtypes = []
@@ -254,6 +259,14 @@ def scan_plan(batch: int, seqlen: int, dim: int, dstate: int, io: str = "bf16",
             "family": inv_f.get(info.family, "none"), "launches": info.launches,
             "channels_per_lane": info.channels_per_lane,
             "workspace_bytes": info.workspace_bytes}
+
+
+def device_status(stream=None) -> int:
+    """Synchronises ``stream`` and returns (and clears) the device status word:
+    bit 0 = a bounded wait in the decode kernel gave up."""
+    v = ctypes.c_uint32(0)
+    check(lib.ssm_get_device_status(_stream_handle(stream), ctypes.byref(v)))
+    return int(v.value)
 
 
 def selective_state_update(state, x, dt, A, B, C, D=None, z=None, out=None, stream=None):

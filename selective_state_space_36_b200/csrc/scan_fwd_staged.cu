@@ -33,7 +33,7 @@
 namespace ssm {
 
 #ifndef SSM_KSTEP
-#define SSM_KSTEP 4
+#define SSM_KSTEP 16
 #endif
 // Time steps processed together: a multiple of G that divides the chunk, and
 // with one channel per lane a multiple of 2G, so the per-step scalar work of a
@@ -124,7 +124,8 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP, ROW = Lay::ROW;
     constexpr int EPV = 16 / sizeof(IO);  // elements per 16-byte piece
     constexpr int ROWV = CPB / EPV;       // pieces per tile row
-    constexpr int KSTEP = KStep<G, CPL>::value;
+    // the checkpoint pass stores a state every 8 steps: its step blocks are 8 long
+    constexpr int KSTEP = MODE == kCkpt ? 8 : KStep<G, CPL>::value;
     constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
     static_assert(T % KSTEP == 0, "a chunk holds whole step blocks");
     extern __shared__ __align__(16) unsigned char smem[];

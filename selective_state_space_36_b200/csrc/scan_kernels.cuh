@@ -73,6 +73,13 @@ bool staged_eligible(const ScanArgs &a, int es);
 size_t staged_smem_bytes(bool bf16, int ns, int g, int cpl);
 bool scan_shape_supported(int ns, int g);
 cudaError_t launch_state_update(const DecodeArgs &a, bool bf16, int ns, int g, cudaStream_t st);
+// decode step with the state moved by TMA bulk copies (dstate 4, 8, 16, 32 or
+// 64; 16-byte aligned state and A); missing_bytes > 0 makes every unit's wait
+// expect bytes that never arrive (a test of the bounded waits)
+bool state_update_bulk_eligible(const DecodeArgs &a, bool bf16);
+cudaError_t launch_state_update_bulk(const DecodeArgs &a, bool bf16, uint32_t missing_bytes, cudaStream_t st);
+// the device status word the kernels' bounded waits report into
+unsigned int read_and_clear_device_status(cudaStream_t st, cudaError_t *err);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
 // staged second pass (checkpoints every scan_bwd_staged_chunk() steps, from
 // the staged forward kernel in kCkpt mode)

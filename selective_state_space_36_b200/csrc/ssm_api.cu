@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 
+#include <atomic>
 #include <mutex>
 #include <stdio.h>
 #include <string.h>
@@ -13,6 +14,15 @@
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// Decode kernel: 1 = bulk-copy kernel where eligible, 0 = per-slice loads only.
+#ifndef SSM_DECODE_BULK
+#define SSM_DECODE_BULK 1
+#endif
+constexpr bool kDecodeBulk = SSM_DECODE_BULK != 0;
+
+// test hook: extra bytes every decode unit's wait expects (0 = none)
+std::atomic<uint32_t> g_inject_wait_bytes{0};
 
 ssm_status fail(ssm_status s, const char *fmt, ...) {
     va_list ap;
@@ -70,11 +80,13 @@ void scan_layout(int64_t dstate, int64_t channels, int sms, int lanes_req, int *
     if (dstate <= 16) {
         int G = lanes_req;
         if (G != 1 && G != 2 && G != 4) {
-            // Four lanes per channel (4 states each) unless the channels alone
-            // already give every SM four 128-thread blocks: the finer split
-            // quadruples the warps available to hide latency and evens out
-            // the work per SM, at ~10% more instructions (shuffles).
-            G = channels >= (int64_t)sms * ssm::kBlock * 4 ? 1 : 4;
+            // One lane per channel (all 16 states) once the channels give the
+            // SMs 1.5 blocks of 128 on average (most SMs then hold two): no
+            // shuffles, ~40% fewer instructions per element, and it measured
+            // ~5% faster at the 1.4B-layer shape (32,768 channels).  Below
+            // that, four lanes per channel (4 states each) quadruple the warps
+            // that hide latency and even out the work per SM.
+            G = 2 * channels >= (int64_t)sms * ssm::kBlock * 3 ? 1 : 4;
         }
         *g = G;
         *ns = 16 / G;
@@ -515,7 +527,9 @@ ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     int ns = 0, g = 0;
     if (staged) {
         const DeviceInfo di = device_info();
-        scan_layout(dims.dstate, channels, di.sms, 0, &ns, &g);
+        // the checkpoint pass (8-step blocks, no readout) measured faster with
+        // four lanes per channel than with one at the 1.4B-layer shape
+        scan_layout(dims.dstate, channels, di.sms, 4, &ns, &g);
         if (ssm::staged_smem_bytes(io == SSM_BF16, ns, g, 1) > (size_t)di.smem_optin)
             return fail(SSM_ERR_UNSUPPORTED, "staged backward needs more shared memory than the device has");
     }
@@ -600,9 +614,25 @@ ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
     a.state = state; a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
     a.A = A; a.Dskip = D; a.out = out;
     a.batch = dims.batch; a.dim = dims.dim; a.dstate = (int)dims.dstate;
-    cudaError_t e = ssm::launch_state_update(a, io == SSM_BF16, 4, g, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (kDecodeBulk && ssm::state_update_bulk_eligible(a, io == SSM_BF16))
+        e = ssm::launch_state_update_bulk(a, io == SSM_BF16, g_inject_wait_bytes.load(), st);
+    else
+        e = ssm::launch_state_update(a, io == SSM_BF16, 4, g, st);
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return SSM_OK;
 }
+
+ssm_status ssm_get_device_status(ssm_stream stream, uint32_t *flags) {
+    g_last_error[0] = 0;
+    if (!flags) return fail(SSM_ERR_INVALID_ARG, "flags is required");
+    cudaError_t e = cudaSuccess;
+    *flags = ssm::read_and_clear_device_status(reinterpret_cast<cudaStream_t>(stream), &e);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    return SSM_OK;
+}
+
+void ssm_test_inject_decode_wait_timeout(int32_t enable) { g_inject_wait_bytes.store(enable ? 16u : 0u); }
 
 }  // extern "C"

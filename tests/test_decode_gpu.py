@@ -26,8 +26,11 @@ def _oracle_step(h, st, A, D, io):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("N", [1, 3, 4, 8, 13, 16, 24, 32, 64])
-def test_decode_steps_small(lib, io, N):
-    cfg = I.DecodeConfig("d", 3, 77, N, steps=20, io=io, seed=N)
+@pytest.mark.parametrize("dim", [77, 80])
+def test_decode_steps_small(lib, io, N, dim):
+    # dim 77: per-slice loads; dim 80 (rows of a multiple of 16 bytes): the
+    # bulk-copy kernel for N = 4 (fp32), 8, 16, 32, 64, with a partial unit
+    cfg = I.DecodeConfig("d", 3, dim, N, steps=20, io=io, seed=N + dim)
     A, D, bias = I.decode_params(cfg)
     h0 = I.decode_h0(cfg)
     state = torch.from_numpy(h0).cuda()
@@ -112,3 +115,52 @@ def test_decode_workload_full_size(lib):
         ref, h = _oracle_step(h, sub, As, Ds, io)
         worst = max(worst, T.check_out(T.from_dev(out[bt][:, dt_]), ref, io))
     T.check_state(T.from_dev(state[bt][:, dt_]), h, io)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_bulk_ring_wraps(lib, io):
+    # 3072 units of 16 KB (6 per batch row, the last one 24 channels wide):
+    # seven per CTA, so every buffer of the copy ring is reused and its
+    # barrier changes phase
+    cfg = I.DecodeConfig("d", 512, 1304, 16, steps=3, io=io, seed=5)
+    A, D, bias = I.decode_params(cfg)
+    h0 = I.decode_h0(cfg)
+    state = torch.from_numpy(h0).cuda()
+    Ad, Dd = torch.from_numpy(A).cuda(), torch.from_numpy(D).cuda()
+    h = h0.astype(np.float64)
+    for k in range(cfg.steps):
+        st = I.decode_step_inputs(cfg, k, bias)
+        out = lib.selective_state_update(state, T.to_dev(st["x"], io), T.to_dev(st["dt"], io), Ad,
+                                         T.to_dev(st["B"], io), T.to_dev(st["C"], io), D=Dd,
+                                         z=T.to_dev(st["z"], io))
+        ref, h = _oracle_step(h, st, A.astype(np.float64), D.astype(np.float64), io)
+        T.check_out(T.from_dev(out), ref, io)
+    T.check_state(T.from_dev(state), h, io)
+    assert lib.device_status() == 0
+
+
+def test_decode_bounded_wait_sets_device_status(lib):
+    # every wait of the state copies runs out (the test hook asks each unit's
+    # barrier for 16 bytes that never come): the kernel gives up after its
+    # time limit, reports bit 0 and the context stays usable
+    cfg = I.DecodeConfig("d", 2, 304, 16, steps=1, io="bf16", seed=6)
+    A, D, bias = I.decode_params(cfg)
+    h0 = I.decode_h0(cfg)
+    Ad, Dd = torch.from_numpy(A).cuda(), torch.from_numpy(D).cuda()
+    st = I.decode_step_inputs(cfg, 0, bias)
+    args = [T.to_dev(st["x"], "bf16"), T.to_dev(st["dt"], "bf16"), Ad, T.to_dev(st["B"], "bf16"),
+            T.to_dev(st["C"], "bf16")]
+    assert lib.device_status() == 0
+    lib.lib.ssm_test_inject_decode_wait_timeout(1)
+    try:
+        lib.selective_state_update(torch.from_numpy(h0).cuda(), *args, D=Dd, z=T.to_dev(st["z"], "bf16"))
+        assert lib.device_status() & 1
+    finally:
+        lib.lib.ssm_test_inject_decode_wait_timeout(0)
+    assert lib.device_status() == 0
+    state = torch.from_numpy(h0).cuda()
+    out = lib.selective_state_update(state, *args, D=Dd, z=T.to_dev(st["z"], "bf16"))
+    ref, h = _oracle_step(h0.astype(np.float64), st, A.astype(np.float64), D.astype(np.float64), "bf16")
+    T.check_out(T.from_dev(out), ref, "bf16")
+    T.check_state(T.from_dev(state), h, "bf16")
+    assert lib.device_status() == 0

@@ -143,3 +143,11 @@ def test_bwd_is_linear_in_dout(family):
         ref = T.from_dev(g1[k]) + T.from_dev(g2[k])
         e = T.grad_err(T.from_dev(g12[k]), ref)
         assert e <= 1e-4, (k, e)
+
+
+def test_bwd_staged_with_one_lane_checkpoint_pass(lib):
+    # 32,768 channels: the checkpointing forward pass takes the one-lane
+    # layout (all 16 states in one thread) that large problems get
+    plan = lib.scan_plan(2, 48, 16384, 16, "bf16")
+    assert plan["lanes"] == 1
+    _check("bf16", 2, 48, 16384, 16, 17, family="staged", h0_sigma=0.5)
