@@ -20,6 +20,10 @@ Parity status of each function (what pins it lives in tests/test_oracle_pins.py)
                           one-step brute force.
   scan_bwd                pinned: central finite differences of scan (every
                           input), torch autograd of an independent fp64 loop.
+  scan_complex            pinned: bit-identical to scan when every imaginary
+                          part is zero, brute-force complex unrolled sum, LTI
+                          convolution with a complex kernel, pure-rotation
+                          closed form (sign of the phase).
 """
 from __future__ import annotations
 
@@ -62,6 +66,8 @@ def _bind(path: str):
                                         _dp, _dp, _dp, _dp, _dp]
     lib.oracle_default_threads.restype = ctypes.c_int
     lib.oracle_default_threads.argtypes = []
+    lib.oracle_selective_scan_complex.restype = ctypes.c_int
+    lib.oracle_selective_scan_complex.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [ctypes.c_int, _dp, _dp]
     lib.oracle_selective_scan_bwd.restype = ctypes.c_int
     lib.oracle_selective_scan_bwd.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [ctypes.c_int] + [_dp] * 11
     return lib
@@ -126,6 +132,50 @@ def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True
     if rc != 0:
         raise RuntimeError(f"oracle_selective_scan failed with code {rc}")
     return out, state
+
+
+def _pairs(a, shape, name):
+    """A complex array as a contiguous float64 (..., 2) array of (re, im)."""
+    if a is None:
+        return None
+    c = np.ascontiguousarray(a, dtype=np.complex128)
+    if c.shape != shape:
+        raise ValueError(f"{name}: expected shape {shape}, got {c.shape}")
+    return c.view(np.float64).reshape(shape + (2,))
+
+
+def scan_complex(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                 h0=None, _lib_handle=None):
+    """Selective scan with complex A, B, C in fp64 (real u, delta, z, D, bias).
+
+    A: (dim, dstate) complex; B, C: (batch, seqlen, dstate) complex; h0:
+    (batch, dim, dstate) complex or None.  y_t = Re(sum_n C_t,n h_t,n) + D u_t.
+    Returns (out (batch, seqlen, dim) real, last_state (batch, dim, dstate) complex).
+    """
+    u = np.asarray(u)
+    batch, seqlen, dim = u.shape
+    dstate = np.asarray(A).shape[1]
+    keep = []
+
+    def p(a, shape, name):
+        arr, ptr = _c64(a, shape, name)
+        keep.append(arr)
+        return ptr
+
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate)
+    Ap, Bp, Cp = _pairs(A, (dim, dstate), "A"), _pairs(B, bc, "B"), _pairs(C, bc, "C")
+    ins = [p(u, seq, "u"), p(delta, seq, "delta"), p(Ap, (dim, dstate, 2), "A"), p(Bp, bc + (2,), "B"),
+           p(Cp, bc + (2,), "C"), p(D, (dim,), "D"), p(z, seq, "z"), p(delta_bias, (dim,), "delta_bias")]
+    out = np.zeros(seq, dtype=np.float64)
+    st = np.zeros((batch, dim, dstate), dtype=np.complex128) if h0 is None else \
+        np.array(h0, dtype=np.complex128, order="C", copy=True).reshape(batch, dim, dstate)
+    stp = st.view(np.float64)
+    rc = (_lib_handle or _load()).oracle_selective_scan_complex(
+        batch, seqlen, dim, dstate, *ins, int(bool(delta_softplus)), out.ctypes.data_as(_dp),
+        stp.ctypes.data_as(_dp))
+    if rc != 0:
+        raise RuntimeError(f"oracle_selective_scan_complex failed with code {rc}")
+    return out, st
 
 
 def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, delta_softplus=True,
@@ -206,6 +256,9 @@ class Variant:
 
     def scan_bwd(self, *a, **kw):
         return scan_bwd(*a, _lib_handle=self._h, **kw)
+
+    def scan_complex(self, *a, **kw):
+        return scan_complex(*a, _lib_handle=self._h, **kw)
 
 
 def compile_variant(source: str, path: str) -> "Variant":

@@ -34,6 +34,7 @@
  * B, C (batch, seqlen, dstate); A (dim, dstate); D, delta_bias (dim);
  * state (batch, dim, dstate).  All values are double.
  */
+#include <complex.h>
 #include <math.h>
 #include <pthread.h>
 #include <stddef.h>
@@ -178,6 +179,69 @@ int oracle_selective_scan(int64_t batch, int64_t seqlen, int64_t dim, int64_t ds
     free(jobs);
     free(th);
     return rc;
+}
+
+/*
+ * Selective scan with a complex diagonal A (and complex B, C): the
+ * parameterisation the Mamba notes single out for audio (【論文要約】Mamba
+ * notes, Figure 10: complex parameters matter there; Table 8, the A
+ * initialisation ablation).  The pages give no formula for it, so this is the
+ * plain reading of the real recurrence with complex numbers:
+ *     Abar = exp(Delta A)            (complex exponential; Delta is real)
+ *     Bbar = Delta B                 (Euler form, as for the real scan)
+ *     h_t  = Abar h_{t-1} + Bbar x_t (complex state)
+ *     y_t  = Re(sum_n C_t,n h_t,n) + D x_t,   out = y silu(z)
+ * u, delta, z, out, D, delta_bias are real as before.  Complex arrays hold
+ * (re, im) pairs: A (dim, dstate, 2), B and C (batch, seqlen, dstate, 2),
+ * state (batch, dim, dstate, 2).  state: NULL => h0 = 0 and the final state
+ * is not returned.  Single-threaded.  Returns 0 on success.
+ */
+int oracle_selective_scan_complex(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                                  const double *u, const double *delta, const double *A,
+                                  const double *B, const double *C, const double *Dskip,
+                                  const double *z, const double *delta_bias, int delta_softplus,
+                                  double *out, double *state)
+{
+    const int64_t L = seqlen, Dm = dim, N = dstate;
+    if (batch < 0 || L < 0 || Dm < 0 || N < 0) return ORACLE_BAD_ARG;
+    if (batch * Dm == 0) return ORACLE_OK;
+    if (L > 0 && (!u || !delta || !B || !C || !out)) return ORACLE_BAD_ARG;
+    if (N > 0 && !A) return ORACLE_BAD_ARG;
+    double complex *h = (double complex *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double complex));
+    if (!h) return ORACLE_NO_MEM;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < Dm; ++d) {
+            const int64_t so = (b * Dm + d) * N;
+            for (int64_t n = 0; n < N; ++n)
+                h[n] = state ? state[2 * (so + n)] + I * state[2 * (so + n) + 1] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t td = (b * L + t) * Dm + d;
+                const int64_t tn = (b * L + t) * N;
+                const double x = u[td];
+                const double s = delta[td] + (delta_bias ? delta_bias[d] : 0.0);
+                const double dlt = delta_softplus ? oracle_softplus(s) : s;
+                double complex acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double complex an = A[2 * (d * N + n)] + I * A[2 * (d * N + n) + 1];
+                    const double complex bn = B[2 * (tn + n)] + I * B[2 * (tn + n) + 1];
+                    const double complex cn = C[2 * (tn + n)] + I * C[2 * (tn + n) + 1];
+                    const double complex abar = cexp(dlt * an);
+                    h[n] = abar * h[n] + (dlt * bn) * x;
+                    acc += cn * h[n];
+                }
+                double y = creal(acc) + (Dskip ? Dskip[d] * x : 0.0);
+                if (z) y *= oracle_silu(z[td]);
+                out[td] = y;
+            }
+            if (state)
+                for (int64_t n = 0; n < N; ++n) {
+                    state[2 * (so + n)] = creal(h[n]);
+                    state[2 * (so + n) + 1] = cimag(h[n]);
+                }
+        }
+    }
+    free(h);
+    return ORACLE_OK;
 }
 
 /*

@@ -39,6 +39,12 @@ MUTANTS = {
     "decode_without_dt": ("h[n] = abar * h[n] + dlt * B[b * dstate + n] * xv;",
                           "h[n] = abar * h[n] + B[b * dstate + n] * xv;"),
     "h0_ignored": ("h[n] = j->state ? j->state[(b * Dm + d) * N + n] : 0.0;", "h[n] = 0.0;"),
+    # complex A
+    "complex_conjugate_phase": ("cexp(dlt * an)", "cexp(dlt * conj(an))"),
+    "complex_readout_imaginary": ("double y = creal(acc) +", "double y = cimag(acc) +"),
+    "complex_B_real_part_only": ("h[n] = abar * h[n] + (dlt * bn) * x;", "h[n] = abar * h[n] + (dlt * creal(bn)) * x;"),
+    "complex_h0_imaginary_dropped": ("h[n] = state ? state[2 * (so + n)] + I * state[2 * (so + n) + 1] : 0.0;",
+                                     "h[n] = state ? state[2 * (so + n)] : 0.0;"),
     # backward
     "bwd_adjoint_not_decayed": ("lam[n] *= abar;", "(void)0;"),
     "bwd_dA_without_decay": ("dA[d * N + n] += lam[n] * hprev * abar * dl[t];",

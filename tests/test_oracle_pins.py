@@ -408,3 +408,95 @@ def test_bwd_matches_torch_autograd(oracle_mod):
                             D=case["D"], z=case["z"], delta_bias=case["delta_bias"], h0=case["h0"])
     for name, gname in _GRAD_OF.items():
         _close(g[gname], t[name].grad.numpy(), 1e-12)
+
+
+# ------------------------------------------------------------ complex A
+def _complex_case(rng, batch=2, L=10, dim=3, N=4, softplus=True, gate=True, dskip=True, h0=True):
+    c = _rand_case(rng, batch, L, dim, N, softplus=softplus, gate=gate, dskip=dskip, h0=h0)
+    c["A"] = c["A"] + 1j * rng.uniform(-4.0, 4.0, size=(dim, N))
+    c["B"] = c["B"] + 1j * rng.standard_normal((batch, L, N))
+    c["C"] = c["C"] + 1j * rng.standard_normal((batch, L, N))
+    if h0:
+        c["h0"] = c["h0"] + 1j * rng.standard_normal((batch, dim, N))
+    return c
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_complex_with_zero_imaginary_parts_is_the_real_scan(oracle_mod, softplus):
+    # with every imaginary part 0 the complex recurrence is the real one, and
+    # the arithmetic is the same operation for operation: bit-identical
+    rng = np.random.default_rng(80 + softplus)
+    c = _rand_case(rng, softplus=softplus)
+    cc = dict(c, A=c["A"] + 0j, B=c["B"] + 0j, C=c["C"] + 0j, h0=c["h0"] + 0j)
+    out_r, st_r = oracle_mod.scan(**c)
+    out_c, st_c = oracle_mod.scan_complex(**cc)
+    assert np.array_equal(out_r, out_c)
+    assert np.array_equal(st_r, st_c.real) and not np.any(st_c.imag)
+
+
+def test_complex_brute_force_unrolled_sum(oracle_mod):
+    # y_t = Re(sum_n sum_{s<=t} C_t (prod_{r=s+1..t} e^{Delta_r A}) Delta_s B_s x_s
+    #          + C_t (prod_{r<=t} e^{Delta_r A}) h0) + D x_t, then the gate;
+    # explicit products with cmath (no running state)
+    import cmath
+    rng = np.random.default_rng(91)
+    c = _complex_case(rng, L=8)
+    u, delta, A, B, C = c["u"], c["delta"], c["A"], c["B"], c["C"]
+    batch, L, dim = u.shape
+    N = A.shape[1]
+    out = np.zeros_like(u)
+    for b in range(batch):
+        for d in range(dim):
+            dl = [math.log1p(math.exp(delta[b, t, d] + c["delta_bias"][d])) for t in range(L)]
+            for t in range(L):
+                acc = 0j
+                for n in range(N):
+                    def prod(lo, hi):
+                        p = 1 + 0j
+                        for r in range(lo, hi + 1):
+                            p *= cmath.exp(dl[r] * A[d, n])
+                        return p
+                    h = prod(0, t) * c["h0"][b, d, n]
+                    for s in range(t + 1):
+                        h += prod(s + 1, t) * dl[s] * B[b, s, n] * u[b, s, d]
+                    acc += C[b, t, n] * h
+                y = acc.real + c["D"][d] * u[b, t, d]
+                out[b, t, d] = y * c["z"][b, t, d] * expit(c["z"][b, t, d])
+    got, _ = oracle_mod.scan_complex(**c)
+    np.testing.assert_allclose(got, out, rtol=1e-11, atol=1e-11)
+
+
+def test_complex_lti_equals_convolution(oracle_mod):
+    # constant Delta, B, C: y = x * K + D x with the complex kernel
+    # K_k = Re(sum_n C_n e^{k Delta A_n} Delta B_n)  (NL-345 eq. (3), complex A)
+    rng = np.random.default_rng(92)
+    L, dim, N, dl = 40, 2, 5, 0.3
+    A = -rng.uniform(0.1, 1.0, size=(dim, N)) + 1j * rng.uniform(-3, 3, size=(dim, N))
+    Bv = rng.standard_normal(N) + 1j * rng.standard_normal(N)
+    Cv = rng.standard_normal(N) + 1j * rng.standard_normal(N)
+    u = rng.standard_normal((1, L, dim))
+    D = rng.standard_normal(dim)
+    out, _ = oracle_mod.scan_complex(u, np.full((1, L, dim), dl), A, np.broadcast_to(Bv, (1, L, N)),
+                                     np.broadcast_to(Cv, (1, L, N)), D=D, delta_softplus=False)
+    for d in range(dim):
+        k = np.arange(L)
+        K = np.real((Cv[None, :] * np.exp(np.outer(k, dl * A[d])) * dl * Bv[None, :]).sum(axis=1))
+        ref = np.convolve(u[0, :, d], K)[:L] + D[d] * u[0, :, d]
+        np.testing.assert_allclose(out[0, :, d], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_complex_pure_rotation_closed_form(oracle_mod):
+    # A = i w (no decay), constant Delta, an impulse at t = 0, B = 1, h0 = 0:
+    # h_t = Delta e^{i w Delta t}; C = 1 reads Delta cos(w Delta t), C = i reads
+    # -Delta sin(w Delta t) (the sign of the phase)
+    L, dl, w = 25, 0.2, 1.7
+    u = np.zeros((1, L, 1))
+    u[0, 0, 0] = 1.0
+    A = np.array([[1j * w]])
+    Bm = np.ones((1, L, 1), dtype=complex)
+    t = np.arange(L)
+    for Cval, ref in [(1.0, dl * np.cos(w * dl * t)), (1j, -dl * np.sin(w * dl * t))]:
+        out, st = oracle_mod.scan_complex(u, np.full((1, L, 1), dl), A, Bm, np.full((1, L, 1), Cval),
+                                          delta_softplus=False)
+        np.testing.assert_allclose(out[0, :, 0], ref, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(st[0, 0, 0], dl * np.exp(1j * w * dl * (L - 1)), rtol=1e-12)
