@@ -6,7 +6,7 @@ softplus(Delta), discretisation, recurrence, readout, D skip, silu(z) gate, the
 fp32 state in and out.  Inputs are seeded synthetic data of that shape.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload mamba1p4b|mamba130m|longseq|decode|mamba1p4b_bwd]
+                  [--workload mamba1p4b|mamba130m|longseq|decode|mamba1p4b_bwd|mamba130m_complex]
 
 The other workloads measure the remaining hot-path kernels the same way:
 mamba130m (batch 8, L 2048, dim 1536), longseq (batch 1, L 1,048,576, dim 1536:
@@ -46,7 +46,7 @@ UNIT = "Gelem/s"
 WORKLOAD = I.MAMBA1P4B
 L2_BYTES = 126 * 1024 * 1024
 WORKLOADS = {"mamba1p4b": I.MAMBA1P4B, "mamba130m": I.MAMBA130M, "longseq": I.LONGSEQ,
-             "decode": I.DECODE, "mamba1p4b_bwd": I.MAMBA1P4B}
+             "decode": I.DECODE, "mamba1p4b_bwd": I.MAMBA1P4B, "mamba130m_complex": I.MAMBA130M}
 SCAN_METRICS = {
     "mamba1p4b": METRIC,
     "mamba130m": "selective-scan fwd Gelem/s (B·L·D) at 130M-layer shape; % of HBM roofline",
@@ -54,6 +54,7 @@ SCAN_METRICS = {
 }
 DECODE_METRIC = "decode state-update steps/s at batch 256, dim 5120, N 16; % of HBM roofline"
 BWD_METRIC = "selective-scan bwd Gelem/s (B·L·D) at 1.4B-layer shape"
+COMPLEX_METRIC = "selective-scan fwd, complex A (S4D-Lin), Gelem/s (B·L·D) at 130M-layer shape"
 
 
 def bwd_sfu_ceiling_per_sm_clock(dstate: int = 16) -> float:
@@ -621,6 +622,48 @@ def run_bwd(args, rank, world, dev):
     return 0
 
 
+def run_complex(args, rank, world, dev):
+    """One step = one ssm_selective_scan_fwd_complex over the 130M-layer
+    workload with complex A = -1/2 + i pi n and complex B, C."""
+    import torch
+    from selective_state_space_36_b200 import binding as lib
+
+    cfg = WORKLOADS[args.workload]
+    if rank:
+        cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
+    x = I.complex_scan_inputs(cfg)
+    d = {k: _upload(v, dev) for k, v in x.items() if isinstance(v, np.ndarray)}
+    state = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, 2, device=dev)
+    out = torch.empty_like(d["u"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lib.selective_scan_fwd_complex(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                       delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
+
+    elapsed_ms, kernel_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
+    ms_per_step = elapsed_ms / args.steps
+    if rank == 0:
+        peaks = measured_peaks()
+        es = 2 if cfg.io == "bf16" else 4
+        abytes = cfg.elements * es * 4 + cfg.batch * cfg.seqlen * cfg.dstate * es * 4
+        achieved = abytes / (kernel_ms * 1e-3) / 1e9
+        line = _base_line(COMPLEX_METRIC, UNIT, whole_job_rate(world, cfg.elements, ms_per_step), world, args,
+                          ms_per_step)
+        line.update({
+            "config": {"workload": cfg.name + "_complex", "batch": cfg.batch, "seqlen": cfg.seqlen,
+                       "dim": cfg.dim, "dstate": cfg.dstate, "io": cfg.io, "A": "-1/2 + i pi n"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel_ms": kernel_ms,
+                         "algorithmic_bytes_per_launch": abytes,
+                         "note": "arithmetic-bound (exp, sincos and complex products per state); "
+                                 "the HBM fraction is context"},
+            "e2e": None, "gpu_launches": args.steps, "clocks": clocks,
+        })
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> int:
     import torch
     import torch.distributed as dist
@@ -633,6 +676,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
             return run_decode(args, rank, world, dev)
         if args.workload == "mamba1p4b_bwd":
             return run_bwd(args, rank, world, dev)
+        if args.workload == "mamba130m_complex":
+            return run_complex(args, rank, world, dev)
         return run_scan(args, rank, world, dev)
     finally:
         if world > 1:

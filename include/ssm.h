@@ -206,6 +206,28 @@ ssm_status ssm_scan_plan(ssm_dims dims, ssm_dtype io, const void *u, const void 
                          const ssm_scan_opts *opts, ssm_scan_plan_info *info);
 
 /*
+ * Selective scan with a complex diagonal A (and complex B, C), one pass over
+ * the sequence: the complex parameterisation the Mamba notes single out for
+ * audio (【論文要約】Mamba notes, Figure 10; Table 8), read as the real
+ * recurrence carried out in complex numbers:
+ *   Abar_n = exp(Delta A_n),  Bbar_n = Delta B_n (Euler),
+ *   h_n <- Abar_n h_n + Bbar_n u,   y = Re(sum_n C_n h_n) + D u,
+ *   out = y * silu(z).
+ * Delta (softplus(delta + bias) or the plain sum), u, z, D, delta_bias and
+ * out are real, with the layouts of ssm_selective_scan_fwd.  Complex arrays
+ * hold (re, im) pairs:
+ *   A          : (dim, dstate, 2) float32
+ *   B, C       : (batch, seqlen, dstate, 2) io
+ *   last_state : (batch, dim, dstate, 2) float32 or NULL; read as h_0 and
+ *                overwritten with h_L (NULL: h_0 = 0, not written).
+ * Returns the statuses of ssm_selective_scan_fwd.  No sequence split.
+ */
+ssm_status ssm_selective_scan_fwd_complex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                          const float *A, const void *B, const void *C, const float *D,
+                                          const void *z, const float *delta_bias, int delta_softplus,
+                                          void *out, float *last_state, ssm_stream stream);
+
+/*
  * Selective scan, backward: the gradients of the scalar loss sum(dout * out)
  * of one ssm_selective_scan_fwd pass (Euler Bbar) with respect to every input.
  * The states are recomputed from checkpoints instead of being kept by the

@@ -22,6 +22,7 @@ FAMILIES = {"auto": 0, "generic": 1, "staged": 2}
 
 # every symbol include/ssm.h declares
 EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
+            "ssm_selective_scan_fwd_complex",
             "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ex", "ssm_selective_state_update",
             "ssm_scan_plan", "ssm_get_device_status", "ssm_test_inject_decode_wait_timeout",
             "ssm_status_string", "ssm_last_error", "ssm_version")
@@ -68,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.ssm_selective_scan_fwd_ex.restype = ctypes.c_int
     lib.ssm_selective_scan_fwd_noalloc.argtypes = scan_args + [ctypes.c_int, _vp]
     lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssm_selective_scan_fwd_complex.argtypes = scan_args + [_vp]
+    lib.ssm_selective_scan_fwd_complex.restype = ctypes.c_int
     lib.ssm_selective_scan_bwd.argtypes = ([SSMDims, ctypes.c_int] + [_vp] * 8 + [ctypes.c_int] +
                                            [_vp] * 11 + [_vp])
     lib.ssm_selective_scan_bwd.restype = ctypes.c_int
@@ -171,6 +174,47 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
         opts = SSMScanOpts(VARIANTS[variant], int(segments), int(lanes), FAMILIES[family], int(cpl),
                            int(bool(zoh_b)))
         check(lib.ssm_selective_scan_fwd_ex(dims, io, *args, ctypes.byref(opts), _stream_handle(stream)))
+    return out
+
+
+def _pairs(t, name):
+    """A complex tensor as its (re, im) float view; real tensors pass through."""
+    if t is not None and torch.is_complex(t):
+        return torch.view_as_real(t.contiguous())
+    return t
+
+
+def selective_scan_fwd_complex(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                               out=None, last_state=None, stream=None):
+    """Selective scan with complex A, B, C; returns ``out`` (real).
+
+    A (dim, dstate) complex64 or (dim, dstate, 2) float32; B, C (batch,
+    seqlen, dstate) complex64 or (batch, seqlen, dstate, 2) in the dtype of u;
+    last_state (batch, dim, dstate, 2) float32 (or a complex64 tensor, whose
+    storage is updated in place) read as h_0 and overwritten with h_L.
+    """
+    io = _io_of(u)
+    batch, seqlen, dim = u.shape
+    A, B, C = _pairs(A, "A"), _pairs(B, "B"), _pairs(C, "C")
+    if last_state is not None and torch.is_complex(last_state):
+        if not last_state.is_contiguous():
+            raise ValueError("last_state must be contiguous")
+        last_state = torch.view_as_real(last_state)
+    dstate = A.shape[1]
+    dev = u.device
+    if out is None:
+        out = torch.empty_like(u)
+    seq, bc = (batch, seqlen, dim), (batch, seqlen, dstate, 2)
+    args = [
+        _ptr(u, "u", u.dtype, seq, dev), _ptr(delta, "delta", u.dtype, seq, dev),
+        _ptr(A, "A", torch.float32, (dim, dstate, 2), dev), _ptr(B, "B", u.dtype, bc, dev),
+        _ptr(C, "C", u.dtype, bc, dev), _ptr(D, "D", torch.float32, (dim,), dev),
+        _ptr(z, "z", u.dtype, seq, dev), _ptr(delta_bias, "delta_bias", torch.float32, (dim,), dev),
+        int(bool(delta_softplus)), _ptr(out, "out", u.dtype, seq, dev),
+        _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate, 2), dev),
+    ]
+    check(lib.ssm_selective_scan_fwd_complex(SSMDims(batch, seqlen, dim, dstate), io, *args,
+                                             _stream_handle(stream)))
     return out
 
 

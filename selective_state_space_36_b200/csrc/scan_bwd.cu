@@ -303,7 +303,7 @@ template <typename IO>
 struct BwdStagedLayout {
     static constexpr int G = 4, NS = 4, NSP = 16, CPB = kBlock / G;
     static constexpr int T = sizeof(IO) == 2 ? 32 : 16;   // steps per staged chunk
-    static constexpr int KC = 8;                          // steps per sub-chunk (checkpoint spacing)
+    static constexpr int KC = kCkptEvery;                 // steps per sub-chunk (checkpoint spacing)
     static constexpr int S = 2;                           // pipeline stages
     static constexpr int ROW = CPB + 32 / (int)sizeof(IO);  // tile row, padded by 32 bytes
     static constexpr int TILE = T * ROW;

@@ -73,11 +73,13 @@ struct StagedCfg {
 #define SSM_ROW_PAD_BYTES 32
 #endif
 
-template <typename IO, int NS, int G, int CPL>
+constexpr int kWarpBlock = 32;
+
+template <typename IO, int NS, int G, int CPL, int TPB = kBlock>
 struct StagedLayout {
     static constexpr int T = StagedCfg<IO>::T;
     static constexpr int S = StagedCfg<IO>::STAGES;
-    static constexpr int GROUPS = kBlock / G;                 // channel groups per block
+    static constexpr int GROUPS = TPB / G;                    // channel groups per block
     static constexpr int CPB = GROUPS * CPL;                  // channels per block
     static constexpr int NSP = NS * G;                        // padded states per channel
     static constexpr int ROW = CPB + (G > 1 ? SSM_ROW_PAD_BYTES / (int)sizeof(IO) : 0);  // tile row (elements)
@@ -116,16 +118,17 @@ __device__ __forceinline__ void store_vals(IO *p, const float (&v)[CPL]) {
     }
 }
 
-template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH>
-__global__ void __launch_bounds__(kBlock)
+template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH, int TPB>
+__global__ void __launch_bounds__(TPB)
 scan_fwd_staged_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
-    using Lay = StagedLayout<IO, NS, G, CPL>;
+    using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
     constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP, ROW = Lay::ROW;
     constexpr int EPV = 16 / sizeof(IO);  // elements per 16-byte piece
     constexpr int ROWV = CPB / EPV;       // pieces per tile row
-    // the checkpoint pass stores a state every 8 steps: its step blocks are 8 long
-    constexpr int KSTEP = MODE == kCkpt ? 8 : KStep<G, CPL>::value;
+    // the checkpoint pass stores a state every kCkptEvery steps: its step
+    // blocks are that long
+    constexpr int KSTEP = MODE == kCkpt ? kCkptEvery : KStep<G, CPL>::value;
     constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
     static_assert(T % KSTEP == 0, "a chunk holds whole step blocks");
     extern __shared__ __align__(16) unsigned char smem[];
@@ -142,6 +145,10 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     const int64_t d0 = (blockIdx.x % tiles) * CPB;
     const int64_t dfirst = d0 + (int64_t)grp * CPL;  // first channel of this group
     const bool active = dfirst < Dm;                  // dim is a multiple of CPL here
+    // checkpoint c of this lane (kCkpt): ckpt[b][c][dfirst][q NS ...]
+    const int64_t ck_stride = Dm * N;
+    float *const ck_base = MODE == kCkpt ? args.ckpt + (b * ((L + kCkptEvery - 1) / kCkptEvery) * Dm + dfirst) * N + q * NS
+                                         : nullptr;
     const int seg = blockIdx.y;
     const int64_t t_begin = (int64_t)seg * args.seg_len;
     const int64_t t_end = t_begin + args.seg_len < L ? t_begin + args.seg_len : L;
@@ -163,7 +170,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         IO *st = stage_ptr(c % S);
         IO *su = st, *sd = st + Lay::TILE, *sz = st + 2 * Lay::TILE;
         IO *rb = st + 3 * Lay::TILE, *rc = rb + Lay::RAW;
-        for (int p = tid; p < T * ROWV; p += kBlock) {
+        for (int p = tid; p < T * ROWV; p += TPB) {
             const int r = p / ROWV, v = p % ROWV;
             const int64_t col = d0 + v * EPV;
             const bool ok = r < rows && col < Dm;
@@ -175,7 +182,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         }
         const int pieces = rows * N / EPV;  // B/C rows of this chunk are contiguous
         const int64_t gbc = (b * L + tc) * N;
-        for (int p = tid; p < pieces; p += kBlock) {
+        for (int p = tid; p < pieces; p += TPB) {
             cp_async16(rb + p * EPV, pB + gbc + p * EPV, true);
             if (MODE != kCkpt) cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
         }
@@ -220,7 +227,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         const IO *rb = st + 3 * Lay::TILE, *rc = rb + Lay::RAW;
         if (rows == T && N == NSP) {
             // whole chunk, no padded states: four values per thread and copy
-            for (int i = 4 * tid; i < T * NSP; i += 4 * kBlock) {
+            for (int i = 4 * tid; i < T * NSP; i += 4 * TPB) {
                 float v[4];
                 io::load4_smem(rb + i, v);
                 *reinterpret_cast<float4 *>(fB + i) = make_float4(v[0], v[1], v[2], v[3]);
@@ -230,7 +237,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 }
             }
         } else {
-            for (int i = tid; i < T * NSP; i += kBlock) {
+            for (int i = tid; i < T * NSP; i += TPB) {
                 const int r = i / NSP, n = i % NSP;
                 const bool ok = r < rows && n < N;
                 fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
@@ -294,10 +301,10 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                         duo[j][cc] = dlo[j][cc] * uvo[j][cc];
                     }
                 }
-                if (MODE == kCkpt && (tc + r0) % args.ckpt_every == 0) {
-                    // the state entering step tc + r0 (ckpt_every is a multiple of KSTEP)
-                    const int64_t nck = (L + args.ckpt_every - 1) / args.ckpt_every;
-                    float *cp = args.ckpt + ((b * nck + (tc + r0) / args.ckpt_every) * Dm + dfirst) * N + q * NS;
+                if (MODE == kCkpt) {
+                    // the state entering step tc + r0 (a multiple of the
+                    // checkpoint spacing: blocks are kCkptEvery steps long)
+                    float *cp = ck_base + ((tc + r0) / kCkptEvery) * ck_stride;
 #pragma unroll
                     for (int p = 0; p < NS / 2; ++p) {
                         if (q * NS + 2 * p < N) cp[2 * p] = h2[0][p].x;
@@ -358,11 +365,11 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     }
 }
 
-template <typename IO, int NS, int G, int CPL, int MODE, bool ZOH>
+template <typename IO, int NS, int G, int CPL, int MODE, bool ZOH, int TPB = kBlock>
 static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
     constexpr bool P = std::is_same<IO, float>::value;
-    using Lay = StagedLayout<IO, NS, G, CPL>;
-    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE, ZOH>;
+    using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
+    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE, ZOH, TPB>;
     // the shared-memory opt-in is a per-device function attribute: set it once per device
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -377,7 +384,7 @@ static cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
         }
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    kern<<<grid, kBlock, Lay::SMEM, st>>>(a);
+    kern<<<grid, TPB, Lay::SMEM, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -385,6 +392,12 @@ template <typename IO, int NS, int G, int CPL, bool ZOH>
 static cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
     constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
     const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
+    if (variant == kVariantSlab && G == 1 && CPL == 1 && a.block_threads == kWarpBlock) {
+        // one-warp blocks of the one-lane layout: 4x the blocks, for balance across SMs
+        constexpr int CPB1 = StagedLayout<IO, NS, 1, 1, kWarpBlock>::CPB;
+        const unsigned bx1 = (unsigned)(a.batch * ((a.dim + CPB1 - 1) / CPB1));
+        return launch_mode<IO, NS, 1, 1, kFull, ZOH, kWarpBlock>(a, dim3(bx1, 1), st);
+    }
     if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull, ZOH>(a, dim3(bx, 1), st);
     if (variant == kVariantCkpt) {
         if (CPL != 1 || ZOH) return cudaErrorInvalidConfiguration;

@@ -15,8 +15,9 @@ constexpr int kBlock = 128;  // threads per block
 constexpr int kChunk = 64;   // time steps of B/C staged in shared memory at once
 
 // kCkpt: forward recurrence only (no readout), storing the state entering
-// every ckpt_every-th step -- the first pass of the backward scan.
+// every kCkptEvery-th step -- the first pass of the backward scan.
 enum ScanMode { kFull = 0, kSegAgg = 1, kSegFinal = 2, kCkpt = 3 };
+constexpr int kCkptEvery = 8;  // kCkpt: steps between stored states
 enum { kVariantSlab = 1, kVariantSplit = 2, kVariantCkpt = 3 };
 // kernel family: generic (direct global loads, any alignment) or staged
 // (cp.async pipeline through shared memory, 16-byte aligned rows)
@@ -36,10 +37,11 @@ struct ScanArgs {
     int zoh_b;        // 1: exact zero-order hold on B (Bbar = expm1(Delta A)/A B); 0: Euler (Delta B)
     int64_t seg_len;  // time steps per segment (== seqlen for one pass)
     int nseg;
-    // kCkpt: states (batch, ceil(seqlen / ckpt_every), dim, dstate); h_0 is
+    // kCkpt: states (batch, ceil(seqlen / kCkptEvery), dim, dstate); h_0 is
     // read from last_state, which is not written
     float *ckpt;
-    int ckpt_every;
+    // staged one-lane slab only: 32 = one-warp blocks, else 128-thread blocks
+    int block_threads;
 };
 
 struct DecodeArgs {
@@ -81,6 +83,9 @@ cudaError_t launch_state_update_bulk(const DecodeArgs &a, bool bf16, uint32_t mi
 // the device status word the kernels' bounded waits report into
 unsigned int read_and_clear_device_status(cudaStream_t st, cudaError_t *err);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
+// complex diagonal A: A, B, C and last_state hold (re, im) pairs
+cudaError_t launch_scan_complex(const ScanArgs &a, bool bf16, cudaStream_t st);
+int64_t scan_complex_channels_per_block();
 // staged second pass (checkpoints every scan_bwd_staged_chunk() steps, from
 // the staged forward kernel in kCkpt mode)
 bool scan_bwd_staged_eligible(const ScanBwdArgs &a, int es);

@@ -53,6 +53,12 @@ constexpr int kTargetBlocksPerSm = 8;
 #endif
 constexpr int kDefaultStagedCpl = SSM_DEFAULT_CPL;
 
+// One-warp blocks for the one-lane staged slab (1) or 128-thread blocks (0).
+#ifndef SSM_ONE_LANE_WARP_BLOCKS
+#define SSM_ONE_LANE_WARP_BLOCKS 0
+#endif
+constexpr bool kOneLaneWarpBlocks = SSM_ONE_LANE_WARP_BLOCKS != 0;
+
 struct DeviceInfo {
     int sms = 148;
     int smem_optin = 227 * 1024;  // dynamic shared memory a block may opt in to
@@ -138,6 +144,7 @@ struct ScanPlan {
     int64_t seg_len = 0;
     size_t ws_bytes = 0;
     int launches = 0;
+    int block_threads = 128;
 };
 
 // Validates sizes and options (not data pointers, which may be absent when
@@ -251,6 +258,13 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
                               (size_t)nseg * channels) * sizeof(float);
         }
     }
+    // The one-lane staged slab runs one-warp blocks: 4x the blocks of 128
+    // threads, so that the last wave is spread over the SMs (at the 1.4B-layer
+    // shape 1024 blocks of 32 channels instead of 256 of 128 on 148 SMs).
+    plan->block_threads = 128;
+    if (kOneLaneWarpBlocks && plan->variant == SSM_VARIANT_SLAB && plan->family == ssm::kFamilyStaged &&
+        plan->g == 1 && plan->cpl == 1 && dims.batch * ((dims.dim + 31) / 32) <= kMaxGridX)
+        plan->block_threads = 32;
     return SSM_OK;
 }
 
@@ -303,6 +317,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     a.zoh_b = p.zoh_b;
     a.seg_len = p.seg_len;
     a.nseg = p.nseg;
+    a.block_threads = p.block_threads;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     if (p.variant == SSM_VARIANT_SLAB) {
@@ -436,6 +451,51 @@ ssm_status ssm_selective_scan_fwd(ssm_dims dims, ssm_dtype io, const void *u, co
                                      out, last_state, nullptr, stream);
 }
 
+ssm_status ssm_selective_scan_fwd_complex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
+                                          const float *A, const void *B, const void *C, const float *D,
+                                          const void *z, const float *delta_bias, int delta_softplus,
+                                          void *out, float *last_state, ssm_stream stream) {
+    g_last_error[0] = 0;
+    size_t es = 0;
+    if (ssm_status s = check_io(io, &es)) return s;
+    if (dims.batch < 0 || dims.seqlen < 0 || dims.dim < 0 || dims.dstate < 0)
+        return fail(SSM_ERR_INVALID_ARG, "negative size (batch %lld, seqlen %lld, dim %lld, dstate %lld)",
+                    (long long)dims.batch, (long long)dims.seqlen, (long long)dims.dim,
+                    (long long)dims.dstate);
+    if (dims.dstate < 1) return fail(SSM_ERR_INVALID_ARG, "dstate must be >= 1");
+    if (dims.dstate > kMaxDstate)
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %lld > %lld", (long long)dims.dstate, (long long)kMaxDstate);
+    if (delta_softplus != 0 && delta_softplus != 1)
+        return fail(SSM_ERR_INVALID_ARG, "delta_softplus must be 0 or 1");
+    const int64_t channels = dims.batch * dims.dim;
+    if (dims.batch != 0 && channels / dims.batch != dims.dim)
+        return fail(SSM_ERR_INVALID_ARG, "batch * dim overflows");
+    if (channels != 0 && dims.seqlen > INT64_MAX / channels / (2 * dims.dstate))
+        return fail(SSM_ERR_INVALID_ARG, "batch * seqlen * dim * dstate overflows");
+    if (channels == 0 || dims.seqlen == 0) return SSM_OK;
+    if (!u || !delta || !A || !B || !C || !out)
+        return fail(SSM_ERR_INVALID_ARG, "u, delta, A, B, C and out are required");
+    if (misaligned(u, es) || misaligned(delta, es) || misaligned(B, es) || misaligned(C, es) ||
+        misaligned(z, es) || misaligned(out, es) || misaligned(A, 4) || misaligned(D, 4) ||
+        misaligned(delta_bias, 4) || misaligned(last_state, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+    const int64_t cpb = ssm::scan_complex_channels_per_block();
+    if (dims.batch * ((dims.dim + cpb - 1) / cpb) > kMaxGridX)
+        return fail(SSM_ERR_UNSUPPORTED, "grid too large");
+    ssm::ScanArgs a{};
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.Dskip = D; a.bias = delta_bias;
+    a.out = out; a.last_state = last_state;
+    a.batch = dims.batch; a.seqlen = dims.seqlen; a.dim = dims.dim;
+    a.dstate = (int)dims.dstate;
+    a.softplus = delta_softplus;
+    a.seg_len = dims.seqlen;
+    a.nseg = 1;
+    cudaError_t e = ssm::launch_scan_complex(a, io == SSM_BF16, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "complex scan launch");
+    return SSM_OK;
+}
+
 ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
                                      const float *A, const void *B, const void *C, const float *D,
                                      const void *z, const float *delta_bias, int delta_softplus,
@@ -560,7 +620,6 @@ ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
         f.seg_len = dims.seqlen;
         f.nseg = 1;
         f.ckpt = a.ckpt;
-        f.ckpt_every = (int)kc;
         e = ssm::launch_scan_staged(f, io == SSM_BF16, ns, g, 1, ssm::kVariantCkpt, st);
         if (e == cudaSuccess) e = ssm::launch_scan_bwd_staged(a, io == SSM_BF16, st);
     } else {

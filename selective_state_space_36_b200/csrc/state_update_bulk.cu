@@ -38,13 +38,25 @@ __device__ unsigned int g_device_status;
 
 namespace {
 
+#ifndef SSM_DECODE_STAGES
+#define SSM_DECODE_STAGES 4
+#endif
+#ifndef SSM_DECODE_AHEAD
+#define SSM_DECODE_AHEAD 2
+#endif
+#ifndef SSM_DECODE_UNIT_FLOATS
+#define SSM_DECODE_UNIT_FLOATS 4096
+#endif
+#ifndef SSM_DECODE_CTAS
+#define SSM_DECODE_CTAS 3
+#endif
 constexpr int kThreads = 256;
-constexpr int kStages = 4;
-constexpr int kAhead = 2;               // units loaded ahead of the one being updated
-constexpr int kUnitFloats = 4096;       // 16 KB of state per unit
+constexpr int kStages = SSM_DECODE_STAGES;
+constexpr int kAhead = SSM_DECODE_AHEAD;          // units loaded ahead of the one being updated
+constexpr int kUnitFloats = SSM_DECODE_UNIT_FLOATS;  // 16 KB of state per unit
 constexpr int kSlices = kUnitFloats / 4;
 constexpr int kPerThread = kSlices / kThreads;
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = SSM_DECODE_CTAS;
 constexpr unsigned long long kWaitNs = 200000000ull;  // a wait gives up after 200 ms
 static_assert(kAhead < kStages, "a buffer must be free before it is refilled");
 

@@ -43,7 +43,8 @@ CHUNK_ROWS = 4096
 
 # stream identifiers: one independent PCG64 family per drawn quantity
 _TID = {"param": 0, "u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "h0": 6,
-        "x": 7, "dt": 8, "dB": 9, "dC": 10, "dz": 11, "dout": 12}
+        "x": 7, "dt": 8, "dB": 9, "dC": 10, "dz": 11, "dout": 12,
+        "B_im": 13, "C_im": 14, "h0_im": 15}
 
 SEQ_NAMES = ("u", "delta", "z", "B", "C")
 
@@ -186,7 +187,7 @@ def _sigma(cfg: ScanConfig, name: str) -> float:
 
 
 def _width(cfg: ScanConfig, name: str) -> int:
-    return cfg.dstate if name in ("B", "C") else cfg.dim
+    return cfg.dstate if name in ("B", "C", "B_im", "C_im") else cfg.dim
 
 
 def _draw_block(cfg: ScanConfig, name: str, b: int, blk: int) -> np.ndarray:
@@ -272,6 +273,56 @@ def draw_dout(cfg: ScanConfig, t0: int = 0, t1: Optional[int] = None,
     """Upstream gradient of the scan output: (batch, t1 - t0, dim) ~ N(0, 1)
     in I/O representation, from its own stream (the loss is sum(dout * out))."""
     return draw_tensor(cfg, "dout", t0, t1, threads)
+
+
+# --------------------------------------------------------------------------
+# complex diagonal A
+# --------------------------------------------------------------------------
+def complex_A(dim: int, dstate: int) -> np.ndarray:
+    """A[d, n] = -1/2 + i pi n for every channel (the S4D-Lin initialisation),
+    as float32 (re, im) pairs of shape (dim, dstate, 2)."""
+    A = np.empty((dim, dstate, 2), dtype=np.float32)
+    A[..., 0] = -0.5
+    A[..., 1] = (np.pi * np.arange(dstate, dtype=np.float64)).astype(np.float32)[None, :]
+    return A
+
+
+def _interleave(re: np.ndarray, im: np.ndarray) -> np.ndarray:
+    out = np.empty(re.shape + (2,), dtype=re.dtype)
+    out[..., 0] = re
+    out[..., 1] = im
+    return out
+
+
+def complex_scan_inputs(cfg: ScanConfig, t0: int = 0, t1: Optional[int] = None,
+                        threads: int = 0) -> Dict[str, Optional[np.ndarray]]:
+    """Inputs of a scan with complex A, B, C, in I/O representation.
+
+    u, delta, z, D, delta_bias as in scan_inputs (same streams); A (dim,
+    dstate, 2) float32 from complex_A; B and C (batch, t1 - t0, dstate, 2)
+    (re, im) pairs, the real parts from the B and C streams and the imaginary
+    parts ~ N(0, 1) from streams of their own; h0 (batch, dim, dstate, 2)
+    float32 or None.
+    """
+    res = scan_inputs(cfg, t0, t1, threads)
+    res["A"] = complex_A(cfg.dim, cfg.dstate)
+    res["B"] = _interleave(res["B"], draw_tensor(cfg, "B_im", t0, t1, threads))
+    res["C"] = _interleave(res["C"], draw_tensor(cfg, "C_im", t0, t1, threads))
+    if res["h0"] is not None:
+        im = np.empty_like(res["h0"])
+        for b in range(cfg.batch):
+            rng = np.random.default_rng([cfg.seed, _TID["h0_im"], b])
+            im[b] = rng.standard_normal((cfg.dim, cfg.dstate), dtype=np.float32) * np.float32(cfg.h0_sigma)
+        res["h0"] = _interleave(res["h0"], im)
+    return res
+
+
+def pairs_to_c128(arr: Optional[np.ndarray], io: str) -> Optional[np.ndarray]:
+    """Exact complex128 values of an (..., 2) array of (re, im) pairs."""
+    if arr is None:
+        return None
+    f = to_f64(arr, io)
+    return f[..., 0] + 1j * f[..., 1]
 
 
 # --------------------------------------------------------------------------

@@ -46,14 +46,15 @@ def out_err(got, ref) -> float:
     return float(np.max(np.abs(got - ref) / (1.0 + np.abs(ref))))
 
 
-def check_out(got, ref, io, what="out"):
+def check_out(got, ref, io, what="out", tol=None):
+    tol = TOL_OUT[io] if tol is None else tol
     e = out_err(got, ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    assert e <= TOL_OUT[io], f"{what}: max err {e:.3e} > {TOL_OUT[io]:.0e} (1+|ref|)"
+    assert e <= tol, f"{what}: max err {e:.3e} > {tol:.1e} (1+|ref|)"
     return e
 
 
-def check_state(got, ref, io, what="last_state"):
+def check_state(got, ref, io, what="last_state", tol=None):
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     if got.size == 0:
         return 0.0
@@ -65,7 +66,8 @@ def check_state(got, ref, io, what="last_state"):
         num = np.max(np.abs(got - ref), axis=-1)
         den = np.max(np.abs(ref), axis=-1) + 1e-30
         e = float(np.max(num / den))
-    assert e <= TOL_STATE[io], f"{what}: max rel err {e:.3e} > {TOL_STATE[io]:.0e}"
+    tol = TOL_STATE[io] if tol is None else tol
+    assert e <= tol, f"{what}: max rel err {e:.3e} > {tol:.1e}"
     return e
 
 
