@@ -73,8 +73,6 @@ struct StagedCfg {
 #define SSM_ROW_PAD_BYTES 32
 #endif
 
-constexpr int kWarpBlock = 32;
-
 template <typename IO, int NS, int G, int CPL, int TPB = kBlock>
 struct StagedLayout {
     static constexpr int T = StagedCfg<IO>::T;
@@ -392,12 +390,6 @@ template <typename IO, int NS, int G, int CPL, bool ZOH>
 static cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
     constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
     const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
-    if (variant == kVariantSlab && G == 1 && CPL == 1 && a.block_threads == kWarpBlock) {
-        // one-warp blocks of the one-lane layout: 4x the blocks, for balance across SMs
-        constexpr int CPB1 = StagedLayout<IO, NS, 1, 1, kWarpBlock>::CPB;
-        const unsigned bx1 = (unsigned)(a.batch * ((a.dim + CPB1 - 1) / CPB1));
-        return launch_mode<IO, NS, 1, 1, kFull, ZOH, kWarpBlock>(a, dim3(bx1, 1), st);
-    }
     if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull, ZOH>(a, dim3(bx, 1), st);
     if (variant == kVariantCkpt) {
         if (CPL != 1 || ZOH) return cudaErrorInvalidConfiguration;

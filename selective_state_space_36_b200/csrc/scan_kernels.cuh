@@ -40,8 +40,6 @@ struct ScanArgs {
     // kCkpt: states (batch, ceil(seqlen / kCkptEvery), dim, dstate); h_0 is
     // read from last_state, which is not written
     float *ckpt;
-    // staged one-lane slab only: 32 = one-warp blocks, else 128-thread blocks
-    int block_threads;
 };
 
 struct DecodeArgs {

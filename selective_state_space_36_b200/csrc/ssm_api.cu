@@ -53,12 +53,6 @@ constexpr int kTargetBlocksPerSm = 8;
 #endif
 constexpr int kDefaultStagedCpl = SSM_DEFAULT_CPL;
 
-// One-warp blocks for the one-lane staged slab (1) or 128-thread blocks (0).
-#ifndef SSM_ONE_LANE_WARP_BLOCKS
-#define SSM_ONE_LANE_WARP_BLOCKS 0
-#endif
-constexpr bool kOneLaneWarpBlocks = SSM_ONE_LANE_WARP_BLOCKS != 0;
-
 struct DeviceInfo {
     int sms = 148;
     int smem_optin = 227 * 1024;  // dynamic shared memory a block may opt in to
@@ -144,7 +138,6 @@ struct ScanPlan {
     int64_t seg_len = 0;
     size_t ws_bytes = 0;
     int launches = 0;
-    int block_threads = 128;
 };
 
 // Validates sizes and options (not data pointers, which may be absent when
@@ -258,13 +251,6 @@ ssm_status plan_scan(ssm_dims dims, ssm_dtype io, const void *u, const void *del
                               (size_t)nseg * channels) * sizeof(float);
         }
     }
-    // The one-lane staged slab runs one-warp blocks: 4x the blocks of 128
-    // threads, so that the last wave is spread over the SMs (at the 1.4B-layer
-    // shape 1024 blocks of 32 channels instead of 256 of 128 on 148 SMs).
-    plan->block_threads = 128;
-    if (kOneLaneWarpBlocks && plan->variant == SSM_VARIANT_SLAB && plan->family == ssm::kFamilyStaged &&
-        plan->g == 1 && plan->cpl == 1 && dims.batch * ((dims.dim + 31) / 32) <= kMaxGridX)
-        plan->block_threads = 32;
     return SSM_OK;
 }
 
@@ -317,7 +303,6 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     a.zoh_b = p.zoh_b;
     a.seg_len = p.seg_len;
     a.nseg = p.nseg;
-    a.block_threads = p.block_threads;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     if (p.variant == SSM_VARIANT_SLAB) {
