@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
     SSM_OK = 0,
     SSM_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad flag */
-    SSM_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (dstate > 64) */
+    SSM_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (dstate > 64) */
     SSM_ERR_CUDA = 3         /* a CUDA call failed; see ssm_last_error() */
 } ssm_status;
 

@@ -13,12 +13,14 @@
 // Layout as the generic real kernel: G = 4 lanes share a channel, lane q
 // holding complex states [q NS, q NS + NS); a block of 128 threads covers 32
 // channels of one batch row; B and C of a chunk of 32 steps are widened to
-// fp32 pairs in shared memory.  Per state and step the decay takes one
-// exponential (SFU in the fast tier) and the accurate sincosf in both tiers:
-// the SFU sine's absolute error (~5e-7) would be a relative phase error of up
-// to 5e-4 per step at the small angles Delta Im A of small Delta, and the
-// phase error of a state adds up over its memory of up to ~1/(Delta |Re A|)
-// steps.
+// fp32 pairs in shared memory; u, delta, z of four steps are loaded ahead of
+// their arithmetic.  Per state and step the decay takes one exponential (SFU
+// in the fast tier) and a sine and cosine of Delta Im A.  The fp32 tier calls
+// sincosf.  The fast tier reduces the angle to [-pi, pi] (Cody and Waite: 2 pi
+// split into a 9-bit head and a tail) and uses the Taylor series below 1/4,
+// where the SFU sine's absolute error (~4e-7) would be a large relative phase
+// error that adds up over a state's memory of ~1/(Delta |Re A|) steps, and the
+// SFU sine and cosine above it.
 #include "scan_kernels.cuh"
 
 namespace ssm {
@@ -28,6 +30,33 @@ namespace {
 constexpr int kCG = 4;                 // lanes per channel
 constexpr int kCCPB = kBlock / kCG;    // channels per block
 constexpr int kCChunk = 32;            // steps of B, C staged at once
+constexpr int kCAhead = 4;             // steps whose u, delta, z are loaded together
+
+constexpr float kInvTwoPi = 0.15915494309189535f;
+constexpr float kTwoPiHi = 6.28125f;               // 9 significant bits: k * kTwoPiHi is exact
+constexpr float kTwoPiLo = 1.9353071795864769e-3f;  // 2 pi - kTwoPiHi
+
+template <bool PRECISE>
+__device__ __forceinline__ void phase(float x, float &s, float &c) {
+    if (PRECISE) {
+        sincosf(x, &s, &c);
+        return;
+    }
+    const float k = rintf(x * kInvTwoPi);
+    const float r = fmaf(-k, kTwoPiLo, fmaf(-k, kTwoPiHi, x));
+    const float r2 = r * r;
+    // sin r = r (1 - r^2/6 (1 - r^2/20 (1 - r^2/42))), cos r = 1 - r^2/2 (1 - r^2/12
+    // (1 - r^2/30 (1 - r^2/56))): truncation below 1e-10 for |r| < 1/4
+    const float ps = r * fmaf(-r2 * (1.f / 6.f), fmaf(-r2 * (1.f / 20.f), fmaf(-r2, 1.f / 42.f, 1.f), 1.f), 1.f);
+    const float pc = fmaf(-r2 * 0.5f,
+                          fmaf(-r2 * (1.f / 12.f), fmaf(-r2 * (1.f / 30.f), fmaf(-r2, 1.f / 56.f, 1.f), 1.f), 1.f),
+                          1.f);
+    float ms, mc;
+    __sincosf(r, &ms, &mc);
+    const bool small = fabsf(r) < 0.25f;
+    s = small ? ps : ms;
+    c = small ? pc : mc;
+}
 
 
 template <typename IO, int NS, bool PRECISE>
@@ -82,10 +111,9 @@ scan_fwd_complex_kernel(const ScanArgs args) {
         }
         __syncthreads();
         if (!active) continue;
-        int64_t off = (b * L + tc) * Dm + d;
-        for (int r = 0; r < rows; ++r, off += Dm) {
-            const float uv = io::load_stream(pu + off);
-            const float s = io::load_stream(pd + off) + bias;
+        const int64_t off0 = (b * L + tc) * Dm + d;
+        // one step: row r of the chunk with its u, (delta + bias), z
+        auto step = [&](int r, float uv, float s, float zv) {
             const float dl = args.softplus ? softplus<PRECISE>(s) : s;
             const float du = dl * uv;
             float yp = 0.f;
@@ -94,7 +122,7 @@ scan_fwd_complex_kernel(const ScanArgs args) {
                 const float2 bv = sB[r][q * NS + i], cv = sC[r][q * NS + i];
                 const float e = decay<PRECISE>(dl, are[i]);
                 float sn, cs;
-                sincosf(dl * aim[i], &sn, &cs);
+                phase<PRECISE>(dl * aim[i], sn, cs);
                 const float ar = e * cs, ai = e * sn;
                 const float nr = fmaf(ar, hr[i], fmaf(-ai, hi[i], du * bv.x));
                 const float ni = fmaf(ar, hi[i], fmaf(ai, hr[i], du * bv.y));
@@ -105,9 +133,27 @@ scan_fwd_complex_kernel(const ScanArgs args) {
             float y = group_sum<G>(yp);
             if (q == 0) {
                 y = fmaf(dskip, uv, y);
-                if (pz) y *= silu<PRECISE>(io::load_stream(pz + off));
-                io::store(po + off, y);
+                if (pz) y *= silu<PRECISE>(zv);
+                io::store(po + off0 + (int64_t)r * Dm, y);
             }
+        };
+        int r = 0;
+        for (; r + kCAhead <= rows; r += kCAhead) {
+            float uv[kCAhead], sv[kCAhead], zv[kCAhead];
+#pragma unroll
+            for (int j = 0; j < kCAhead; ++j) {
+                const int64_t o = off0 + (int64_t)(r + j) * Dm;
+                uv[j] = io::load_stream(pu + o);
+                sv[j] = io::load_stream(pd + o) + bias;
+                zv[j] = (pz && q == 0) ? io::load_stream(pz + o) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < kCAhead; ++j) step(r + j, uv[j], sv[j], zv[j]);
+        }
+        for (; r < rows; ++r) {
+            const int64_t o = off0 + (int64_t)r * Dm;
+            step(r, io::load_stream(pu + o), io::load_stream(pd + o) + bias,
+                 (pz && q == 0) ? io::load_stream(pz + o) : 0.f);
         }
     }
     if (!active || !args.last_state) return;
