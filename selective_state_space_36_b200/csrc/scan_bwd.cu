@@ -299,6 +299,14 @@ scan_bwd_kernel(const ScanBwdArgs args) {
 //   dB, dC     as in the generic kernel: a [KC][channel][state] tile in shared
 //              memory, summed over the 32 channels and added with vector
 //              atomics.
+// Thread groups that share the channel sum of the dB/dC tile (1: 64 threads
+// sum all 32 channels; 2: all 128 threads, 16 channels each, two atomic adds
+// per output -- measured 13 % slower at the 1.4B-layer shape: twice the
+// global atomics and more register spills).
+#ifndef SSM_BWD_RED_SPLIT
+#define SSM_BWD_RED_SPLIT 1
+#endif
+
 template <typename IO>
 struct BwdStagedLayout {
     static constexpr int G = 4, NS = 4, NSP = 16, CPB = kBlock / G;
@@ -597,16 +605,22 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                     dD_acc = fmaf(dyo[j], uo[j], dD_acc);
                 }
             }
-            // ---- dB, dC of the sub-chunk: sum the tile over the block's channels
+            // ---- dB, dC of the sub-chunk: sum the tile over the block's
+            // channels (SPLIT groups of threads each sum CPB / SPLIT channels
+            // and add their partial sums)
             __syncthreads();
-            if (tid < 2 * KC * NQ) {
-                const int nq = tid % NQ;
-                const int kk = (tid / NQ) % KC;
-                const int which = tid / (NQ * KC);  // 0: dC, 1: dB
-                const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) + nq;
+            constexpr int SPLIT = kBlock / (2 * KC * NQ) < SSM_BWD_RED_SPLIT ? kBlock / (2 * KC * NQ)
+                                                                             : SSM_BWD_RED_SPLIT;
+            if (tid < SPLIT * 2 * KC * NQ) {
+                const int task = tid % (2 * KC * NQ), part = tid / (2 * KC * NQ);
+                const int nq = task % NQ;
+                const int kk = (task / NQ) % KC;
+                const int which = task / (NQ * KC);  // 0: dC, 1: dB
+                const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) + nq +
+                                    part * (CPB / SPLIT) * NQ;
                 float2 a01 = make_float2(0.f, 0.f), a23 = a01, b01 = a01, b23 = a01;
 #pragma unroll
-                for (int cc = 0; cc < CPB; cc += 2) {
+                for (int cc = 0; cc < CPB / SPLIT; cc += 2) {
                     const float4 v = col[cc * NQ], w = col[(cc + 1) * NQ];
                     a01 = add2(a01, make_float2(v.x, v.y));
                     a23 = add2(a23, make_float2(v.z, v.w));
