@@ -116,7 +116,7 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
-SCAN_KERNEL_SOURCES = ("scan_fwd_staged.cu", "scan_common.cuh", "scan_kernels.cuh", "ssm_device.cuh")
+SCAN_KERNEL_SOURCES = ("scan_fwd_staged.cuh", "scan_common.cuh", "scan_kernels.cuh", "ssm_device.cuh", "cp_async.cuh")
 
 
 def kernel_source_sha() -> str:
