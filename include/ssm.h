@@ -21,6 +21,13 @@
  * exact form through ssm_selective_scan_fwd_ex.  The D skip and the silu(z)
  * gate are the Mamba block's epilogue fused into the scan.
  *
+ * Entry points: the scan (ssm_selective_scan_fwd, _ex with execution choices
+ * and the exact ZOH form, _noalloc without device allocation), its gradient
+ * (ssm_selective_scan_bwd, _ex), the scan with a complex diagonal A
+ * (ssm_selective_scan_fwd_complex), the one-token decode step
+ * (ssm_selective_state_update), planning (ssm_scan_plan), the device status
+ * word of the bounded waits (ssm_get_device_status) and error reporting.
+ *
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers (cudaMalloc / cudaMallocAsync /
  *    torch CUDA memory) on the current device; the caller owns every buffer.
@@ -36,7 +43,8 @@
  *  - Every pointer must be aligned to its element size; no other alignment is
  *    required.  Sizes are arbitrary (ragged tails are masked); 1 <= dstate <= 64.
  *  - Work is enqueued on "stream" (a cudaStream_t; NULL is the legacy default
- *    stream).  No entry point synchronises the stream or the device.
+ *    stream).  No entry point synchronises the stream or the device, except
+ *    ssm_get_device_status, which synchronises "stream" to read the word.
  *  - Argument errors return SSM_ERR_INVALID_ARG or SSM_ERR_UNSUPPORTED before
  *    anything is enqueued.  A failed launch returns SSM_ERR_CUDA.  The message
  *    of the last failure on the calling thread is ssm_last_error().
