@@ -100,8 +100,15 @@ typedef struct CUstream_st *ssm_stream;
  * GPU, the sequence is split into segments scanned in parallel and joined
  * with the associative combine (a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2); the
  * per-segment carries (8 bytes per (batch, segment, dim, dstate) plus 4 per
- * (batch, segment, dim)) are allocated with cudaMallocAsync on "stream" and
- * released with cudaFreeAsync on the same stream.
+ * (batch, segment, dim)) are taken on "stream" from the library's workspace
+ * pool and released on the same stream (see "Workspace memory" below).
+ *
+ * Workspace memory (the split scan's carries, the backward's checkpoints):
+ * stream-ordered allocations (cudaMallocFromPoolAsync / cudaFreeAsync) from a
+ * pool the library creates per device, which keeps freed memory for later
+ * calls instead of returning it to the driver: a repeated call reuses its
+ * workspace.  The pool holds at most the largest amount of workspace in use
+ * at once, until the process exits.
  */
 ssm_status ssm_selective_scan_fwd(ssm_dims dims, ssm_dtype io,
                                   const void *u, const void *delta, const float *A,
@@ -159,7 +166,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io,
  * call time.  (The paper has no counterpart: this is a deployment option.)
  *
  * Who needs it: a serving runtime that reserved nearly all of the GPU's memory
- * for its own pool at start-up, so a cudaMallocAsync from the driver's pool
+ * for its own pool at start-up, so growing the library's workspace pool
  * would fail or fragment that reservation; a real-time or latency-budgeted
  * path that may not take the allocator's locks; an embedding where all device
  * memory is owned by the host application.  The only scratch the scan needs
@@ -259,8 +266,9 @@ ssm_status ssm_selective_scan_fwd_complex(ssm_dims dims, ssm_dtype io, const voi
  * atomics, so their last bits depend on the order blocks finish in.
  * Workspace: (batch, ceil(seqlen / K), dim, dstate) float32 state checkpoints
  * (K = 8 on the staged path; 16, 8 or 4 on the generic one for dstate <= 16,
- * 32, 64), taken with cudaMallocAsync and released with cudaFreeAsync on
- * "stream".  Output buffers must not overlap each other or any input.
+ * 32, 64), taken from the library's workspace pool on "stream" (see
+ * ssm_selective_scan_fwd).  Output buffers must not overlap each other or any
+ * input.
  */
 ssm_status ssm_selective_scan_bwd(ssm_dims dims, ssm_dtype io, const void *u, const void *delta,
                                   const float *A, const void *B, const void *C, const float *D,

@@ -100,6 +100,44 @@ void scan_layout(int64_t dstate, int64_t channels, int sms, int lanes_req, int *
     *g = 4;
 }
 
+// Workspaces (the split scan's carries, the backward's checkpoints) come from
+// a stream-ordered pool per device that keeps freed memory (no release
+// threshold): a repeated call reuses its workspace instead of having it
+// mapped again after every synchronisation, as the device's default pool
+// would.  The pool holds at most the largest workspace in use at once.
+constexpr int kMaxPoolDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxPoolDevices] = {};
+
+cudaError_t workspace_alloc(void **p, size_t bytes, cudaStream_t st) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxPoolDevices) return cudaMallocAsync(p, bytes, st);
+    cudaMemPool_t pool = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mu);
+        if (!g_pool[dev]) {
+            cudaMemPoolProps props{};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t created = nullptr;
+            e = cudaMemPoolCreate(&created, &props);
+            if (e != cudaSuccess) return e;
+            uint64_t keep = UINT64_MAX;
+            e = cudaMemPoolSetAttribute(created, cudaMemPoolAttrReleaseThreshold, &keep);
+            if (e != cudaSuccess) {
+                (void)cudaMemPoolDestroy(created);
+                return e;
+            }
+            g_pool[dev] = created;
+        }
+        pool = g_pool[dev];
+    }
+    return cudaMallocFromPoolAsync(p, bytes, pool, st);
+}
+
 ssm_status check_io(ssm_dtype io, size_t *elem) {
     if (io == SSM_F32) { *elem = 4; return SSM_OK; }
     if (io == SSM_BF16) { *elem = 2; return SSM_OK; }
@@ -311,7 +349,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
         return SSM_OK;
     }
     void *ws = nullptr;
-    cudaError_t e = cudaMallocAsync(&ws, p.ws_bytes, st);
+    cudaError_t e = workspace_alloc(&ws, p.ws_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
     const size_t n_h0 = (size_t)dims.batch * dims.dim * dims.dstate;
     a.seg_h0 = static_cast<float *>(ws);
@@ -330,7 +368,7 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
 // Sequence-split scan without any device allocation.
 //
 // The split scan needs a carry buffer (segment end states and Delta sums).
-// ssm_selective_scan_fwd takes it from cudaMallocAsync; this variant takes it
+// ssm_selective_scan_fwd takes it from the workspace pool; this variant takes it
 // from the fixed scratch array below, which the CUDA runtime places in device
 // memory when the library's module is loaded on a GPU and keeps until the
 // process exits.  Host code must not pass the array's name to a kernel (on the
@@ -590,7 +628,7 @@ ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     const int64_t kc = staged ? ssm::scan_bwd_staged_chunk() : ssm::scan_bwd_chunk((int)dims.dstate);
     const size_t ws_bytes = (size_t)channels * ((dims.seqlen + kc - 1) / kc) * dims.dstate * sizeof(float);
     void *ws = nullptr;
-    cudaError_t e = cudaMallocAsync(&ws, ws_bytes, st);
+    cudaError_t e = workspace_alloc(&ws, ws_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "checkpoint workspace allocation");
     a.ckpt = static_cast<float *>(ws);
     if (staged) {
