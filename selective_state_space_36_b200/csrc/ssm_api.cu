@@ -53,6 +53,11 @@ constexpr int kTargetBlocksPerSm = 8;
 #endif
 constexpr int kDefaultStagedCpl = SSM_DEFAULT_CPL;
 
+// Lanes per channel of the backward's checkpoint pass (0: the forward's choice).
+#ifndef SSM_BWD_CKPT_LANES
+#define SSM_BWD_CKPT_LANES 4
+#endif
+
 struct DeviceInfo {
     int sms = 148;
     int smem_optin = 227 * 1024;  // dynamic shared memory a block may opt in to
@@ -611,8 +616,9 @@ ssm_status ssm_selective_scan_bwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
     if (staged) {
         const DeviceInfo di = device_info();
         // the checkpoint pass (8-step blocks, no readout) measured faster with
-        // four lanes per channel than with one at the 1.4B-layer shape
-        scan_layout(dims.dstate, channels, di.sms, 4, &ns, &g);
+        // four lanes per channel than with one at the 1.4B-layer shape (a
+        // whole backward call: 2.19 vs 2.49 ms)
+        scan_layout(dims.dstate, channels, di.sms, SSM_BWD_CKPT_LANES, &ns, &g);
         if (ssm::staged_smem_bytes(io == SSM_BF16, ns, g, 1) > (size_t)di.smem_optin)
             return fail(SSM_ERR_UNSUPPORTED, "staged backward needs more shared memory than the device has");
     }

@@ -145,9 +145,9 @@ def test_bwd_is_linear_in_dout(family):
         assert e <= 1e-4, (k, e)
 
 
-def test_bwd_staged_with_one_lane_checkpoint_pass(lib):
-    # 32,768 channels: the checkpointing forward pass takes the one-lane
-    # layout (all 16 states in one thread) that large problems get
+def test_bwd_staged_at_a_one_lane_forward_shape(lib):
+    # 32,768 channels, where the forward scan takes the one-lane layout (its
+    # checkpoint pass keeps four lanes per channel): all gradients
     plan = lib.scan_plan(2, 48, 16384, 16, "bf16")
     assert plan["lanes"] == 1
     _check("bf16", 2, 48, 16384, 16, 17, family="staged", h0_sigma=0.5)
