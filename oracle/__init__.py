@@ -24,6 +24,11 @@ Parity status of each function (what pins it lives in tests/test_oracle_pins.py)
                           part is zero, brute-force complex unrolled sum, LTI
                           convolution with a complex kernel, pure-rotation
                           closed form (sign of the phase).
+  ssd_scan                pinned: equal to scan with A[d, :] = A_head and the
+                          head's Delta for every channel of the head; the
+                          quadratic (masked attention) form; the chunked block
+                          decomposition at several chunk lengths; Delta -> 0;
+                          split/resume.
 """
 from __future__ import annotations
 
@@ -70,6 +75,8 @@ def _bind(path: str):
     lib.oracle_selective_scan_complex.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [ctypes.c_int, _dp, _dp]
     lib.oracle_selective_scan_bwd.restype = ctypes.c_int
     lib.oracle_selective_scan_bwd.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [ctypes.c_int] + [_dp] * 11
+    lib.oracle_ssd_scan.restype = ctypes.c_int
+    lib.oracle_ssd_scan.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int, _dp, _dp]
     return lib
 
 
@@ -241,6 +248,41 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, _lib_handle=None):
     return out, st
 
 
+def ssd_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
+             _lib_handle=None):
+    """Mamba-2 SSD layer (linear / recurrent form) in fp64.
+
+    x, z: (batch, seqlen, heads, headdim); dt: (batch, seqlen, heads) (raw);
+    A, D, dt_bias: (heads,); B, C: (batch, seqlen, groups, dstate);
+    h0: (batch, heads, headdim, dstate) or None.
+    Returns (out (batch, seqlen, heads, headdim), last_state (batch, heads, headdim, dstate)).
+    """
+    x = np.asarray(x)
+    batch, seqlen, heads, headdim = x.shape
+    groups, dstate = np.asarray(B).shape[2:]
+    keep = []
+
+    def p(a, shape, name):
+        arr, ptr = _c64(a, shape, name)
+        keep.append(arr)
+        return ptr
+
+    seq = (batch, seqlen, heads, headdim)
+    bc = (batch, seqlen, groups, dstate)
+    px, pdt = p(x, seq, "x"), p(dt, (batch, seqlen, heads), "dt")
+    pA, pB, pC = p(A, (heads,), "A"), p(B, bc, "B"), p(C, bc, "C")
+    pD, pz, pb = p(D, (heads,), "D"), p(z, seq, "z"), p(dt_bias, (heads,), "dt_bias")
+    out = np.zeros(seq, dtype=np.float64)
+    state = (np.zeros((batch, heads, headdim, dstate), dtype=np.float64) if h0 is None
+             else np.array(h0, dtype=np.float64, order="C", copy=True).reshape(batch, heads, headdim, dstate))
+    rc = (_lib_handle or _load()).oracle_ssd_scan(batch, seqlen, heads, headdim, groups, dstate, px, pdt, pA,
+                                                  pB, pC, pD, pz, pb, int(bool(dt_softplus)),
+                                                  out.ctypes.data_as(_dp), state.ctypes.data_as(_dp))
+    if rc != 0:
+        raise RuntimeError(f"oracle_ssd_scan failed with code {rc}")
+    return out, state
+
+
 class Variant:
     """The same API bound to another build of the oracle source (used by the
     mutation tests, which compile deliberately broken copies)."""
@@ -259,6 +301,9 @@ class Variant:
 
     def scan_complex(self, *a, **kw):
         return scan_complex(*a, _lib_handle=self._h, **kw)
+
+    def ssd_scan(self, *a, **kw):
+        return ssd_scan(*a, _lib_handle=self._h, **kw)
 
 
 def compile_variant(source: str, path: str) -> "Variant":

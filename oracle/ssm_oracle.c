@@ -370,3 +370,64 @@ int oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, double *stat
     }
     return ORACLE_OK;
 }
+
+/*
+ * Mamba-2's structured state space duality (SSD) layer, in its linear
+ * (recurrent) form ("Transformers are SSMs" review, nubint.ai: 提案手法 --
+ * an SSM is a matrix transformation; the linear recurrence and the quadratic,
+ * attention-like form compute the same map).  The review prints no formula;
+ * the plain reading, shared with the Mamba notes' selective SSM, is:
+ *   heads h = 0..H-1 of P channels each; groups g = 0..G-1 of H/G heads that
+ *   share B_t and C_t (the review's grouped-value attention); A is one scalar
+ *   per head, so Abar is a scalar times the identity;
+ *   Delta_t = softplus(dt[b,t,h] + dt_bias[h]) (or the plain sum), one per head;
+ *   for every channel (b, h, p) and state n, in time order:
+ *       state[n] = exp(Delta_t A_h) state[n] + Delta_t B[b,t,g,n] x[b,t,h,p]
+ *       y        = sum_n C[b,t,g,n] state[n] + D_h x[b,t,h,p]
+ *       out      = y * silu(z[b,t,h,p])   (z NULL: no gate; D NULL: no skip)
+ * Layouts (dense, row-major): x, z, out (batch, seqlen, heads, headdim);
+ * dt (batch, seqlen, heads); A, D, dt_bias (heads); B, C (batch, seqlen,
+ * groups, dstate); state (batch, heads, headdim, dstate), h0 in and h_L out
+ * (NULL: h0 = 0, not returned).  Single-threaded; returns 0 on success.
+ */
+int oracle_ssd_scan(int64_t batch, int64_t seqlen, int64_t heads, int64_t headdim, int64_t groups,
+                    int64_t dstate, const double *x, const double *dt, const double *A,
+                    const double *B, const double *C, const double *D, const double *z,
+                    const double *dt_bias, int dt_softplus, double *out, double *state)
+{
+    if (batch < 0 || seqlen < 0 || heads < 0 || headdim < 0 || groups < 1 || dstate < 0) return ORACLE_BAD_ARG;
+    if (heads % groups != 0) return ORACLE_BAD_ARG;
+    if (batch * heads * headdim == 0) return ORACLE_OK;
+    if (seqlen > 0 && (!x || !dt || !A || !B || !C || !out)) return ORACLE_BAD_ARG;
+    const int64_t L = seqlen, H = heads, P = headdim, N = dstate, hpg = heads / groups;
+    double *h = (double *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+    if (!h) return ORACLE_NO_MEM;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t hd = 0; hd < H; ++hd) {
+            const int64_t g = hd / hpg;
+            for (int64_t p = 0; p < P; ++p) {
+                double *st = state ? state + ((b * H + hd) * P + p) * N : NULL;
+                for (int64_t n = 0; n < N; ++n) h[n] = st ? st[n] : 0.0;
+                for (int64_t t = 0; t < L; ++t) {
+                    const double s = dt[(b * L + t) * H + hd] + (dt_bias ? dt_bias[hd] : 0.0);
+                    const double dlt = dt_softplus ? oracle_softplus(s) : s;
+                    const double abar = exp(dlt * A[hd]);
+                    const int64_t xi = ((b * L + t) * H + hd) * P + p;
+                    const int64_t bi = ((b * L + t) * groups + g) * N;
+                    const double xv = x[xi];
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        h[n] = abar * h[n] + dlt * B[bi + n] * xv;
+                        acc += C[bi + n] * h[n];
+                    }
+                    double y = acc + (D ? D[hd] * xv : 0.0);
+                    if (z) y *= oracle_silu(z[xi]);
+                    out[xi] = y;
+                }
+                if (st)
+                    for (int64_t n = 0; n < N; ++n) st[n] = h[n];
+            }
+        }
+    free(h);
+    return ORACLE_OK;
+}

@@ -45,6 +45,15 @@ MUTANTS = {
     "complex_B_real_part_only": ("h[n] = abar * h[n] + (dlt * bn) * x;", "h[n] = abar * h[n] + (dlt * creal(bn)) * x;"),
     "complex_h0_imaginary_dropped": ("h[n] = state ? state[2 * (so + n)] + I * state[2 * (so + n) + 1] : 0.0;",
                                      "h[n] = state ? state[2 * (so + n)] : 0.0;"),
+    # Mamba-2 SSD
+    "ssd_group_index": ("const int64_t g = hd / hpg;", "const int64_t g = hd % groups;"),
+    "ssd_input_without_delta": ("h[n] = abar * h[n] + dlt * B[bi + n] * xv;", "h[n] = abar * h[n] + B[bi + n] * xv;"),
+    "ssd_decay_after_input": ("h[n] = abar * h[n] + dlt * B[bi + n] * xv;", "h[n] = abar * (h[n] + dlt * B[bi + n] * xv);"),
+    "ssd_readout_with_B": ("acc += C[bi + n] * h[n];", "acc += B[bi + n] * h[n];"),
+    "ssd_state_transposed": ("double *st = state ? state + ((b * H + hd) * P + p) * N : NULL;",
+                             "double *st = state ? state + (b * H + hd) * P * N + p : NULL;"),
+    "ssd_bias_ignored": ("const double s = dt[(b * L + t) * H + hd] + (dt_bias ? dt_bias[hd] : 0.0);",
+                         "const double s = dt[(b * L + t) * H + hd];"),
     # backward
     "bwd_adjoint_not_decayed": ("lam[n] *= abar;", "(void)0;"),
     "bwd_dA_without_decay": ("dA[d * N + n] += lam[n] * hprev * abar * dl[t];",

@@ -500,3 +500,169 @@ def test_complex_pure_rotation_closed_form(oracle_mod):
                                           delta_softplus=False)
         np.testing.assert_allclose(out[0, :, 0], ref, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(st[0, 0, 0], dl * np.exp(1j * w * dl * (L - 1)), rtol=1e-12)
+
+
+# ------------------------------------------------------------------ Mamba-2 SSD
+# "Transformers are SSMs" review (nubint.ai), 提案手法: the SSM as a matrix
+# transformation (a semiseparable matrix), its linear (recurrent) and
+# quadratic (attention-like) forms computing the same map, and the block
+# decomposition of that matrix behind the SSD algorithm.  The oracle's
+# ssd_scan is the linear form; these pins compare it with the selective-scan
+# oracle (scalar A per head is a diagonal A with equal entries), with the
+# quadratic form written as a masked matrix product, and with the chunked
+# block decomposition, each computed here in numpy.
+
+def _ssd_case(rng, batch=2, L=13, H=4, P=3, G=2, N=5, softplus=True, bias=True, gate=True, dskip=True,
+              h0=True):
+    return dict(
+        x=rng.standard_normal((batch, L, H, P)),
+        dt=rng.standard_normal((batch, L, H)) * 0.7,
+        A=-rng.uniform(0.2, 2.0, size=H),
+        B=rng.standard_normal((batch, L, G, N)),
+        C=rng.standard_normal((batch, L, G, N)),
+        D=rng.standard_normal(H) if dskip else None,
+        z=rng.standard_normal((batch, L, H, P)) if gate else None,
+        dt_bias=rng.standard_normal(H) * 0.5 if bias else None,
+        dt_softplus=softplus,
+        h0=rng.standard_normal((batch, H, P, N)) if h0 else None)
+
+
+def _ssd_delta(c):
+    s = c["dt"] + (c["dt_bias"] if c["dt_bias"] is not None else 0.0)
+    return np.logaddexp(0.0, s) if c["dt_softplus"] else s
+
+
+def _ssd_epilogue(c, y):
+    H = c["x"].shape[2]
+    if c["D"] is not None:
+        y = y + c["D"].reshape(1, 1, H, 1) * c["x"]
+    if c["z"] is not None:
+        y = y * c["z"] * expit(c["z"])
+    return y
+
+
+def _ssd_quadratic(c):
+    """Quadratic (masked attention) form: per (b, h), with Delta's running sum
+    S_t = sum_{r<=t} Delta_r, y = (Lmask o (C B^T)) diag(Delta) X + C_t
+    e^{A S_t} h0, Lmask[t, s] = e^{A (S_t - S_s)} for s <= t, else 0."""
+    x, A, B, C = c["x"], c["A"], c["B"], c["C"]
+    batch, L, H, P = x.shape
+    G = B.shape[2]
+    dl = _ssd_delta(c)
+    y = np.zeros_like(x)
+    last = np.zeros((batch, H, P, B.shape[3]))
+    for b in range(batch):
+        for h in range(H):
+            g = h // (H // G)
+            S = np.cumsum(dl[b, :, h])
+            mask = np.tril(np.exp(A[h] * (S[:, None] - S[None, :])))
+            M = mask * (C[b, :, g] @ B[b, :, g].T) * dl[b, None, :, h]
+            y[b, :, h] = M @ x[b, :, h]
+            wlast = np.exp(A[h] * (S[-1] - S)) * dl[b, :, h]
+            last[b, h] = (x[b, :, h] * wlast[:, None]).T @ B[b, :, g]
+            if c["h0"] is not None:
+                decay = np.exp(A[h] * S)
+                y[b, :, h] += decay[:, None] * (C[b, :, g] @ c["h0"][b, h].T)
+                last[b, h] += np.exp(A[h] * S[-1]) * c["h0"][b, h]
+    return _ssd_epilogue(c, y), last
+
+
+def _ssd_chunked(c, Q):
+    """Block decomposition at chunk length Q: diagonal blocks by the quadratic
+    form inside each chunk, off-diagonal blocks through the chunk-boundary
+    states, which pass from chunk to chunk with the chunk's total decay."""
+    x, A, B, C = c["x"], c["A"], c["B"], c["C"]
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dl = _ssd_delta(c)
+    y = np.zeros_like(x)
+    last = np.zeros((batch, H, P, N))
+    for b in range(batch):
+        for h in range(H):
+            g = h // (H // G)
+            st = c["h0"][b, h].copy() if c["h0"] is not None else np.zeros((P, N))
+            for t0 in range(0, L, Q):
+                sl = slice(t0, min(L, t0 + Q))
+                d, xx, Bc, Cc = dl[b, sl, h], x[b, sl, h], B[b, sl, g], C[b, sl, g]
+                S = np.cumsum(d)
+                mask = np.tril(np.exp(A[h] * (S[:, None] - S[None, :])))
+                y[b, sl, h] = (mask * (Cc @ Bc.T) * d[None, :]) @ xx          # diagonal block
+                y[b, sl, h] += np.exp(A[h] * S)[:, None] * (Cc @ st.T)         # from the carried state
+                w = np.exp(A[h] * (S[-1] - S)) * d
+                st = np.exp(A[h] * S[-1]) * st + (xx * w[:, None]).T @ Bc      # state at the chunk's end
+            last[b, h] = st
+    return _ssd_epilogue(c, y), last
+
+
+def test_ssd_is_the_selective_scan_with_scalar_A_per_head(oracle_mod):
+    rng = np.random.default_rng(40)
+    c = _ssd_case(rng)
+    out, last = oracle_mod.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                                    dt_bias=c["dt_bias"], dt_softplus=c["dt_softplus"], h0=c["h0"])
+    batch, L, H, P = c["x"].shape
+    G, N = c["B"].shape[2:]
+    hpg = H // G
+    for g in range(G):
+        hs = slice(g * hpg, (g + 1) * hpg)
+        ch = hpg * P
+        rep = lambda a: np.repeat(a[hs], P)  # one value per channel (h, p) of the group
+        o, s = oracle_mod.scan(c["x"][:, :, hs].reshape(batch, L, ch),
+                               np.repeat(c["dt"][:, :, hs], P, axis=2), np.repeat(rep(c["A"])[:, None], N, 1),
+                               c["B"][:, :, g], c["C"][:, :, g], D=rep(c["D"]),
+                               z=c["z"][:, :, hs].reshape(batch, L, ch), delta_bias=rep(c["dt_bias"]),
+                               delta_softplus=c["dt_softplus"], h0=c["h0"][:, hs].reshape(batch, ch, N))
+        np.testing.assert_array_equal(out[:, :, hs].reshape(batch, L, ch), o)
+        np.testing.assert_array_equal(last[:, hs].reshape(batch, ch, N), s)
+
+
+@pytest.mark.parametrize("variant", ["full", "no_softplus", "no_gate_no_skip", "no_bias_no_h0"])
+def test_ssd_equals_quadratic_form(oracle_mod, variant):
+    rng = np.random.default_rng(41)
+    kw = dict(full={}, no_softplus=dict(softplus=False), no_gate_no_skip=dict(gate=False, dskip=False),
+              no_bias_no_h0=dict(bias=False, h0=False))[variant]
+    c = _ssd_case(rng, **kw)
+    if not c["dt_softplus"]:
+        c["dt"] = np.abs(c["dt"])  # a positive step keeps the decays bounded
+    out, last = oracle_mod.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                                    dt_bias=c["dt_bias"], dt_softplus=c["dt_softplus"], h0=c["h0"])
+    ro, rl = _ssd_quadratic(c)
+    np.testing.assert_allclose(out, ro, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(last, rl, rtol=1e-10, atol=1e-11)
+
+
+@pytest.mark.parametrize("Q", [1, 3, 7, 64])
+def test_ssd_equals_chunked_block_decomposition(oracle_mod, Q):
+    rng = np.random.default_rng(42)
+    c = _ssd_case(rng, L=23, H=4, P=2, G=1, N=6)
+    out, last = oracle_mod.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                                    dt_bias=c["dt_bias"], dt_softplus=c["dt_softplus"], h0=c["h0"])
+    ro, rl = _ssd_chunked(c, Q)
+    np.testing.assert_allclose(out, ro, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(last, rl, rtol=1e-10, atol=1e-11)
+
+
+def test_ssd_delta_zero_keeps_state_exactly(oracle_mod):
+    rng = np.random.default_rng(43)
+    c = _ssd_case(rng, bias=False, softplus=False, gate=False)
+    c["dt"][:] = 0.0
+    out, last = oracle_mod.ssd_scan(c["x"], c["dt"], c["A"], c["B"], c["C"], D=c["D"], z=None,
+                                    dt_bias=None, dt_softplus=False, h0=c["h0"])
+    np.testing.assert_array_equal(last, c["h0"])
+    H = c["x"].shape[2]
+    G = c["B"].shape[2]
+    for h in range(H):
+        g = h // (H // G)
+        ref = np.einsum("btn,bpn->btp", c["C"][:, :, g], c["h0"][:, h]) + c["D"][h] * c["x"][:, :, h]
+        np.testing.assert_allclose(out[:, :, h], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_ssd_split_and_resume_equals_one_pass(oracle_mod):
+    rng = np.random.default_rng(44)
+    c = _ssd_case(rng, L=17)
+    args = lambda sl, h0: (c["x"][:, sl], c["dt"][:, sl], c["A"], c["B"][:, sl], c["C"][:, sl])
+    kw = lambda sl: dict(D=c["D"], z=c["z"][:, sl], dt_bias=c["dt_bias"], dt_softplus=True)
+    out, last = oracle_mod.ssd_scan(*args(slice(None), None), h0=c["h0"], **kw(slice(None)))
+    o1, s1 = oracle_mod.ssd_scan(*args(slice(0, 6), None), h0=c["h0"], **kw(slice(0, 6)))
+    o2, s2 = oracle_mod.ssd_scan(*args(slice(6, None), None), h0=s1, **kw(slice(6, None)))
+    np.testing.assert_array_equal(np.concatenate([o1, o2], axis=1), out)
+    np.testing.assert_array_equal(s2, last)
