@@ -6,19 +6,25 @@ softplus(Delta), discretisation, recurrence, readout, D skip, silu(z) gate, the
 fp32 state in and out.  Inputs are seeded synthetic data of that shape.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload mamba1p4b|mamba130m|longseq|decode|mamba1p4b_bwd|mamba130m_complex]
+                  [--workload mamba1p4b|mamba130m|longseq|decode|mamba1p4b_bwd|mamba130m_complex|mamba2_ssd]
 
 The other workloads measure the remaining hot-path kernels the same way:
 mamba130m (batch 8, L 2048, dim 1536), longseq (batch 1, L 1,048,576, dim 1536:
 the sequence-split variant) and decode (one ssm_selective_state_update step at
 batch 256, dim 5120, N 16; two state buffers alternate so that the 84 MB state
 cannot simply stay in the 126 MB L2) and mamba1p4b_bwd (one
-ssm_selective_scan_bwd call on the 1.4B-layer workload with a seeded dout).
+ssm_selective_scan_bwd call on the 1.4B-layer workload with a seeded dout),
+mamba130m_complex (the scan with a complex diagonal A) and mamba2_ssd (one
+ssm_ssd_scan_fwd call: Mamba-2's SSD layer, batch 8, L 2048, 64 heads of 64,
+dstate 128, on the tensor cores).
 
-Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of
-the workload on its GPU (independent batches, no collective on the data path:
-weak scaling); the timed region is bracketed by a barrier and a device
-synchronisation and its length is the maximum over ranks.
+Prints one JSON line (rank 0).  With --gpus N > 1 the script starts N ranks
+itself (torchrun, one process per GPU) unless it already runs under one.  The
+N ranks share one global workload of N times the workload's batch, whose
+batch rows are split over the ranks (selective_state_space_36_b200.shard):
+weak scaling, no collective on the data path.  The timed region is bracketed
+by a barrier and a device synchronisation and its length is the maximum over
+ranks; value = the global workload's elements over that time.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on the host
 cores on a bounded sample of the same workload (rank 0 only).
@@ -46,7 +52,8 @@ UNIT = "Gelem/s"
 WORKLOAD = I.MAMBA1P4B
 L2_BYTES = 126 * 1024 * 1024
 WORKLOADS = {"mamba1p4b": I.MAMBA1P4B, "mamba130m": I.MAMBA130M, "longseq": I.LONGSEQ,
-             "decode": I.DECODE, "mamba1p4b_bwd": I.MAMBA1P4B, "mamba130m_complex": I.MAMBA130M}
+             "decode": I.DECODE, "mamba1p4b_bwd": I.MAMBA1P4B, "mamba130m_complex": I.MAMBA130M,
+             "mamba2_ssd": I.MAMBA2_1P3B}
 SCAN_METRICS = {
     "mamba1p4b": METRIC,
     "mamba130m": "selective-scan fwd Gelem/s (B·L·D) at 130M-layer shape; % of HBM roofline",
@@ -78,21 +85,23 @@ def bwd_algorithmic_bytes(cfg: I.ScanConfig, ckpt_every: int = 8) -> int:
     return seq + bc + ck
 
 
-def alu_ceiling_per_sm_clock(dstate: int = 16) -> float:
+def alu_ceiling_per_sm_clock(dstate: int = 16, sfu_decays=None) -> float:
     """Elements per SM clock that the arithmetic of the scan allows on B200.
 
-    Model built from measured unit costs (probes/pipe_rates.cu): an SFU op
-    (ex2, tanh) occupies ~4 issue cycles of its SM sub-partition and its unit
-    for 8 cycles per warp; an f32x2 op 1 issue cycle.  Per element the method
-    needs dstate decays exp(Delta A_n), 2 SFU ops for softplus and silu, 2
-    packed FP32 issue cycles per state (Delta A, Delta u B, state FMA, readout
-    FMA) and ~14 more issue cycles (softplus polynomial, gate, loads, stores).
-    A decay costs 4 issue cycles on the SFU or ~4.5 as an FMA-pipe polynomial;
-    the best split of the decays between the two balances the SFU unit
-    against the issue slots.  Four sub-partitions x 32 lanes per SM clock.
+    Model built from measured unit costs (B200 pipe rates: the SFU returns 16
+    ex2 per SM clock; next to scalar FFMA an SFU instruction takes ~4 issue
+    cycles of its SM sub-partition and its unit for 8 cycles per warp; an
+    f32x2 op takes 1 issue cycle).  Per element the method needs dstate
+    decays exp(Delta A_n), 2 SFU ops for softplus and silu, 2 packed FP32
+    issue cycles per state (Delta A, Delta u B, state FMA, readout FMA) and
+    ~14 more issue cycles (softplus polynomial, gate, loads, stores).  A
+    decay costs 4 issue cycles on the SFU or ~4.5 as an FMA-pipe polynomial.
+    With ``sfu_decays`` = m of the dstate decays on the SFU (the rest on the
+    FMA pipe) the ceiling is that of the shipped code; with None, the best m.
+    Four sub-partitions x 32 lanes per SM clock.
     """
     best = 0.0
-    for m in range(dstate + 1):            # decays on the SFU
+    for m in (range(dstate + 1) if sfu_decays is None else [min(dstate, sfu_decays * dstate // 16)]):
         sfu_cycles = 8.0 * (m + 2)
         issue_cycles = 4.0 * (m + 2) + 4.5 * (dstate - m) + 2.0 * dstate + 14.0
         best = max(best, 128.0 / max(sfu_cycles, issue_cycles))
@@ -151,10 +160,23 @@ def committed_traffic(sha: str):
 
 
 # ------------------------------------------------------------ multi-GPU logic
-def rank_config(rank: int) -> I.ScanConfig:
-    """Each rank scans its own copy of the workload (independent batches: no
-    exchange on the data path); rank 0's is the single-GPU workload."""
-    return WORKLOAD if rank == 0 else WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank)
+def sharded_workload(args, rank: int, world: int):
+    """The global workload of a run on `world` GPUs and this rank's share.
+
+    Weak scaling: the global batch is the workload's batch times the number
+    of GPUs, and the batch rows are split over the ranks (scan_shard), so each
+    GPU scans the workload's shape; a run on one GPU is the workload itself.
+    Rows are drawn by their global index, so the gathered result of N ranks
+    equals one process scanning the global batch."""
+    from selective_state_space_36_b200.shard import scan_shard
+    cfg = WORKLOADS[args.workload]
+    if getattr(args, "batch", 0) or getattr(args, "seqlen", 0):
+        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
+        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"{args.workload}_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
+    if world > 1:
+        gb = cfg.batch * world
+        cfg = cfg.with_(batch=gb, name=cfg.name.replace(f"_b{cfg.batch}_", f"_b{gb}_", 1))
+    return cfg, scan_shard(cfg.batch, cfg.dim, world, rank)
 
 
 def max_over_ranks(values, device=None):
@@ -222,73 +244,74 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_rate(cfg: I.ScanConfig, budget_s: float):
-    """The fp64 oracle, as it stands, on blocks of the workload (one batch row,
-    every channel, 2048 consecutive steps each) until ``budget_s`` seconds have
-    been spent (at least one block) or the workload is done.  Returns
-    (Gelem/s, threads, elements, seconds)."""
-    import oracle
+# The oracle's sample, the same for the reference arm and the cpu_baseline of
+# our arm: one batch row of the workload, its first REF_CHANNELS channels,
+# every time step (channels are independent, so this is the workload's own
+# arithmetic on a bounded part of it).
+REF_CHANNELS = 1024
+
+
+def _oracle_block(cfg: I.ScanConfig, b: int):
+    """fp64 inputs of the sample block of batch row b."""
     A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip, cfg.dt_min, cfg.dt_max)
-    A, D, bias = A.astype(np.float64), D.astype(np.float64), bias.astype(np.float64)
-    threads = min(oracle.default_threads(), cfg.dim)
-    blocks = [(b, t0, t1) for b in range(cfg.batch) for t0, t1 in I.iter_time_blocks(cfg.seqlen, 2048)]
-    done, spent = 0, 0.0
-    state = {}
-    for b, t0, t1 in blocks:
-        if spent >= budget_s and done:
-            break
-        x = {k: I.to_f64(I.draw_rows(cfg, k, b, t0, t1), cfg.io)[None] for k in I.SEQ_NAMES}
-        t_start = time.perf_counter()
-        _, state[b] = oracle.scan(x["u"], x["delta"], A, x["B"], x["C"], D=D, z=x["z"], delta_bias=bias,
-                                  delta_softplus=True, h0=state.get(b))
-        spent += time.perf_counter() - t_start
-        done += (t1 - t0) * cfg.dim
+    ch = slice(0, min(REF_CHANNELS, cfg.dim))
+    x = {}
+    for k in I.SEQ_NAMES:
+        rows = I.to_f64(I.draw_rows(cfg, k, b, 0, cfg.seqlen), cfg.io)
+        x[k] = np.ascontiguousarray((rows if k in ("B", "C") else rows[:, ch])[None])
+    x.update(A=A[ch].astype(np.float64), D=D[ch].astype(np.float64), bias=bias[ch].astype(np.float64))
+    return x
+
+
+def _time_oracle_block(x) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.scan(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"], delta_bias=x["bias"],
+                delta_softplus=True)
+    return time.perf_counter() - t0
+
+
+def oracle_rate(cfg: I.ScanConfig, budget_s: float):
+    """The fp64 oracle, as it stands, on sample blocks of the workload (one
+    per batch row in turn) until ``budget_s`` seconds have been spent (at
+    least one block).  Returns (Gelem/s, threads, elements, seconds)."""
+    import oracle
+    threads = min(oracle.default_threads(), REF_CHANNELS, cfg.dim)
+    done, spent, b = 0, 0.0, 0
+    while b == 0 or (spent < budget_s and b < 64):
+        x = _oracle_block(cfg, b % cfg.batch)
+        spent += _time_oracle_block(x)
+        done += x["u"].shape[1] * x["u"].shape[2]
+        b += 1
     return done / spent / 1e9, threads, done, spent
 
 
 def run_reference(args, rank: int) -> int:
     if rank != 0:
         return 0
-    per_step = []
-    # each step: the oracle on REF_CHANNELS channels of one batch row of the
-    # workload, all 2048 time steps (channels are independent, so this is the
-    # workload's own arithmetic on a bounded sample)
-    REF_CHANNELS = 1024
-    total_el = 0
-    gen_cfg = WORKLOAD
-    A, D, bias = I.channel_params(gen_cfg.seed, gen_cfg.dim, gen_cfg.dstate, gen_cfg.d_skip)
-    A, D, bias = A[:REF_CHANNELS], D[:REF_CHANNELS], bias[:REF_CHANNELS]
     import oracle
-    xs = []
-    for b in range(min(2, gen_cfg.batch)):
-        row = {k: I.to_f64(I.draw_rows(gen_cfg, k, b, 0, gen_cfg.seqlen), gen_cfg.io)[None]
-               for k in I.SEQ_NAMES}
-        for k in ("u", "delta", "z"):
-            row[k] = np.ascontiguousarray(row[k][:, :, :REF_CHANNELS])
-        xs.append(row)
+    cfg = WORKLOAD
+    xs = [_oracle_block(cfg, b) for b in range(min(2, cfg.batch))]
     threads = min(oracle.default_threads(), REF_CHANNELS)
+    per_step = []
     for i in range(args.warmup + args.steps):
-        x = xs[i % len(xs)]
-        t0 = time.perf_counter()
-        oracle.scan(x["u"], x["delta"], A.astype(np.float64), x["B"], x["C"], D=D.astype(np.float64),
-                    z=x["z"], delta_bias=bias.astype(np.float64), delta_softplus=True)
-        dt = time.perf_counter() - t0
+        dt = _time_oracle_block(xs[i % len(xs)])
         if i >= args.warmup:
             per_step.append(dt)
-            total_el += gen_cfg.seqlen * REF_CHANNELS
     secs = sum(per_step)
-    value = total_el / secs / 1e9
+    el = args.steps * cfg.seqlen * min(REF_CHANNELS, cfg.dim)
+    value = el / secs / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD.name, "batch": WORKLOAD.batch, "seqlen": WORKLOAD.seqlen,
-                   "dim": WORKLOAD.dim, "dstate": WORKLOAD.dstate, "io": WORKLOAD.io,
+        "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
+                   "dim": cfg.dim, "dstate": cfg.dstate, "io": cfg.io,
                    "parallelism": "host threads over channels"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"per step: {REF_CHANNELS} channels x {WORKLOAD.seqlen} steps of "
-                                   f"one batch row of the {WORKLOAD.name} workload"},
+                         "sample": f"per step: one batch row x {REF_CHANNELS} channels x {cfg.seqlen} steps "
+                                   f"of the {cfg.name} workload"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -305,20 +328,28 @@ def _upload(a, dev):
     return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
 
-def _scan_device_inputs(cfg: I.ScanConfig, dev):
-    """Device copies of a scan workload's inputs.  Long sequences are drawn and
-    copied block by block so that the host never holds them whole."""
+def _scan_device_inputs(cfg: I.ScanConfig, dev, sh=None):
+    """Device copies of a scan workload's inputs, or of one rank's shard of
+    them (rows [b0, b1) and channels [d0, d1) of the global workload, drawn
+    by their global indices).  Long sequences are drawn and copied block by
+    block so that the host never holds them whole."""
     import torch
+    from selective_state_space_36_b200.shard import Shard
+    sh = sh or Shard(0, cfg.batch, 0, cfg.dim)
     A, D, bias = I.channel_params(cfg.seed, cfg.dim, cfg.dstate, cfg.d_skip, cfg.dt_min, cfg.dt_max)
     dt = torch.bfloat16 if cfg.io == "bf16" else torch.float32
     d = {}
     for k in I.SEQ_NAMES:
-        w = cfg.dstate if k in ("B", "C") else cfg.dim
-        d[k] = torch.empty((cfg.batch, cfg.seqlen, w), dtype=dt, device=dev)
-        for b in range(cfg.batch):
+        bc = k in ("B", "C")
+        w = cfg.dstate if bc else sh.dim
+        d[k] = torch.empty((sh.batch, cfg.seqlen, w), dtype=dt, device=dev)
+        for i, b in enumerate(range(sh.b0, sh.b1)):
             for t0, t1 in I.iter_time_blocks(cfg.seqlen, 1 << 16):
-                d[k][b, t0:t1].copy_(_upload(I.draw_rows(cfg, k, b, t0, t1), dev))
-    d.update(A=_upload(A, dev), D=_upload(D, dev), delta_bias=_upload(bias, dev))
+                rows = I.draw_rows(cfg, k, b, t0, t1)
+                d[k][i, t0:t1].copy_(_upload(rows if bc else rows[:, sh.d0:sh.d1], dev))
+    cs = slice(sh.d0, sh.d1)
+    d.update(A=_upload(np.ascontiguousarray(A[cs]), dev), D=_upload(np.ascontiguousarray(D[cs]), dev),
+             delta_bias=_upload(np.ascontiguousarray(bias[cs]), dev))
     return d
 
 
@@ -373,27 +404,25 @@ def _e2e(step_with_copies, steps, stream, dev, world):
     return ms
 
 
-def _base_line(metric, unit, value, world, args, ms_per_step, higher=True):
+def _base_line(metric, unit, value, world, args, ms_per_step, higher=True, io="bf16"):
+    # dtype: the arithmetic type (fp32 everywhere); io_dtype: the element type
+    # of the tensors read and written (bf16 for the benchmark workloads)
     return {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": higher,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic"}
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "io_dtype": io, "data": "synthetic"}
 
 
 def run_scan(args, rank, world, dev):
     import torch
     from selective_state_space_36_b200 import binding as lib
 
-    cfg = WORKLOADS[args.workload]
-    if rank:
-        cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
-    if args.batch or args.seqlen:
-        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
-        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"{args.workload}_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
-    d = _scan_device_inputs(cfg, dev)
-    state = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
+    gcfg, sh = sharded_workload(args, rank, world)
+    cfg = gcfg.with_(batch=sh.batch, dim=sh.dim)  # this rank's part
+    d = _scan_device_inputs(gcfg, dev, sh)
+    state = torch.zeros(sh.batch, sh.dim, cfg.dstate, device=dev)
     out = torch.empty_like(d["u"])
     stream = torch.cuda.current_stream(dev)
-    plan = lib.scan_plan(cfg.batch, cfg.seqlen, cfg.dim, cfg.dstate, cfg.io)
+    plan = lib.scan_plan(sh.batch, cfg.seqlen, sh.dim, cfg.dstate, cfg.io)
 
     # Each step scans one batch of the workload and resumes from the state the
     # previous step left in last_state (a continued sequence): the same work.
@@ -406,8 +435,8 @@ def run_scan(args, rank, world, dev):
     metric = SCAN_METRICS.get(args.workload, METRIC)
     if args.no_e2e:
         if rank == 0:
-            print(json.dumps({"metric": metric, "value": whole_job_rate(world, cfg.elements, ms_per_step),
-                              "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": cfg.name},
+            print(json.dumps({"metric": metric, "value": gcfg.elements / (ms_per_step * 1e-3) / 1e9,
+                              "unit": UNIT, "kernel_ms": kernel_ms, "config": {"workload": gcfg.name},
                               "note": "profiling run: no e2e, no cpu baseline"}), flush=True)
         return 0
 
@@ -434,36 +463,40 @@ def run_scan(args, rank, world, dev):
             host_state.copy_(state, non_blocking=True)
 
         e2e_ms = _e2e(e2e_step, e2e_steps, stream, dev, world)
-        e2e = {"value": whole_job_rate(world, cfg.elements, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        e2e = {"value": gcfg.elements / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "steps": e2e_steps}
 
     if rank == 0:
         peaks = measured_peaks()
-        abytes = algorithmic_bytes(cfg)
+        abytes = algorithmic_bytes(cfg)  # one launch on this rank
         achieved_gbs = abytes / (kernel_ms * 1e-3) / 1e9
         sm_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        alu_peak = alu_ceiling_per_sm_clock(cfg.dstate) * sms * sm_mhz * 1e6 / 1e9
+        info = lib.build_info()
+        per_clk = alu_ceiling_per_sm_clock(cfg.dstate, info["sfu_decays_per_16"])
+        alu_peak = per_clk * sms * sm_mhz * 1e6 / 1e9
         kernel_gelem = cfg.elements / (kernel_ms * 1e-3) / 1e9
         sha = kernel_source_sha()
-        line = _base_line(metric, UNIT, whole_job_rate(world, cfg.elements, ms_per_step), world, args,
-                          ms_per_step)
+        line = _base_line(metric, UNIT, gcfg.elements / (ms_per_step * 1e-3) / 1e9, world, args, ms_per_step,
+                          io=cfg.io)
         line.update({
-            "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "dim": cfg.dim,
-                       "dstate": cfg.dstate, "io": cfg.io, "per_gpu": "one full workload per GPU",
-                       "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"inputs {abytes / 1e6:.0f} MB > {L2_BYTES >> 20} MB L2; no flush",
+            "config": {"workload": gcfg.name, "global_batch": gcfg.batch, "batch": gcfg.batch,
+                       "seqlen": cfg.seqlen, "dim": gcfg.dim, "dstate": cfg.dstate, "io": cfg.io,
+                       "per_gpu": f"rows {sh.b0}..{sh.b1 - 1}, channels {sh.d0}..{sh.d1 - 1} on rank 0",
+                       "parallelism": f"dp{world} (batch rows, no exchange)" if world > 1 else "single",
+                       "l2": f"inputs {abytes / 1e6:.0f} MB per GPU > {L2_BYTES >> 20} MB L2; no flush",
                        "plan": plan},
             "roofline": {
-                "bound": "alu", "achieved": kernel_gelem, "peak": alu_peak, "unit": "Gelem/s",
-                "frac": kernel_gelem / alu_peak,
-                "peak_source": (f"derived: {alu_ceiling_per_sm_clock(cfg.dstate):.3f} elem/clk/SM x {sms} SMs x "
-                                f"{sm_mhz:.0f} MHz (measured SFU/FMA issue costs)"),
+                "bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"],
+                "peak_source": peaks["source"] + " (copy bandwidth)",
                 "traffic": committed_traffic(sha) if args.workload == "mamba1p4b" and plan["launches"] == 1 else None,
                 "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": abytes,
-                "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": achieved_gbs / peaks["hbm_gbs"],
-                        "peak_source": peaks["source"] + " (copy bandwidth)"},
+                "alu": {"achieved": kernel_gelem, "peak": alu_peak, "unit": "Gelem/s",
+                        "frac": kernel_gelem / alu_peak,
+                        "peak_source": (f"derived for the shipped arithmetic ({info['sfu_decays_per_16']} of 16 "
+                                        f"decays on the SFU): {per_clk:.3f} elem/clk/SM x {sms} SMs x "
+                                        f"{sm_mhz:.0f} MHz (measured SFU/FMA issue costs)")},
                 "kernel_source_sha": sha},
             "e2e": e2e,
             "gpu_launches": args.steps * plan["launches"],
@@ -472,8 +505,8 @@ def run_scan(args, rank, world, dev):
         if world == 1 and not args.no_cpu_baseline:
             v, threads, el, secs = oracle_rate(cfg, budget_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"{el} elements of {cfg.name} in blocks of whole channels "
-                                              f"x 2048 steps ({secs:.1f} s)"}
+                                    "sample": f"{el} elements of {cfg.name} in blocks of one batch row x "
+                                              f"{REF_CHANNELS} channels x 2048 steps ({secs:.1f} s)"}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -563,17 +596,13 @@ def run_bwd(args, rank, world, dev):
     import torch
     from selective_state_space_36_b200 import binding as lib
 
-    cfg = WORKLOADS[args.workload]
-    if rank:
-        cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
-    if args.batch or args.seqlen:
-        b_, l_ = args.batch or cfg.batch, args.seqlen or cfg.seqlen
-        cfg = cfg.with_(batch=b_, seqlen=l_, name=f"{args.workload}_b{b_}_l{l_}_d{cfg.dim}_n{cfg.dstate}")
-    d = _scan_device_inputs(cfg, dev)
+    gcfg, sh = sharded_workload(args, rank, world)
+    d = _scan_device_inputs(gcfg, dev, sh)
+    cfg = gcfg.with_(batch=sh.batch, dim=sh.dim)  # this rank's part
     dout = torch.empty_like(d["u"])
-    for b in range(cfg.batch):
+    for i, b in enumerate(range(sh.b0, sh.b1)):
         for t0, t1 in I.iter_time_blocks(cfg.seqlen, 1 << 16):
-            dout[b, t0:t1].copy_(_upload(I.draw_rows(cfg, "dout", b, t0, t1), dev))
+            dout[i, t0:t1].copy_(_upload(I.draw_rows(gcfg, "dout", b, t0, t1)[:, sh.d0:sh.d1], dev))
     h0 = torch.zeros(cfg.batch, cfg.dim, cfg.dstate, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -583,7 +612,7 @@ def run_bwd(args, rank, world, dev):
 
     elapsed_ms, call_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
     ms_per_step = elapsed_ms / args.steps
-    value = whole_job_rate(world, cfg.elements, ms_per_step)
+    value = gcfg.elements / (ms_per_step * 1e-3) / 1e9
     if args.no_e2e:
         if rank == 0:
             print(json.dumps({"metric": BWD_METRIC, "value": value, "unit": UNIT, "kernel_ms": call_ms,
@@ -664,6 +693,87 @@ def run_complex(args, rank, world, dev):
     return 0
 
 
+SSD_METRIC = "SSD (Mamba-2) fwd Gelem/s (B·L·heads·headdim) at batch 8, L 2048, 64 heads x 64, dstate 128"
+SSD_CHUNK = 128
+
+
+def ssd_algorithmic_bytes(cfg: I.SsdConfig) -> int:
+    """x, z, dt, B, C read and out written once (bf16)."""
+    per_tok = 2 * (3 * cfg.heads * cfg.headdim + cfg.heads + 2 * cfg.groups * cfg.dstate)
+    return cfg.batch * cfg.seqlen * per_tok
+
+
+def ssd_flops(cfg: I.SsdConfig, q: int = SSD_CHUNK) -> int:
+    """Dense products of the chunked decomposition at chunk length q, per
+    (batch row, head, chunk): C B^T (2 q^2 N), M X (2 q^2 P), C H^T (2 q N P)
+    and the chunk state B^T (w o X) (2 q N P)."""
+    chunks = (cfg.seqlen + q - 1) // q
+    n, p = cfg.dstate, cfg.headdim
+    return cfg.batch * cfg.heads * chunks * (2 * q * q * n + 2 * q * q * p + 4 * q * n * p)
+
+
+def run_ssd(args, rank, world, dev):
+    """One step = one ssm_ssd_scan_fwd over the Mamba-2 workload (batch rows
+    split over the ranks as for the scan workloads)."""
+    import torch
+    from selective_state_space_36_b200 import binding as lib
+    from selective_state_space_36_b200.shard import scan_shard
+    g = I.MAMBA2_1P3B
+    if args.batch or args.seqlen:
+        g = g.with_(batch=args.batch or g.batch, seqlen=args.seqlen or g.seqlen)
+    if world > 1:
+        g = g.with_(batch=g.batch * world, name=g.name.replace(f"_b{g.batch}_", f"_b{g.batch * world}_", 1))
+    sh = scan_shard(g.batch, g.heads, world, rank)
+    cfg = g.with_(batch=sh.batch)
+    d = {}
+    for k in ("x", "dt", "B", "C", "z"):
+        rows = np.stack([I.ssd_rows(g, k, b) for b in range(sh.b0, sh.b1)])
+        d[k] = _upload(rows, dev)
+    A, D, bias = I.ssd_params(g)
+    d.update(A=_upload(A, dev), D=_upload(D, dev), dt_bias=_upload(bias, dev))
+    state = torch.zeros(cfg.batch, cfg.heads, cfg.headdim, cfg.dstate, device=dev)
+    out = torch.empty_like(d["x"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lib.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"], dt_bias=d["dt_bias"],
+                         out=out, last_state=state, stream=stream)
+
+    elapsed_ms, kernel_ms, clocks = _time_steps(step, args.steps, args.warmup, stream, dev, world)
+    ms_per_step = elapsed_ms / args.steps
+    value = g.elements / (ms_per_step * 1e-3) / 1e9
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"metric": SSD_METRIC, "value": value, "unit": UNIT, "kernel_ms": kernel_ms,
+                              "config": {"workload": g.name}, "note": "profiling run"}), flush=True)
+        return 0
+    if rank == 0:
+        peaks = measured_peaks()
+        abytes = ssd_algorithmic_bytes(cfg)
+        flops = ssd_flops(cfg)
+        gbs = abytes / (kernel_ms * 1e-3) / 1e9
+        tfs = flops / (kernel_ms * 1e-3) / 1e12
+        tpeak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        line = _base_line(SSD_METRIC, UNIT, value, world, args, ms_per_step, io="bf16")
+        line.update({
+            "config": {"workload": g.name, "global_batch": g.batch, "seqlen": g.seqlen, "heads": g.heads,
+                       "headdim": g.headdim, "groups": g.groups, "dstate": g.dstate, "chunk": SSD_CHUNK,
+                       "parallelism": f"dp{world} (batch rows, no exchange)" if world > 1 else "single",
+                       "l2": f"inputs {abytes / 1e6:.0f} MB per GPU > {L2_BYTES >> 20} MB L2; no flush"},
+            "roofline": {
+                "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"] + " (copy bandwidth)",
+                "traffic": None, "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": abytes,
+                "tensor": {"achieved": tfs, "peak": tpeak, "unit": "TFLOP/s", "frac": tfs / tpeak,
+                           "flops_per_launch": flops,
+                           "peak_source": peaks["source"] + (" bf16 dense, sustained"
+                                                             if peaks.get("bf16_tflops_sustained") else " bf16 dense")}},
+            "e2e": None, "gpu_launches": args.steps, "clocks": clocks,
+        })
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> int:
     import torch
     import torch.distributed as dist
@@ -678,6 +788,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> int:
             return run_bwd(args, rank, world, dev)
         if args.workload == "mamba130m_complex":
             return run_complex(args, rank, world, dev)
+        if args.workload == "mamba2_ssd":
+            return run_ssd(args, rank, world, dev)
         return run_scan(args, rank, world, dev)
     finally:
         if world > 1:
@@ -697,9 +809,21 @@ def main() -> int:
     ap.add_argument("--no-e2e", action="store_true", help="device-timed loop only (profiling cases)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mamba1p4b")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: re-run this command under torchrun
+        import socket
+        import subprocess
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+        return subprocess.call(cmd)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "ours" and world != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE {world}; using {world}", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args, rank)
     return run_ours(args, rank, world, local_rank)

@@ -24,7 +24,8 @@
  * Entry points: the scan (ssm_selective_scan_fwd, _ex with execution choices
  * and the exact ZOH form, _noalloc without device allocation), its gradient
  * (ssm_selective_scan_bwd, _ex), the scan with a complex diagonal A
- * (ssm_selective_scan_fwd_complex), the one-token decode step
+ * (ssm_selective_scan_fwd_complex), Mamba-2's SSD layer (ssm_ssd_scan_fwd),
+ * the one-token decode step
  * (ssm_selective_state_update), planning (ssm_scan_plan), the device status
  * word of the bounded waits (ssm_get_device_status) and error reporting.
  *
@@ -174,20 +175,22 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io,
  * from a fixed static array inside the library instead of allocating.
  *
  * Same arguments and results as ssm_selective_scan_fwd, with the sequence
- * split always requested: segments = the number of segments (0 = automatic,
- * capped so the carries fit).  When the sequence is too short to split, one
- * pass runs and no scratch is used.
+ * split always requested: segments = the number of segments, or 0 for the
+ * automatic count, lowered to the largest count whose carries fit the scratch;
+ * when not even two segments fit, one pass runs (it needs no scratch).  When
+ * the sequence is too short to split, one pass runs and no scratch is used.
  *
  * Limits and behaviour:
  *  - The scratch holds SSM_NOALLOC_SCRATCH_BYTES (16 MiB).  A split needs
- *    4 * batch * dim * (dstate * (segments + 1) + segments) bytes; a request
- *    that does not fit returns SSM_ERR_UNSUPPORTED before anything is
- *    enqueued.  Every GPU on which the library is loaded holds these 16 MiB
- *    until the process exits.
+ *    4 * batch * dim * (dstate * (segments + 1) + segments) bytes; an explicit
+ *    segment count that does not fit returns SSM_ERR_UNSUPPORTED before
+ *    anything is enqueued.  Every GPU on which the library is loaded holds
+ *    these 16 MiB until the process exits.
  *  - No cudaMalloc, cudaMallocAsync, cudaFree or allocating library routine is
- *    called.  The first call on each device looks up the scratch's device
- *    address (cudaGetSymbolAddress) with that device current; make that first
- *    call before any stream capture.
+ *    called.  The first call on each device (and the first after a
+ *    cudaDeviceReset, which replaces the device's context) looks up the
+ *    scratch's device address (cudaGetSymbolAddress) with that device
+ *    current; make that first call before any stream capture.
  *  - All calls share the one scratch array, which keeps the last call's
  *    contents.  Nothing in it needs to start at zero (each call writes every
  *    word it later reads), but calls whose GPU work overlaps in time -- on
@@ -319,10 +322,50 @@ ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
                                       const void *z, void *out, ssm_stream stream);
 
 /*
+ * Mamba-2's SSD layer ("Transformers are SSMs: Generalized Models and
+ * Efficient Algorithms Through Structured State Space Duality", review on
+ * nubint.ai, 提案手法): the selective SSM with one scalar A per head, whose
+ * sequence map is a semiseparable matrix, computed by its block
+ * decomposition -- the quadratic (attention-like) form inside chunks of 128
+ * tokens and the linear (recurrent) form between chunks -- on the tensor
+ * cores.  For every batch row b, head h (of P = headdim channels) and time t:
+ *
+ *   Delta_t = softplus(dt[b,t,h] + dt_bias[h])      (or the plain sum)
+ *   H_t     = exp(Delta_t A[h]) H_{t-1} + Delta_t x[b,t,h,:] B[b,t,g,:]^T
+ *   y       = H_t C[b,t,g,:] + D[h] x[b,t,h,:],     out = y * silu(z[b,t,h,:])
+ *
+ * with H (headdim x dstate) per (b, h) and g = h / (heads / groups) the
+ * group whose B, C the head reads.  Layouts (dense, row-major):
+ *   x, z, out  : (batch, seqlen, heads, headdim) bf16; z may be NULL (no gate)
+ *   dt         : (batch, seqlen, heads) bf16, the raw step
+ *   A, D, dt_bias : (heads) float32; D and dt_bias may be NULL (zero)
+ *   B, C       : (batch, seqlen, groups, dstate) bf16
+ *   last_state : (batch, heads, headdim, dstate) float32 or NULL; read as H_0
+ *                and overwritten with H_L (NULL: H_0 = 0, not returned).
+ * Supported: io = SSM_BF16, headdim = 64, dstate = 64 or 128, heads a
+ * multiple of groups, x, z, B, C, out 16-byte aligned (SSM_ERR_UNSUPPORTED
+ * otherwise).  Arithmetic: products on the tensor cores with bf16 operands
+ * and fp32 accumulation; the intra-chunk matrix and the state copy read by
+ * the inter-chunk product are rounded to bf16, the state itself is carried in
+ * fp32 and updated from a two-term (high + low bf16) product.  A wait inside
+ * the kernel that runs out (2 s) sets bit 1 of the device status word
+ * (ssm_get_device_status); the outputs are then not valid.
+ */
+typedef struct {
+    int64_t batch, seqlen, heads, headdim, groups, dstate;
+} ssm_ssd_dims;
+
+ssm_status ssm_ssd_scan_fwd(ssm_ssd_dims dims, ssm_dtype io, const void *x, const void *dt, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int dt_softplus, void *out, float *last_state,
+                            ssm_stream stream);
+
+/*
  * Reads and clears the device status word of the current device, after
  * synchronising "stream".  Bit 0: a bounded wait inside the decode kernel
  * (its state copies, see ssm_selective_state_update) gave up; the outputs of
- * the launches since the last read are then not valid.  The word is shared by
+ * the launches since the last read are then not valid.  Bit 1: a bounded
+ * wait inside the SSD kernel (ssm_ssd_scan_fwd) gave up.  The word is shared by
  * every launch on the device.  Returns SSM_ERR_CUDA if the copies or the
  * synchronisation fail.
  */
@@ -336,6 +379,26 @@ ssm_status ssm_get_device_status(ssm_stream stream, uint32_t *flags);
  * test the bounded waits without a GPU fault.  Process-wide; 0 disables.
  */
 void ssm_test_inject_decode_wait_timeout(int32_t enable);
+
+/* Build parameters that set the arithmetic of the library's kernels (no
+ * counterpart in the method; lets a benchmark state the ceiling of the code
+ * it runs). */
+typedef struct {
+    int32_t sfu_decays_per_16; /* of every 16 decays exp(Delta A) of the bf16 (fast) scan
+                                  tier, how many the SFU computes; the rest are computed
+                                  on the FMA pipe by a polynomial */
+    int32_t reserved[7];
+} ssm_build_info;
+
+void ssm_get_build_info(ssm_build_info *info);
+
+/*
+ * Test hook (no counterpart in the method): evaluates, for n float32 inputs x,
+ * the FMA-pipe exp2 that computes part of the decays of the bf16 scan tier
+ * (poly[i]) and the SFU's ex2.approx (sfu[i]); device pointers, enqueued on
+ * "stream".  Lets a test bound the polynomial's error on the GPU itself.
+ */
+ssm_status ssm_test_exp2_poly(const float *x, float *poly, float *sfu, int64_t n, ssm_stream stream);
 
 /* Static description of a status code. */
 const char *ssm_status_string(ssm_status status);

@@ -25,7 +25,8 @@ EXPORTED = ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selectiv
             "ssm_selective_scan_fwd_complex",
             "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ex", "ssm_selective_state_update",
             "ssm_scan_plan", "ssm_get_device_status", "ssm_test_inject_decode_wait_timeout",
-            "ssm_status_string", "ssm_last_error", "ssm_version")
+            "ssm_status_string", "ssm_last_error", "ssm_version", "ssm_get_build_info", "ssm_ssd_scan_fwd",
+            "ssm_test_exp2_poly")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -46,6 +47,15 @@ class SSMScanPlanInfo(ctypes.Structure):
                 ("lanes", ctypes.c_int32), ("family", ctypes.c_int32),
                 ("launches", ctypes.c_int32), ("channels_per_lane", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_int64)]
+
+
+class SSMSsdDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("heads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("groups", ctypes.c_int64), ("dstate", ctypes.c_int64)]
+
+
+class SSMBuildInfo(ctypes.Structure):
+    _fields_ = [("sfu_decays_per_16", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 class SSMError(RuntimeError):
@@ -93,6 +103,12 @@ def _load() -> ctypes.CDLL:
     lib.ssm_last_error.restype = ctypes.c_char_p
     lib.ssm_version.argtypes = []
     lib.ssm_version.restype = ctypes.c_int
+    lib.ssm_get_build_info.argtypes = [ctypes.POINTER(SSMBuildInfo)]
+    lib.ssm_get_build_info.restype = None
+    lib.ssm_ssd_scan_fwd.argtypes = [SSMSsdDims, ctypes.c_int] + [_vp] * 9 + [ctypes.c_int, _vp, _vp, _vp]
+    lib.ssm_ssd_scan_fwd.restype = ctypes.c_int
+    lib.ssm_test_exp2_poly.argtypes = [_vp, _vp, _vp, ctypes.c_int64, _vp]
+    lib.ssm_test_exp2_poly.restype = ctypes.c_int
     return lib
 
 
@@ -285,6 +301,49 @@ def selective_scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=Non
         _ptr(last_state, "last_state", torch.float32, (batch, dim, dstate), dev),
         int(segments), _stream_handle(stream)))
     return out
+
+
+def ssd_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, out=None, last_state=None,
+                 stream=None):
+    """Mamba-2 SSD layer on CUDA bf16 tensors; returns ``out``.
+
+    x, z: (batch, seqlen, heads, headdim); dt: (batch, seqlen, heads);
+    B, C: (batch, seqlen, groups, dstate); A, D, dt_bias: (heads,) float32;
+    last_state (batch, heads, headdim, dstate) float32 is read as H_0 and
+    overwritten with H_L."""
+    batch, seqlen, heads, headdim = x.shape
+    groups, dstate = B.shape[2], B.shape[3]
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    seq, bc = (batch, seqlen, heads, headdim), (batch, seqlen, groups, dstate)
+    check(lib.ssm_ssd_scan_fwd(
+        SSMSsdDims(batch, seqlen, heads, headdim, groups, dstate), _io_of(x),
+        _ptr(x, "x", x.dtype, seq, dev), _ptr(dt, "dt", x.dtype, (batch, seqlen, heads), dev),
+        _ptr(A, "A", torch.float32, (heads,), dev), _ptr(B, "B", x.dtype, bc, dev), _ptr(C, "C", x.dtype, bc, dev),
+        _ptr(D, "D", torch.float32, (heads,), dev), _ptr(z, "z", x.dtype, seq, dev),
+        _ptr(dt_bias, "dt_bias", torch.float32, (heads,), dev), int(bool(dt_softplus)),
+        _ptr(out, "out", x.dtype, seq, dev),
+        _ptr(last_state, "last_state", torch.float32, (batch, heads, headdim, dstate), dev),
+        _stream_handle(stream)))
+    return out
+
+
+def test_exp2_poly(x: torch.Tensor, stream=None):
+    """(FMA-pipe exp2, SFU ex2.approx) of the float32 CUDA tensor x."""
+    x = x.contiguous()
+    poly, sfu = torch.empty_like(x), torch.empty_like(x)
+    dev = x.device
+    check(lib.ssm_test_exp2_poly(_ptr(x, "x", torch.float32, None, dev), _ptr(poly, "poly", torch.float32, None, dev),
+                                 _ptr(sfu, "sfu", torch.float32, None, dev), x.numel(), _stream_handle(stream)))
+    return poly, sfu
+
+
+def build_info() -> dict:
+    """Build parameters of the loaded library (ssm_get_build_info)."""
+    info = SSMBuildInfo()
+    lib.ssm_get_build_info(ctypes.byref(info))
+    return {"sfu_decays_per_16": int(info.sfu_decays_per_16)}
 
 
 def scan_plan(batch: int, seqlen: int, dim: int, dstate: int, io: str = "bf16",

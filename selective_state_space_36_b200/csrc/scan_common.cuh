@@ -225,7 +225,8 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
                 for (int c = 0; c < CPL; ++c) {
                     if (!PRECISE) {
                         const float2 x2 = mul2(d2[c], A2[c][p]);
-                        const float2 a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
+                        const float2 a2 = poly_pair(p) ? exp2_poly2(x2)
+                                                       : make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
                         float2 bu = mul2(u2[c], b2);
                         if (ZOH)
                             bu = mul2(bu, zoh_phi2(mul2(x2, make_float2(kLn2, kLn2)), a2, invA2[c][p], id2[c]));

@@ -118,8 +118,26 @@ __device__ __forceinline__ void store_vals(IO *p, const float (&v)[CPL]) {
     }
 }
 
+// Barrier of one virtual block (below): a warp barrier when the virtual block
+// is one warp, else hardware barrier 1 + vb with the virtual block's threads.
+// Only the one-pass mode packs several virtual blocks per CTA; the others
+// use the CTA barrier.
+template <int TPB, int MODE>
+__device__ __forceinline__ void vblock_sync(int vb) {
+    if (TPB == 32) __syncwarp();
+    else if (MODE != kFull) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(vb + 1), "n"(TPB) : "memory");
+}
+
+// Threads a CTA of the staged kernel may have (several virtual blocks): at
+// most 256, so that ptxas may give every thread 255 registers.
+template <int G>
+struct StagedMaxThreads {
+    static constexpr int value = 256;
+};
+
 template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH, int TPB>
-__global__ void __launch_bounds__(TPB)
+__global__ void __launch_bounds__(StagedMaxThreads<G>::value)
 scan_fwd_staged_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
     using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
@@ -131,18 +149,27 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     constexpr int KSTEP = MODE == kCkpt ? kCkptEvery : KStep<G, CPL>::value;
     constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
     static_assert(T % KSTEP == 0, "a chunk holds whole step blocks");
-    extern __shared__ __align__(16) unsigned char smem[];
+    // A CTA holds blockDim.x / TPB virtual blocks.  Virtual block vb of CTA
+    // k works on unit k + vb * gridDim.x -- one (batch row, channel tile) for
+    // the whole sequence (segment) -- with its own shared memory and its own
+    // barrier, independently of the CTA's other virtual blocks; several of
+    // them per CTA let the launch place the units evenly over the SMs.
+    extern __shared__ __align__(16) unsigned char smem_all[];
+    const int vb = threadIdx.x / TPB;
+    const int64_t unit = blockIdx.x + (int64_t)vb * gridDim.x;
+    if (unit >= args.units) return;  // no barrier is shared with other virtual blocks
+    unsigned char *smem = smem_all + vb * Lay::SMEM;
     float *fB = reinterpret_cast<float *>(smem + S * Lay::STAGE_BYTES);
     float *fC = fB + T * NSP;
 
     const int64_t L = args.seqlen, Dm = args.dim;
     const int N = args.dstate;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x % TPB;
     const int q = tid % G;
     const int grp = tid / G;
     const int64_t tiles = (Dm + CPB - 1) / CPB;
-    const int64_t b = blockIdx.x / tiles;
-    const int64_t d0 = (blockIdx.x % tiles) * CPB;
+    const int64_t b = unit / tiles;
+    const int64_t d0 = (unit % tiles) * CPB;
     const int64_t dfirst = d0 + (int64_t)grp * CPL;  // first channel of this group
     const bool active = dfirst < Dm;                  // dim is a multiple of CPL here
     // checkpoint c of this lane (kCkpt): ckpt[b][c][dfirst][q NS ...]
@@ -220,7 +247,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         if (c + S - 1 < nchunks) issue(c + S - 1);
         cp_async_commit();
         cp_async_wait<S - 1>();  // this thread's copies of chunk c have landed
-        __syncthreads();         // ... and everyone else's
+        vblock_sync<TPB, MODE>(vb);    // ... and everyone else's
         const int64_t tc = t_begin + (int64_t)c * T;
         const int rows = (int)(t_end - tc < T ? t_end - tc : T);
         const IO *st = stage_ptr(c % S);
@@ -244,7 +271,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 if (MODE != kCkpt) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
             }
         }
-        __syncthreads();
+        vblock_sync<TPB, MODE>(vb);
         if (active) {
             const int col = grp * CPL;
             // this lane's rows of the tiles start at step q, its B/C slice at state q NS
@@ -349,7 +376,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 for (int r0 = 0; r0 < rows; r0 += KSTEP) step_block(r0, rows);
             }
         }
-        __syncthreads();  // stage c % S and the fp32 B/C buffers are free again
+        vblock_sync<TPB, MODE>(vb);  // stage c % S and the fp32 B/C buffers are free again
     }
     cp_async_wait<0>();
 #pragma unroll
@@ -365,41 +392,104 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     }
 }
 
-template <typename IO, int NS, int G, int CPL, int MODE, bool ZOH, int TPB = kBlock>
-inline cudaError_t launch_mode(const ScanArgs &a, dim3 grid, cudaStream_t st) {
-    constexpr bool P = std::is_same<IO, float>::value;
-    using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
-    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE, ZOH, TPB>;
-    // the shared-memory opt-in is a per-device function attribute: set it once per device
-    static std::atomic<unsigned long long> configured{0};
+// Threads of a virtual block of the one-pass scan, by lanes per channel.  One
+// warp per virtual block (32 channels at one lane per channel) gives the
+// finest unit of work, so the units spread over the SMs with the least
+// imbalance; each virtual block widens its own copy of the B/C rows.
+#ifndef SSM_VB_THREADS_G1
+#define SSM_VB_THREADS_G1 32
+#endif
+#ifndef SSM_VB_THREADS_G2
+#define SSM_VB_THREADS_G2 128
+#endif
+#ifndef SSM_VB_THREADS_G4
+#define SSM_VB_THREADS_G4 128
+#endif
+template <int G>
+struct SlabTPB {
+    static constexpr int value = G == 1 ? SSM_VB_THREADS_G1 : (G == 2 ? SSM_VB_THREADS_G2 : SSM_VB_THREADS_G4);
+};
+
+// SM count and opt-in shared memory of the current device (cached per device).
+inline cudaError_t staged_device_limits(int *sms, int *smem_optin) {
+    static std::atomic<int> cache_sms[64], cache_smem[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const int slot = dev & 63;
+    int s = cache_sms[slot].load(std::memory_order_relaxed), m = cache_smem[slot].load(std::memory_order_relaxed);
+    if (s <= 0 || m <= 0) {
+        e = cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&m, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        cache_sms[slot].store(s, std::memory_order_relaxed);
+        cache_smem[slot].store(m, std::memory_order_relaxed);
+    }
+    *sms = s;
+    *smem_optin = m;
+    return cudaSuccess;
+}
+
+// Launches the staged kernel over `units` (batch row, channel tile) units and
+// `nseg` sequence segments (grid y).  The one-pass mode (kFull) packs
+// ceil(units / SMs) virtual blocks into each CTA (as far as threads, shared
+// memory and hardware barriers allow), so that every SM receives the same
+// number of units up to one; the other modes run one virtual block per CTA.
+template <typename IO, int NS, int G, int CPL, int MODE, bool ZOH, int TPB>
+inline cudaError_t launch_mode(ScanArgs a, int64_t units, unsigned nseg, cudaStream_t st) {
+    constexpr bool P = std::is_same<IO, float>::value;
+    using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
+    auto kern = scan_fwd_staged_kernel<IO, NS, G, CPL, P, MODE, ZOH, TPB>;
+    int sms = 0, optin = 0;
+    cudaError_t e = staged_device_limits(&sms, &optin);
+    if (e != cudaSuccess) return e;
+    int vmax = StagedMaxThreads<G>::value / TPB;
+#ifdef SSM_VPB_MAX
+    if (vmax > SSM_VPB_MAX) vmax = SSM_VPB_MAX;
+#endif
+    if (TPB > 32 && vmax > 15) vmax = 15;  // hardware barriers 1..15
+    if ((size_t)vmax * Lay::SMEM > (size_t)optin) vmax = (int)((size_t)optin / Lay::SMEM);
+    if (MODE != kFull) vmax = 1;
+    if (vmax < 1) return cudaErrorInvalidConfiguration;
+    // the shared-memory opt-in is a per-device function attribute: set it once per device
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_relaxed) & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(vmax * Lay::SMEM));
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return e;
         }
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    kern<<<grid, TPB, Lay::SMEM, st>>>(a);
+    int64_t vpb = (units + sms - 1) / sms;
+    if (vpb > vmax) vpb = vmax;
+    if (vpb < 1) vpb = 1;
+    const int64_t gx = (units + vpb - 1) / vpb;
+    if (gx > 2147483647LL) return cudaErrorInvalidConfiguration;
+    a.units = units;
+    kern<<<dim3((unsigned)gx, nseg), (unsigned)(vpb * TPB), vpb * Lay::SMEM, st>>>(a);
     return cudaGetLastError();
 }
 
 template <typename IO, int NS, int G, int CPL, bool ZOH>
 inline cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
+    constexpr int TPBS = SlabTPB<G>::value;
+    constexpr int CPBS = StagedLayout<IO, NS, G, CPL, TPBS>::CPB;
     constexpr int CPB = StagedLayout<IO, NS, G, CPL>::CPB;
-    const unsigned bx = (unsigned)(a.batch * ((a.dim + CPB - 1) / CPB));
-    if (variant == kVariantSlab) return launch_mode<IO, NS, G, CPL, kFull, ZOH>(a, dim3(bx, 1), st);
+    const int64_t units = a.batch * ((a.dim + CPB - 1) / CPB);
+    if (variant == kVariantSlab)
+        return launch_mode<IO, NS, G, CPL, kFull, ZOH, TPBS>(a, a.batch * ((a.dim + CPBS - 1) / CPBS), 1, st);
     if (variant == kVariantCkpt) {
         if (CPL != 1 || ZOH) return cudaErrorInvalidConfiguration;
-        return launch_mode<IO, NS, G, 1, kCkpt, false>(a, dim3(bx, 1), st);
+        return launch_mode<IO, NS, G, 1, kCkpt, false, kBlock>(a, units, 1, st);
     }
-    cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg, ZOH>(a, dim3(bx, (unsigned)(a.nseg - 1)), st);
+    cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg, ZOH, kBlock>(a, units, (unsigned)(a.nseg - 1), st);
     if (e != cudaSuccess) return e;
-    return launch_mode<IO, NS, G, CPL, kSegFinal, ZOH>(a, dim3(bx, (unsigned)a.nseg), st);
+    return launch_mode<IO, NS, G, CPL, kSegFinal, ZOH, kBlock>(a, units, (unsigned)a.nseg, st);
 }
 
 // Exact ZOH on B is built for one channel per lane only.

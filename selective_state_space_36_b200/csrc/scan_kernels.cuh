@@ -40,6 +40,8 @@ struct ScanArgs {
     // kCkpt: states (batch, ceil(seqlen / kCkptEvery), dim, dstate); h_0 is
     // read from last_state, which is not written
     float *ckpt;
+    // staged kernel: (batch row, channel tile) work units; set by its launcher
+    int64_t units;
 };
 
 struct DecodeArgs {
@@ -78,8 +80,10 @@ cudaError_t launch_state_update(const DecodeArgs &a, bool bf16, int ns, int g, c
 // expect bytes that never arrive (a test of the bounded waits)
 bool state_update_bulk_eligible(const DecodeArgs &a, bool bf16);
 cudaError_t launch_state_update_bulk(const DecodeArgs &a, bool bf16, uint32_t missing_bytes, cudaStream_t st);
-// the device status word the kernels' bounded waits report into
+// the device status word the kernels' bounded waits report into (bit 0: a
+// decode wait ran out; bit 1: an SSD scan wait ran out)
 unsigned int read_and_clear_device_status(cudaStream_t st, cudaError_t *err);
+cudaError_t device_status_address(unsigned int **p);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
 // complex diagonal A: A, B, C and last_state hold (re, im) pairs
 cudaError_t launch_scan_complex(const ScanArgs &a, bool bf16, cudaStream_t st);
@@ -90,6 +94,22 @@ bool scan_bwd_staged_eligible(const ScanBwdArgs &a, int es);
 int scan_bwd_staged_chunk();
 cudaError_t launch_scan_bwd_staged(const ScanBwdArgs &a, bool bf16, cudaStream_t st);
 int64_t scan_bwd_chunk(int dstate);              // time steps between checkpoints
+
+// Mamba-2 SSD layer (bf16 x, dt, B, C, z, out; fp32 A, D, dt_bias, state):
+// x, z, out (batch, seqlen, heads, headdim); dt (batch, seqlen, heads);
+// B, C (batch, seqlen, groups, dstate); state (batch, heads, headdim, dstate)
+struct SsdFwdArgs {
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *D, *dt_bias;
+    void *out;
+    float *state;
+    int64_t batch, seqlen, heads, headdim, groups, dstate;
+    int softplus;
+};
+bool ssd_fwd_supported(const SsdFwdArgs &a);
+// the fast tier's FMA-pipe exp2 (and the SFU's ex2) of n values, for tests
+cudaError_t launch_exp2_poly_check(const float *x, float *poly, float *sfu, int64_t n, cudaStream_t st);  // headdim 64, dstate 64 or 128, 16-byte aligned tensors
+cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st);
 int64_t scan_bwd_channels_per_block();
 
 }  // namespace ssm

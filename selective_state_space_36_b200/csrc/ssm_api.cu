@@ -165,7 +165,13 @@ const char *ssm_status_string(ssm_status s) {
 
 const char *ssm_last_error(void) { return g_last_error; }
 
-int ssm_version(void) { return 100; }
+int ssm_version(void) { return 200; }
+
+void ssm_get_build_info(ssm_build_info *info) {
+    if (!info) return;
+    memset(info, 0, sizeof(*info));
+    info->sfu_decays_per_16 = 16 - 4 * SSM_POLY_PAIRS;
+}
 
 }  // extern "C"
 
@@ -377,8 +383,11 @@ ssm_status ssm_selective_scan_fwd_ex(ssm_dims dims, ssm_dtype io, const void *u,
 // from the fixed scratch array below, which the CUDA runtime places in device
 // memory when the library's module is loaded on a GPU and keeps until the
 // process exits.  Host code must not pass the array's name to a kernel (on the
-// host it is only a shadow symbol): the device address is looked up once per
-// device with cudaGetSymbolAddress while that device is current.
+// host it is only a shadow symbol): the device address is looked up with
+// cudaGetSymbolAddress while the device is current, once per device and CUDA
+// context -- a device reset (cudaDeviceReset) destroys the context and the
+// module with it, so an address cached across it would be stale; the cache is
+// keyed by the context's unique id and the lookup is repeated for a new one.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = (size_t)SSM_NOALLOC_SCRATCH_BYTES;
@@ -386,7 +395,39 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void *g_noalloc_addr[kMaxDevices] = {};
+struct ScratchAddr {
+    unsigned long long ctx_id = 0;  // 0: unknown (look up again)
+    void *addr = nullptr;
+};
+ScratchAddr g_noalloc_addr[kMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (0 if there is none
+// or the driver cannot say), through driver entry points fetched by the
+// runtime, so the library needs no link-time dependency on the driver.
+unsigned long long current_context_id() {
+    using GetCurrent = int (*)(void **);
+    using GetId = int (*)(void *, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(f);
+        (void)cudaGetLastError();
+    });
+    if (!get_current || !get_id) return 0;
+    void *ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
 
 ssm_status noalloc_scratch_address(void **addr) {
     int dev = -1;
@@ -394,13 +435,17 @@ ssm_status noalloc_scratch_address(void **addr) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(SSM_ERR_UNSUPPORTED, "device index %d >= %d", dev, kMaxDevices);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+    ScratchAddr &c = g_noalloc_addr[dev];
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || c.ctx_id != ctx || !c.addr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-        g_noalloc_addr[dev] = p;
+        c.addr = p;
+        // the lookup makes the device's primary context current if it was not
+        c.ctx_id = ctx ? ctx : current_context_id();
     }
-    *addr = g_noalloc_addr[dev];
+    *addr = c.addr;
     return SSM_OK;
 }
 
@@ -421,14 +466,26 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
     if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &p)) return s;
     if (p.launches == 0) return SSM_OK;  // empty problem
     if (p.ws_bytes > kNoAllocScratchBytes && segments == 0) {
-        // automatic segment count: take the largest that fits the scratch
-        const size_t per_seg = ((size_t)dims.batch * dims.dim * (dims.dstate + 1)) * sizeof(float);
-        const size_t fixed = (size_t)dims.batch * dims.dim * dims.dstate * sizeof(float);
-        const size_t fit = kNoAllocScratchBytes > fixed ? (kNoAllocScratchBytes - fixed) / per_seg : 0;
-        if (fit >= 2) {
-            o.segments = (int)(fit > 65535 ? 65535 : fit);
-            if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &p)) return s;
+        // Automatic segment count: the largest count whose carries fit the
+        // scratch, found by bisection on the planner's own workspace size
+        // (which grows with the count), so the two never disagree; when even
+        // two segments do not fit, one pass runs, which needs no scratch.
+        int lo = 1, hi = p.nseg;  // carries(lo) fit (one pass: none), carries(hi) do not
+        while (hi - lo > 1) {
+            const int mid = lo + (hi - lo) / 2;
+            o.segments = mid;
+            ScanPlan t;
+            if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &t)) return s;
+            if (t.ws_bytes <= kNoAllocScratchBytes) lo = mid;
+            else hi = mid;
         }
+        if (lo >= 2) {
+            o.segments = lo;
+        } else {
+            o.variant = SSM_VARIANT_SLAB;
+            o.segments = 0;
+        }
+        if (ssm_status s = plan_scan(dims, io, u, delta, B, C, z, out, delta_softplus, &o, &p)) return s;
     }
     if (p.ws_bytes > kNoAllocScratchBytes)
         return fail(SSM_ERR_UNSUPPORTED, "the split needs %zu bytes of scratch but the static scratch holds %zu "
@@ -452,7 +509,7 @@ ssm_status ssm_selective_scan_fwd_noalloc(ssm_dims dims, ssm_dtype io, const voi
     a.seg_len = p.seg_len;
     a.nseg = p.nseg;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (p.variant == SSM_VARIANT_SLAB) {  // too short to split: one pass, no scratch
+    if (p.variant == SSM_VARIANT_SLAB) {  // too short to split, or too wide for the scratch: one pass
         cudaError_t e = ssm::launch_scan_fwd(a, io == SSM_BF16, p.ns, p.g, p.cpl, ssm::kVariantSlab, p.family, st);
         if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
         return SSM_OK;
@@ -712,12 +769,63 @@ ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
     return SSM_OK;
 }
 
+ssm_status ssm_ssd_scan_fwd(ssm_ssd_dims dims, ssm_dtype io, const void *x, const void *dt, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int dt_softplus, void *out, float *last_state,
+                            ssm_stream stream) {
+    g_last_error[0] = 0;
+    size_t es = 0;
+    if (ssm_status s = check_io(io, &es)) return s;
+    if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.headdim < 0 || dims.groups < 0 ||
+        dims.dstate < 0)
+        return fail(SSM_ERR_INVALID_ARG, "negative size");
+    if (dims.groups < 1 || dims.heads % dims.groups != 0)
+        return fail(SSM_ERR_INVALID_ARG, "heads (%lld) must be a multiple of groups (%lld >= 1)",
+                    (long long)dims.heads, (long long)dims.groups);
+    if (dt_softplus != 0 && dt_softplus != 1) return fail(SSM_ERR_INVALID_ARG, "dt_softplus must be 0 or 1");
+    if (io != SSM_BF16) return fail(SSM_ERR_UNSUPPORTED, "the SSD layer runs on bf16 tensors only");
+    if (dims.headdim != 64) return fail(SSM_ERR_UNSUPPORTED, "headdim %lld (64 is built)", (long long)dims.headdim);
+    if (dims.dstate != 64 && dims.dstate != 128)
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %lld (64 or 128 are built)", (long long)dims.dstate);
+    if (dims.batch == 0 || dims.heads == 0 || dims.seqlen == 0) return SSM_OK;  // state unchanged
+    if (dims.seqlen > 0x7fffffffLL || dims.batch > 0x7fffffffLL || dims.heads * dims.headdim > 0x7fffffffLL ||
+        dims.groups * dims.dstate > 0x7fffffffLL)
+        return fail(SSM_ERR_UNSUPPORTED, "a tensor coordinate exceeds 32 bits");
+    if (!x || !dt || !A || !B || !C || !out) return fail(SSM_ERR_INVALID_ARG, "x, dt, A, B, C and out are required");
+    if (misaligned(dt, 2) || misaligned(A, 4) || misaligned(D, 4) || misaligned(dt_bias, 4) ||
+        misaligned(last_state, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+    if (misaligned(x, 16) || misaligned(z, 16) || misaligned(B, 16) || misaligned(C, 16) || misaligned(out, 16))
+        return fail(SSM_ERR_UNSUPPORTED, "x, z, B, C and out must be 16-byte aligned (tensor-memory copies)");
+    ssm::SsdFwdArgs a{};
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.dt_bias = dt_bias; a.out = out; a.state = last_state;
+    a.batch = dims.batch; a.seqlen = dims.seqlen; a.heads = dims.heads; a.headdim = dims.headdim;
+    a.groups = dims.groups; a.dstate = dims.dstate; a.softplus = dt_softplus;
+    if (!ssm::ssd_fwd_supported(a))
+        return fail(SSM_ERR_UNSUPPORTED, "the driver offers no tensor-map encoder (cuTensorMapEncodeTiled)");
+    cudaError_t e = ssm::launch_ssd_fwd(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "SSD kernel launch");
+    return SSM_OK;
+}
+
 ssm_status ssm_get_device_status(ssm_stream stream, uint32_t *flags) {
     g_last_error[0] = 0;
     if (!flags) return fail(SSM_ERR_INVALID_ARG, "flags is required");
     cudaError_t e = cudaSuccess;
     *flags = ssm::read_and_clear_device_status(reinterpret_cast<cudaStream_t>(stream), &e);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    return SSM_OK;
+}
+
+ssm_status ssm_test_exp2_poly(const float *x, float *poly, float *sfu, int64_t n, ssm_stream stream) {
+    g_last_error[0] = 0;
+    if (n < 0) return fail(SSM_ERR_INVALID_ARG, "n must be >= 0");
+    if (n > 0 && (!x || !poly || !sfu)) return fail(SSM_ERR_INVALID_ARG, "x, poly and sfu are required");
+    if (misaligned(x, 4) || misaligned(poly, 4) || misaligned(sfu, 4))
+        return fail(SSM_ERR_INVALID_ARG, "a pointer is not aligned to its element size");
+    cudaError_t e = ssm::launch_exp2_poly_check(x, poly, sfu, n, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "exp2 check launch");
     return SSM_OK;
 }
 

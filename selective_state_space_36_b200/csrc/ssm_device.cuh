@@ -172,6 +172,61 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return d;
 }
 
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n.reg .b64 ra, rb, rd;\nmov.b64 ra, {%2,%3};\nmov.b64 rb, {%4,%5};\n"
+        "sub.rn.f32x2 rd, ra, rb;\nmov.b64 {%0,%1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// ------------------------------------------- 2^x on the FMA pipe (two lanes)
+// The SFU computes 16 ex2 per SM clock, which caps a scan that needs one
+// decay per state and step; part of the decays are therefore computed on the
+// FMA pipe instead.  Method (Cody and Waite's argument reduction followed by
+// a polynomial, as in Muller, "Elementary Functions", ch. 11):
+//   x is clamped to [-125, 127] (below, 2^x is < 2^-125: the SFU result would
+//   be flushed to zero and either is negligible against the input term; above,
+//   fp32 would overflow);
+//   r = round(x) by adding and subtracting 1.5 * 2^23, which rounds to an
+//   integer in fp32; f = x - r, exact, in [-1/2, 1/2];
+//   2^f = 1 + f (c1 + f (c2 + f (c3 + f (c4 + f c5)))), a degree-5 polynomial
+//   fitted here to 2^f on [-1/2, 1/2] (Lawson-weighted least squares on 4000
+//   Chebyshev nodes, relative error; constant term 1 exactly, so x = 0 gives
+//   exactly 1); relative error 1.1e-7, 1.6e-7 with fp32 Horner evaluation,
+//   against ~2^-22.5 for ex2.approx;
+//   2^r is inserted into the exponent field: the low bits of t = x + 1.5 2^23
+//   hold r, so bits(2^f) + (bits(t) << 23) is the result (exponent 126 or 127
+//   of 2^f plus r in [-125, 127] stays a normal number).
+#define SSM_EXP2_C {0.6931470036506653f, 0.24022242426872253f, 0.05550733581185341f, \
+                    0.009671512991189957f, 0.001326472731307149f}
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float c[5] = SSM_EXP2_C;
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    x.x = fminf(fmaxf(x.x, -125.f), 127.f);
+    x.y = fminf(fmaxf(x.y, -125.f), 127.f);
+    const float2 t = add2(x, make_float2(kRound, kRound));
+    const float2 f = sub2(x, sub2(t, make_float2(kRound, kRound)));
+    float2 p = make_float2(c[4], c[4]);
+    p = fma2(p, f, make_float2(c[3], c[3]));
+    p = fma2(p, f, make_float2(c[2], c[2]));
+    p = fma2(p, f, make_float2(c[1], c[1]));
+    p = fma2(p, f, make_float2(c[0], c[0]));
+    p = fma2(p, f, make_float2(1.f, 1.f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Pairs of states whose decays use exp2_poly2 instead of the SFU: pair p of a
+// lane's states does when (p mod 4) < SSM_POLY_PAIRS, i.e. SSM_POLY_PAIRS / 4
+// of the decays (for lanes holding at least 8 states).
+#ifndef SSM_POLY_PAIRS
+#define SSM_POLY_PAIRS 1
+#endif
+__device__ __forceinline__ constexpr bool poly_pair(int p) { return (p & 3) < SSM_POLY_PAIRS; }
+
 template <bool PRECISE>
 __device__ __forceinline__ float scale_A(float a) {
     return PRECISE ? a : a * kLog2e;

@@ -319,6 +319,10 @@ unsigned int read_and_clear_device_status(cudaStream_t st, cudaError_t *err) {
     return v;
 }
 
+cudaError_t device_status_address(unsigned int **p) {
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(p), g_device_status);
+}
+
 bool state_update_bulk_eligible(const DecodeArgs &a, bool bf16) {
     const size_t es = bf16 ? 2 : 4;
     auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) % 16) == 0; };

@@ -369,3 +369,83 @@ def decode_step_inputs(cfg: DecodeConfig, step: int,
 def iter_time_blocks(seqlen: int, block: int) -> Iterable[Tuple[int, int]]:
     for t0 in range(0, seqlen, block):
         yield t0, min(seqlen, t0 + block)
+
+
+# --------------------------------------------------------------------------
+# Mamba-2 SSD layer
+# --------------------------------------------------------------------------
+_SSD_TID = {"ssd_param": 20, "ssd_x": 21, "ssd_dt": 22, "ssd_B": 23, "ssd_C": 24, "ssd_z": 25, "ssd_h0": 26}
+
+
+@dataclass(frozen=True)
+class SsdConfig:
+    """One SSD workload: x, z (batch, seqlen, heads, headdim), dt (batch,
+    seqlen, heads), B, C (batch, seqlen, groups, dstate), all bf16; A, D,
+    dt_bias (heads,) float32; state (batch, heads, headdim, dstate) float32."""
+    name: str
+    batch: int
+    seqlen: int
+    heads: int
+    headdim: int
+    groups: int
+    dstate: int
+    seed: int = 5
+    dt_sigma: float = 0.5
+    dt_min: float = 1e-3
+    dt_max: float = 1e-1
+    h0_sigma: Optional[float] = None
+    has_z: bool = True
+
+    @property
+    def elements(self) -> int:
+        return self.batch * self.seqlen * self.heads * self.headdim
+
+    def with_(self, **kw) -> "SsdConfig":
+        return replace(self, **kw)
+
+
+# Mamba-2 at the 1.4B-layer shape: d_inner 4096 as 64 heads of 64, dstate 128,
+# one group of B, C shared by every head.
+MAMBA2_1P3B = SsdConfig("mamba2_b8_l2048_h64_p64_n128", 8, 2048, 64, 64, 1, 128, seed=5)
+
+
+def ssd_params(cfg: SsdConfig) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """A, D, dt_bias (heads,) float32: A_h = -U(1, 16) (one scalar per head),
+    D ~ U(0.5, 1.5), dt_bias = inverse softplus of dt0 log-uniform in
+    [dt_min, dt_max] (as channel_params).  Draw order: A, dt0, D."""
+    rng = np.random.default_rng([cfg.seed, _SSD_TID["ssd_param"]])
+    A = (-rng.uniform(1.0, 16.0, size=cfg.heads)).astype(np.float32)
+    dt0 = np.exp(rng.uniform(math.log(cfg.dt_min), math.log(cfg.dt_max), size=cfg.heads))
+    bias = (dt0 + np.log(-np.expm1(-dt0))).astype(np.float32)
+    D = rng.uniform(0.5, 1.5, size=cfg.heads).astype(np.float32)
+    return A, D, bias
+
+
+def ssd_rows(cfg: SsdConfig, name: str, b: int) -> np.ndarray:
+    """Batch row b of an SSD sequence tensor ("x", "z", "dt", "B", "C") as bf16
+    bits: x, z (seqlen, heads, headdim); dt (seqlen, heads) ~ N(0, dt_sigma^2)
+    (the raw step); B, C (seqlen, groups, dstate); all others ~ N(0, 1)."""
+    shape = {"x": (cfg.heads, cfg.headdim), "z": (cfg.heads, cfg.headdim), "dt": (cfg.heads,),
+             "B": (cfg.groups, cfg.dstate), "C": (cfg.groups, cfg.dstate)}[name]
+    rng = np.random.default_rng([cfg.seed, _SSD_TID["ssd_" + name], b])
+    v = rng.standard_normal((cfg.seqlen,) + shape, dtype=np.float32)
+    if name == "dt":
+        v *= np.float32(cfg.dt_sigma)
+    return f32_to_bf16_bits(v)
+
+
+def ssd_inputs(cfg: SsdConfig) -> Dict[str, Optional[np.ndarray]]:
+    """All inputs of one SSD call: x, dt, B, C, z (bf16 bits, with a batch
+    axis), A, D, dt_bias (float32), h0 (float32 or None)."""
+    res: Dict[str, Optional[np.ndarray]] = {
+        k: np.stack([ssd_rows(cfg, k, b) for b in range(cfg.batch)]) for k in ("x", "dt", "B", "C", "z")}
+    if not cfg.has_z:
+        res["z"] = None
+    res["A"], res["D"], res["dt_bias"] = ssd_params(cfg)
+    if cfg.h0_sigma is not None:
+        rng = np.random.default_rng([cfg.seed, _SSD_TID["ssd_h0"]])
+        res["h0"] = (rng.standard_normal((cfg.batch, cfg.heads, cfg.headdim, cfg.dstate), dtype=np.float32)
+                     * np.float32(cfg.h0_sigma))
+    else:
+        res["h0"] = None
+    return res

@@ -1,18 +1,26 @@
-"""The multi-process logic of bench.py on CPU: two gloo ranks.
+"""The multi-process path of bench.py on CPU: two and three gloo ranks.
 
-Each rank scans its own independent copy of the workload (different seeds, no
-exchange on the data path), the timings are reduced with a maximum over ranks,
-and the whole-job rate counts every rank's elements over the slowest rank's
-time.  The data path itself is also shown to shard without exchange: two ranks
-running the fp64 oracle on disjoint channel halves reproduce the one-process
-result exactly once gathered.
+bench.py runs one global workload whose batch rows are split over the ranks
+by selective_state_space_36_b200.shard.scan_shard (channels of every row when
+there are fewer rows than ranks); rows are drawn by their global index, and
+there is no exchange on the data path.  Here each rank takes its shard of
+small problems with the same partition code, scans it with the fp64 oracle,
+and the gathered outputs and states must equal one process scanning the whole
+problem bit for bit.  The timing reduction (maximum over ranks) and the
+whole-job rate are checked too.
 """
 import os
 import socket
+from types import SimpleNamespace
 
 import numpy as np
 import pytest
 import torch.multiprocessing as mp
+
+from selective_state_space_36_b200.shard import Shard, scan_shard
+
+SMALL = [dict(name="rows", batch=4, seqlen=40, dim=24, dstate=4),      # batch >= ranks: rows split
+         dict(name="channels", batch=1, seqlen=33, dim=40, dstate=16)]  # batch < ranks: channels split
 
 
 def _free_port():
@@ -21,40 +29,62 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _small_cfg(c):
+    from selective_state_space_36_b200 import inputs as I
+    return I.ScanConfig(c["name"], c["batch"], c["seqlen"], c["dim"], c["dstate"], io="bf16", seed=3, h0_sigma=0.2)
+
+
+def _oracle_on(cfg, sh: Shard):
+    """The oracle on rows [b0, b1), channels [d0, d1) of cfg, drawn by their
+    global indices (as bench.py draws a rank's share)."""
+    import oracle
+    from selective_state_space_36_b200 import inputs as I
+    x = I.scan_inputs(cfg)
+    f = lambda k: I.to_f64(x[k], "bf16")
+    rs, cs = slice(sh.b0, sh.b1), slice(sh.d0, sh.d1)
+    return oracle.scan(f("u")[rs, :, cs], f("delta")[rs, :, cs], x["A"][cs].astype(float), f("B")[rs],
+                       f("C")[rs], D=x["D"][cs].astype(float), z=f("z")[rs, :, cs],
+                       delta_bias=x["delta_bias"][cs].astype(float), h0=x["h0"][rs, cs].astype(float),
+                       nthreads=1)
+
+
 def _worker(rank, world, port, q):
-    import torch
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import bench
-        import oracle
-        from selective_state_space_36_b200 import inputs as I
-        cfg = bench.rank_config(rank)
-        first = I.draw_rows(cfg, "u", 0, 0, 4)
-        got = [None] * world
-        dist.all_gather_object(got, first.tobytes())
+        args = SimpleNamespace(workload="mamba1p4b", batch=0, seqlen=0)
+        gcfg, sh = bench.sharded_workload(args, rank, world)
+        parts = {}
+        for c in SMALL:
+            cfg = _small_cfg(c)
+            s = scan_shard(cfg.batch, cfg.dim, world, rank)
+            o, st = _oracle_on(cfg, s)
+            got = [None] * world
+            dist.all_gather_object(got, (s, o, st))
+            parts[c["name"]] = got
         mx = bench.max_over_ranks([10.0 + rank, 5.0 - rank])
-        rate = bench.whole_job_rate(world, 1000, mx[0])
-        # shard a small problem by channels: rank r takes half of the dims
-        small = I.ScanConfig("shard", 2, 40, 12, 4, io="bf16", seed=3, h0_sigma=0.2)
-        x = I.scan_inputs(small)
-        lo, hi = rank * small.dim // world, (rank + 1) * small.dim // world
-        f = lambda k: I.to_f64(x[k], "bf16")
-        sl = slice(lo, hi)
-        o, st = oracle.scan(f("u")[:, :, sl], f("delta")[:, :, sl], x["A"][sl].astype(float), f("B"), f("C"),
-                            D=x["D"][sl].astype(float), z=f("z")[:, :, sl],
-                            delta_bias=x["delta_bias"][sl].astype(float), h0=x["h0"][:, sl].astype(float),
-                            nthreads=1)
-        parts = [None] * world
-        dist.all_gather_object(parts, (lo, hi, o, st))
-        q.put((rank, got, mx, rate, parts))
+        q.put((rank, gcfg, sh, parts, mx))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks():
-    world, port = 2, _free_port()
+def test_scan_shard_covers_the_workload_once():
+    for batch, dim, world in [(8, 4096, 1), (16, 4096, 2), (8, 4096, 8), (5, 1536, 3), (1, 1536, 8),
+                              (3, 100, 4), (2, 7, 3)]:
+        seen = np.zeros((batch, dim), dtype=int)
+        for r in range(world):
+            s = scan_shard(batch, dim, world, r)
+            seen[s.b0:s.b1, s.d0:s.d1] += 1
+            if batch < world and s.d1 < dim:
+                assert s.d1 % 8 == 0  # channel blocks keep 16-byte aligned bf16 rows
+        assert np.all(seen == 1), (batch, dim, world)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_gather_the_one_process_result(world):
+    port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
@@ -64,20 +94,20 @@ def test_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    import oracle
     from selective_state_space_36_b200 import inputs as I
-    import bench
-    assert bench.rank_config(0) == I.MAMBA1P4B
-    small = I.ScanConfig("shard", 2, 40, 12, 4, io="bf16", seed=3, h0_sigma=0.2)
-    x = I.scan_inputs(small)
-    f = lambda k: I.to_f64(x[k], "bf16")
-    full_o, full_st = oracle.scan(f("u"), f("delta"), x["A"].astype(float), f("B"), f("C"),
-                                  D=x["D"].astype(float), z=f("z"), delta_bias=x["delta_bias"].astype(float),
-                                  h0=x["h0"].astype(float), nthreads=1)
-    for rank, got, mx, rate, parts in res:
-        assert got[0] != got[1], "ranks must draw independent inputs"
-        assert mx == [11.0, 5.0]
-        assert rate == pytest.approx(2 * 1000 / 11e-3 / 1e9)
-        o = np.concatenate([p[2] for p in sorted(parts, key=lambda p: p[0])], axis=2)
-        st = np.concatenate([p[3] for p in sorted(parts, key=lambda p: p[0])], axis=1)
-        assert np.array_equal(o, full_o) and np.array_equal(st, full_st)
+    full = {c["name"]: _oracle_on(_small_cfg(c), Shard(0, c["batch"], 0, c["dim"])) for c in SMALL}
+    rows_seen = set()
+    for rank, gcfg, sh, parts, mx in res:
+        # the benchmark's global workload: the 1.4B-layer shape with world x 8 rows
+        assert gcfg.batch == I.MAMBA1P4B.batch * world and gcfg.dim == I.MAMBA1P4B.dim
+        assert (sh.d0, sh.d1) == (0, gcfg.dim)
+        rows_seen |= set(range(sh.b0, sh.b1))
+        assert mx == [10.0 + world - 1, 5.0]
+        for c in SMALL:
+            fo, fs = full[c["name"]]
+            o, st = np.zeros_like(fo), np.zeros_like(fs)
+            for s, po, pst in parts[c["name"]]:
+                o[s.b0:s.b1, :, s.d0:s.d1] = po
+                st[s.b0:s.b1, s.d0:s.d1] = pst
+            assert np.array_equal(o, fo) and np.array_equal(st, fs), c["name"]
+    assert rows_seen == set(range(I.MAMBA1P4B.batch * world))

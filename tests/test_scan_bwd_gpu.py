@@ -100,6 +100,27 @@ def test_bwd_mamba1p4b_launch_shape_subset():
     print("[bwd 1.4B subset] " + " ".join(f"{k}={v:.1e}" for k, v in errs.items()))
 
 
+@pytest.mark.slow
+def test_bwd_mamba1p4b_full_shape_sampled_channels():
+    # the whole 1.4B-layer workload (batch 8, L 2048, dim 4096) in one call;
+    # the per-channel gradients (du, ddelta, dz, dA, dD, ddelta_bias, dh0) of
+    # sampled channels of every batch row against the oracle on those
+    # channels (channels are independent; dB and dC sum over all channels and
+    # are checked on the 256-channel launch above)
+    cfg = I.MAMBA1P4B.with_(h0_sigma=0.3)
+    x, dout = I.scan_inputs(cfg), I.draw_dout(cfg)
+    got = T.gpu_bwd(x, "bf16", dout)
+    dsel = np.array([0, 1, 127, 128, 2049, 3071, 4094, 4095])
+    sub = T.channel_subset(x, dsel)
+    ref = T.oracle_bwd(sub, "bf16", dout[:, :, dsel])
+    ds = torch.as_tensor(dsel, device="cuda")
+    picked = {"du": got["du"][:, :, ds], "ddelta": got["ddelta"][:, :, ds], "dz": got["dz"][:, :, ds],
+              "dA": got["dA"][ds], "dD": got["dD"][ds], "ddelta_bias": got["ddelta_bias"][ds],
+              "dh0": got["dh0"][:, ds]}
+    errs = T.check_grads(picked, ref, "bf16", list(picked))
+    print("[bwd 1.4B full, sampled channels] " + " ".join(f"{k}={v:.1e}" for k, v in errs.items()))
+
+
 def test_bwd_families_agree_mid_size():
     # the two families on a shape too large for the oracle to take quickly
     cfg, x, dout = _case("bf16", 4, 1000, 512, 16, 9, h0_sigma=0.5)

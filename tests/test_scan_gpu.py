@@ -30,11 +30,14 @@ def _case(io, batch, L, dim, N, seed, **kw):
     return cfg, I.scan_inputs(cfg)
 
 
-def _check(x, io, **kw):
+def _check(x, io, report=None, **kw):
     out, state = T.gpu_scan(x, io, **kw)
     ref_out, ref_state = T.oracle_scan(x, io)
     e1 = T.check_out(T.from_dev(out), ref_out, io)
     e2 = T.check_state(T.from_dev(state), ref_state, io)
+    if report:
+        e3 = T.state_err_elementwise(T.from_dev(state), ref_state)
+        print(f"[{report}] out {e1:.2e} (1+|y|); state norm-wise {e2:.2e}, elementwise with floor {e3:.2e}")
     return e1, e2
 
 
@@ -55,14 +58,14 @@ def test_tiny_fp32_workload_with_h0_and_every_variant():
 @pytest.mark.slow
 def test_mamba130m_workload_full():
     x = I.scan_inputs(I.MAMBA130M)
-    _check(x, "bf16")
+    _check(x, "bf16", report="mamba130m")
 
 
 @pytest.mark.slow
 def test_mamba1p4b_workload_full():
     """The benchmark's workload and launch configuration, every element."""
     x = I.scan_inputs(I.MAMBA1P4B)
-    _check(x, "bf16")
+    _check(x, "bf16", report="mamba1p4b")
 
 
 # ------------------------------------------------------ layouts and variants

@@ -74,3 +74,43 @@ def test_noalloc_rejects_a_split_larger_than_its_scratch(lib):
     assert b"static scratch" in lib.lib.ssm_last_error()
     torch.cuda.synchronize()
     assert torch.all(out == 7.0)  # nothing was launched
+
+
+def _oracle_rows(x, io, dsel):
+    sub = T.channel_subset(x, dsel)
+    return T.oracle_scan(sub, io)
+
+
+@pytest.mark.parametrize("shape,split_segments", [
+    # batch 8 x dim 8192 x 16 states: the automatic split (3 segments) needs
+    # 17.5 MB of carries; 2 segments (13.1 MB) fit the 16 MiB scratch
+    ((8, 512, 8192), 2),
+    # batch 32 x dim 4096: even 2 segments need 26 MB, so one pass runs
+    ((32, 256, 4096), 1),
+])
+def test_noalloc_automatic_segments_fit_the_scratch(lib, shape, split_segments):
+    batch, seqlen, dim = shape
+    scratch = 16 * 1024 * 1024
+    auto = lib.scan_plan(batch, seqlen, dim, 16, "bf16", variant="split")
+    assert auto["workspace_bytes"] > scratch  # the default split would not fit
+    if split_segments >= 2:
+        fits = lib.scan_plan(batch, seqlen, dim, 16, "bf16", variant="split", segments=split_segments)
+        over = lib.scan_plan(batch, seqlen, dim, 16, "bf16", variant="split", segments=split_segments + 1)
+        assert fits["workspace_bytes"] <= scratch < over["workspace_bytes"]
+    cfg = I.ScanConfig("na_auto", batch, seqlen, dim, 16, io="bf16", seed=33, h0_sigma=0.3, d_skip="uniform")
+    x = I.scan_inputs(cfg)
+    d = _dev(x, "bf16")
+    for _ in range(2):  # two calls in a row through the same scratch
+        out, state = _run(lib, "noalloc", d, x, 0)
+        ref_state = d["h0"].clone()
+        ref_out = lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                         delta_bias=d["delta_bias"], last_state=ref_state)
+        torch.cuda.synchronize()
+        T.check_out(T.from_dev(out), T.from_dev(ref_out), "bf16")
+        T.check_state(T.from_dev(state), T.from_dev(ref_state), "bf16")
+    # sampled channels of every batch row against the fp64 oracle
+    dsel = np.array([0, 1, 127, 128, dim // 2 + 5, dim - 1])
+    ro, rs = _oracle_rows(x, "bf16", dsel)
+    ds = torch.as_tensor(dsel, device="cuda")
+    T.check_out(T.from_dev(out[:, :, ds]), ro, "bf16")
+    T.check_state(T.from_dev(state[:, ds]), rs, "bf16")
