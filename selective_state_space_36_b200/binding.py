@@ -105,7 +105,7 @@ def _load() -> ctypes.CDLL:
     lib.ssm_version.restype = ctypes.c_int
     lib.ssm_get_build_info.argtypes = [ctypes.POINTER(SSMBuildInfo)]
     lib.ssm_get_build_info.restype = None
-    lib.ssm_ssd_scan_fwd.argtypes = [SSMSsdDims, ctypes.c_int] + [_vp] * 9 + [ctypes.c_int, _vp, _vp, _vp]
+    lib.ssm_ssd_scan_fwd.argtypes = [SSMSsdDims, ctypes.c_int] + [_vp] * 8 + [ctypes.c_int, _vp, _vp, _vp]
     lib.ssm_ssd_scan_fwd.restype = ctypes.c_int
     lib.ssm_test_exp2_poly.argtypes = [_vp, _vp, _vp, ctypes.c_int64, _vp]
     lib.ssm_test_exp2_poly.restype = ctypes.c_int

@@ -129,15 +129,18 @@ __device__ __forceinline__ void vblock_sync(int vb) {
     else asm volatile("bar.sync %0, %1;" ::"r"(vb + 1), "n"(TPB) : "memory");
 }
 
-// Threads a CTA of the staged kernel may have (several virtual blocks): at
-// most 256, so that ptxas may give every thread 255 registers.
-template <int G>
+// Threads a CTA of the staged kernel may have.  Only the one-pass mode packs
+// several virtual blocks per CTA: up to 512 threads for layouts whose lanes
+// hold at most 8 states (they stay below 128 registers), else 256, so that
+// ptxas may give every thread up to 255 registers.  The other modes launch
+// one 128-thread block per unit.
+template <int G, int NS, int CPL, int MODE>
 struct StagedMaxThreads {
-    static constexpr int value = 256;
+    static constexpr int value = MODE != kFull ? kBlock : (G > 1 && NS * CPL <= 8 ? 512 : 256);
 };
 
 template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH, int TPB>
-__global__ void __launch_bounds__(StagedMaxThreads<G>::value)
+__global__ void __launch_bounds__(StagedMaxThreads<G, NS, CPL, MODE>::value)
 scan_fwd_staged_kernel(const ScanArgs args) {
     using io = io_traits<IO>;
     using Lay = StagedLayout<IO, NS, G, CPL, TPB>;
@@ -443,7 +446,7 @@ inline cudaError_t launch_mode(ScanArgs a, int64_t units, unsigned nseg, cudaStr
     int sms = 0, optin = 0;
     cudaError_t e = staged_device_limits(&sms, &optin);
     if (e != cudaSuccess) return e;
-    int vmax = StagedMaxThreads<G>::value / TPB;
+    int vmax = StagedMaxThreads<G, NS, CPL, MODE>::value / TPB;
 #ifdef SSM_VPB_MAX
     if (vmax > SSM_VPB_MAX) vmax = SSM_VPB_MAX;
 #endif
@@ -465,8 +468,11 @@ inline cudaError_t launch_mode(ScanArgs a, int64_t units, unsigned nseg, cudaStr
         }
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
+    // one CTA per SM with all units resident at once; when the units do not
+    // fit that way, CTAs of several units would spread unevenly over the SMs,
+    // so one unit per CTA is launched instead
     int64_t vpb = (units + sms - 1) / sms;
-    if (vpb > vmax) vpb = vmax;
+    if (vpb > vmax) vpb = 1;
     if (vpb < 1) vpb = 1;
     const int64_t gx = (units + vpb - 1) / vpb;
     if (gx > 2147483647LL) return cudaErrorInvalidConfiguration;

@@ -221,9 +221,14 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 
 // Pairs of states whose decays use exp2_poly2 instead of the SFU: pair p of a
 // lane's states does when (p mod 4) < SSM_POLY_PAIRS, i.e. SSM_POLY_PAIRS / 4
-// of the decays (for lanes holding at least 8 states).
+// of the decays (for lanes holding at least 8 states).  Off by default: on
+// B200 the one-lane scan at the 1.4B-layer shape measured 156.6 Gelem/s with
+// every decay on the SFU, 126.9 with a quarter and 111.7 with half of them on
+// the polynomial -- with ~1.75 warps per scheduler the kernel is bound by
+// the latency of each warp's instruction stream, not by SFU throughput, and
+// the polynomial lengthens that stream.
 #ifndef SSM_POLY_PAIRS
-#define SSM_POLY_PAIRS 1
+#define SSM_POLY_PAIRS 0
 #endif
 __device__ __forceinline__ constexpr bool poly_pair(int p) { return (p & 3) < SSM_POLY_PAIRS; }
 
