@@ -355,12 +355,301 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
     if (warp == 0) tmem_dealloc(tm, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Pipelined form: the tiles of chunk c + 1 (C, B, X; two stages) are copied
+// while chunk c computes, the masked intra-chunk matrix M stays in tensor
+// memory as the A operand of M X (no shared-memory round trip), and z / out
+// move between registers and global memory directly, so that the double
+// buffers fit in shared memory.  Inside a chunk the products and the
+// element-wise phases overlap: C B^T and C H^T run while the threads form
+// w o X; B^T (w o X) runs while they mask C B^T; M X runs while they update
+// the carried state.
+enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kNumTiles2 };
+constexpr uint32_t kSmemBytes2 = kNumTiles2 * kTileBytes + 1024;
+constexpr uint32_t kColM = 320;  // bf16 M as the A operand: 64 columns (two values per column)
+
+__global__ void __launch_bounds__(kThreads, 1)
+ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+                         const __grid_constant__ CUtensorMap mapC, const __nv_bfloat16 *__restrict__ zg,
+                         __nv_bfloat16 *__restrict__ og, const SsdArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                          ~static_cast<uintptr_t>(1023));
+    auto tile = [&](int i) { return sm + (uint32_t)i * kTileBytes; };
+    __shared__ uint64_t bar_ld[2], bar_mma1, bar_mma2, bar_mma3;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[8];
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = (warp & 3) * 32 + lane;
+    const int half = warp >> 2;
+    const int64_t b = blockIdx.x / a.heads, h = blockIdx.x % a.heads;
+    const int g = (int)(h / (a.heads / a.groups));
+    const int N = a.dstate;
+    const int ntiles = N / 64, ksteps = N / 16;
+    const int64_t L = a.seqlen;
+    const float Ah = a.A[h] * kLog2e;
+    const float Dh = a.D ? a.D[h] : 0.f;
+    const float bias = a.dt_bias ? a.dt_bias[h] : 0.f;
+    const __nv_bfloat16 *dt = static_cast<const __nv_bfloat16 *>(a.dt);
+
+    if (tid == 0) {
+        mbar_init(&bar_ld[0], 1);
+        mbar_init(&bar_ld[1], 1);
+        mbar_init(&bar_mma1, 1);
+        mbar_init(&bar_mma2, 1);
+        mbar_init(&bar_mma3, 1);
+        mbar_fence_init();
+        s_abort = 0;
+    }
+    if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = s_tmem;
+    const uint32_t tlane = tm + ((uint32_t)((warp & 3) * 32) << 16);
+    const int nchunks = (int)((L + kQ - 1) / kQ);
+
+    auto issue = [&](int cc) {  // thread 0: the tiles of chunk cc into stage cc & 1
+        const int st = cc & 1;
+        const int base = st ? kC0s1 : kC0s0;
+        mbar_expect_tx(&bar_ld[st], (uint32_t)(2 * ntiles + 1) * kTileBytes);
+        const int32_t t0 = cc * kQ;
+        for (int kt = 0; kt < ntiles; ++kt) {
+            tma_load_3d(tile(base + kt), &mapC, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
+            tma_load_3d(tile(base + 2 + kt), &mapB, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
+        }
+        tma_load_3d(tile(base + 4), &mapX, (int32_t)(h * kP), t0, (int32_t)b, &bar_ld[st]);
+    };
+    if (tid == 0 && nchunks > 0) issue(0);
+
+    float H[32];
+    const bool nrow = r < N;
+    const int64_t sbase = ((b * a.heads + h) * kP + 32 * half) * N + r;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
+        store_piece(tile(kH2), r, 4 * half + j, v);
+    }
+    fence_proxy_async();
+    __syncthreads();
+
+    auto wait = [&](uint64_t *bar, uint32_t par) {
+        if (!mbar_wait(bar, par, kWaitNs)) {
+            atomicOr(a.status, 2u);
+            s_abort = 1;
+        }
+    };
+
+    int c = 0;
+    for (; c < nchunks; ++c) {
+        const int st = c & 1;
+        const int64_t t0 = (int64_t)c * kQ;
+        const int64_t trow = t0 + r;
+        const bool valid = trow < L;
+        const int tC0 = st ? kC0s1 : kC0s0, tB0 = tC0 + 2, tX = tC0 + 4;
+        // 1. the next chunk's tiles into the other stage (its last readers,
+        // the previous chunk's products and threads, are done)
+        if (tid == 0 && c + 1 < nchunks) issue(c + 1);
+        // 2. z of row r (this thread's half of the head's channels) into
+        // registers, Delta and its running sum
+        uint4 zr[4];
+        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            zr[j] = (zg && valid) ? __ldg(reinterpret_cast<const uint4 *>(zg + grow) + j) : make_uint4(0, 0, 0, 0);
+        float dl = 0.f;
+        if (valid) {
+            const float sv = __bfloat162float(dt[(b * L + trow) * a.heads + h]) + bias;
+            dl = a.softplus ? softplus<false>(sv) : sv;
+        }
+        float cum = dl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, cum, o);
+            if (lane >= o) cum += v;
+        }
+        if (lane == 31) s_wsum[warp] = cum;
+        __syncthreads();
+        for (int w2 = 0; w2 < (warp & 3); ++w2) cum += s_wsum[(warp & ~3) + w2];
+        if (half == 0) {
+            s_dl[r] = dl;
+            s_cum[r] = cum;
+        }
+        wait(&bar_ld[st], (uint32_t)(c >> 1) & 1u);
+        __syncthreads();
+        if (s_abort) break;
+        const float cum_end = s_cum[kQ - 1];
+
+        // 3. C B^T and C H_prev^T
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id_cb = idesc_bf16(128, 128, kMajorK, kMajorK);
+            const uint32_t id_yo = idesc_bf16(128, kP, kMajorK, kMajorMN);
+            for (int k = 0; k < ksteps; ++k) {
+                const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
+                const uint64_t bd = desc_sw128(smem_u32(tile(tB0 + k / 4)) + (k % 4) * 32, 16, 1024);
+                mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
+            }
+            for (int k = 0; k < ksteps; ++k) {
+                const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
+                const uint64_t bd = desc_sw128(smem_u32(tile(kH2)) + k * 2048, 16, 1024);
+                mma_bf16(tm + kColYoff, ad, bd, id_yo, k > 0);
+            }
+            mma_commit(&bar_mma1);
+        }
+        // 4. w o X as bf16 high and low parts
+        {
+            const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float x8[8], hi[8], lo[8];
+                load_piece(tile(tX), r, 4 * half + j, x8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float xw = w * x8[i];
+                    hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
+                    lo[i] = xw - hi[i];
+                }
+                store_piece(tile(kXh2), r, 4 * half + j, hi);
+                store_piece(tile(kXl2), r, 4 * half + j, lo);
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        // 5. chunk state B^T (w o X)
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id_s = idesc_bf16(128, kP, kMajorMN, kMajorMN);
+            for (int part = 0; part < 2; ++part)
+                for (int k = 0; k < kQ / 16; ++k) {
+                    const uint64_t ad = desc_sw128(smem_u32(tile(tB0)) + k * 2048, kTileBytes, 1024);
+                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kXl2 : kXh2)) + k * 2048, 16, 1024);
+                    mma_bf16(tm + kColS, ad, bd, id_s, part > 0 || k > 0);
+                }
+            mma_commit(&bar_mma2);
+        }
+        // 6. M = Lmask o C B^T o Delta_s, row t = r, columns s of this half,
+        // into tensor memory (two bf16 per column)
+        wait(&bar_mma1, (uint32_t)c & 1u);
+        fence_after_sync();
+        {
+            uint32_t packed[32];
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                float cb[32];
+                tmem_ld32(tlane + kColCB + 64 * half + 32 * blk, cb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int s0 = 64 * half + 32 * blk + 2 * i;
+                    const float m0 = s0 <= r ? cb[2 * i] * ex2_approx(Ah * (cum - s_cum[s0])) * s_dl[s0] : 0.f;
+                    const float m1 =
+                        s0 + 1 <= r ? cb[2 * i + 1] * ex2_approx(Ah * (cum - s_cum[s0 + 1])) * s_dl[s0 + 1] : 0.f;
+                    packed[16 * blk + i] = pack_bf16x2(m0, m1);
+                }
+            }
+            tmem_st32(tlane + kColM + 32 * half, packed);
+            tmem_wait_st();
+        }
+        fence_before_sync();
+        __syncthreads();
+        if (s_abort) break;
+        // 7. Y_diag = M X, M from tensor memory
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id_y = idesc_bf16(128, kP, kMajorK, kMajorMN);
+            for (int k = 0; k < kQ / 16; ++k) {
+                const uint64_t bd = desc_sw128(smem_u32(tile(tX)) + k * 2048, 16, 1024);
+                mma_bf16_ts(tm + kColY, tm + kColM + 8 * k, bd, id_y, k > 0);
+            }
+            mma_commit(&bar_mma3);
+        }
+        // 8. carried state
+        wait(&bar_mma2, (uint32_t)c & 1u);
+        fence_after_sync();
+        {
+            float sv[32];
+            tmem_ld32(tlane + kColS + 32 * half, sv);
+            tmem_wait_ld();
+            const float gdec = ex2_approx(Ah * cum_end);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
+                store_piece(tile(kH2), r, 4 * half + j, v);
+            }
+        }
+        // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), straight to global memory
+        wait(&bar_mma3, (uint32_t)c & 1u);
+        fence_after_sync();
+        {
+            float yd[32], yo[32];
+            tmem_ld32(tlane + kColY + 32 * half, yd);
+            tmem_ld32(tlane + kColYoff + 32 * half, yo);
+            tmem_wait_ld();
+            const float et = ex2_approx(Ah * cum);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float x8[8];
+                load_piece(tile(tX), r, 4 * half + j, x8);
+                const uint32_t zw[4] = {zr[j].x, zr[j].y, zr[j].z, zr[j].w};
+                uint32_t ow[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float y0 = fmaf(Dh, x8[2 * i], fmaf(et, yo[8 * j + 2 * i], yd[8 * j + 2 * i]));
+                    float y1 = fmaf(Dh, x8[2 * i + 1], fmaf(et, yo[8 * j + 2 * i + 1], yd[8 * j + 2 * i + 1]));
+                    if (zg) {
+                        y0 *= silu<false>(__uint_as_float(zw[i] << 16));
+                        y1 *= silu<false>(__uint_as_float(zw[i] & 0xffff0000u));
+                    }
+                    ow[i] = pack_bf16x2(y0, y1);
+                }
+                if (valid) reinterpret_cast<uint4 *>(og + grow)[j] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (s_abort) break;
+    }
+    if (s_abort) {
+        // let whatever was issued finish (bounded) before the memory goes away
+        (void)mbar_wait(&bar_ld[c & 1], (uint32_t)(c >> 1) & 1u, kWaitNs);
+        if (c + 1 < nchunks) (void)mbar_wait(&bar_ld[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u, kWaitNs);
+        (void)mbar_wait(&bar_mma1, (uint32_t)c & 1u, kWaitNs);
+        (void)mbar_wait(&bar_mma2, (uint32_t)c & 1u, kWaitNs);
+        (void)mbar_wait(&bar_mma3, (uint32_t)c & 1u, kWaitNs);
+    } else if (a.state && nrow) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a.state[sbase + (int64_t)i * N] = H[i];
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, kTmemCols);
+}
+
 }  // namespace
 }  // namespace ssm
 
 namespace ssm {
 
 namespace {
+
+// 1: the pipelined kernel (double-buffered tiles, M in tensor memory);
+// 0: the plain one (one chunk at a time, every tile in shared memory).
+#ifndef SSM_SSD_PIPELINED
+#define SSM_SSD_PIPELINED 1
+#endif
+constexpr bool kSsdPipelined = SSM_SSD_PIPELINED != 0;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -435,12 +724,19 @@ cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (!configured[dev & 63]) {
         e = cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes2);
         if (e != cudaSuccess) return e;
         configured[dev & 63] = true;
     }
     const int64_t grid = a.batch * a.heads;
     if (grid > 2147483647LL) return cudaErrorInvalidConfiguration;
-    ssd_fwd_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mx, mz, mb, mc, mo, k);
+    if (kSsdPipelined)
+        ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads, kSmemBytes2, st>>>(
+            mx, mb, mc, static_cast<const __nv_bfloat16 *>(a.z), static_cast<__nv_bfloat16 *>(a.out), k);
+    else
+        ssd_fwd_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mx, mz, mb, mc, mo, k);
     return cudaGetLastError();
 }
 
