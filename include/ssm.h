@@ -345,9 +345,10 @@ ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
  * Supported: io = SSM_BF16, headdim = 64, dstate = 64 or 128, heads a
  * multiple of groups, x, z, B, C, out 16-byte aligned (SSM_ERR_UNSUPPORTED
  * otherwise).  Arithmetic: products on the tensor cores with bf16 operands
- * and fp32 accumulation; the intra-chunk matrix and the state copy read by
- * the inter-chunk product are rounded to bf16, the state itself is carried in
- * fp32 and updated from a two-term (high + low bf16) product.  A wait inside
+ * and fp32 accumulation; the masked intra-chunk matrix is rounded to bf16;
+ * the state is carried in fp32, and both products that involve it (the
+ * chunk's state update and the inter-chunk output) take a two-term operand,
+ * a bf16 high part plus the bf16 rounding of the rest.  A wait inside
  * the kernel that runs out (2 s) sets bit 1 of the device status word
  * (ssm_get_device_status); the outputs are then not valid.
  */

@@ -395,15 +395,19 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     }
 }
 
-// Threads of a virtual block of the one-pass scan, by lanes per channel.  One
-// warp per virtual block (32 channels at one lane per channel) gives the
-// finest unit of work, so the units spread over the SMs with the least
-// imbalance; each virtual block widens its own copy of the B/C rows.
+// Threads of a virtual block of the one-pass scan, by lanes per channel.
+// Measured on B200 (Gelem/s; 1.4B layer = 32,768 channels, 130M layer =
+// 12,288 channels): two lanes per channel in 64-thread virtual blocks, seven
+// per CTA, 164.6 at the 1.4B layer (one lane: 156.7 in one-warp virtual
+// blocks, 155.9 in 128-thread blocks); four lanes in 128-thread blocks, one
+// per CTA, 122.6 at the 130M layer (packed three per CTA: 113.6; 32- or
+// 64-thread virtual blocks: 104-108, each re-widening the B/C rows for fewer
+// channels).
 #ifndef SSM_VB_THREADS_G1
-#define SSM_VB_THREADS_G1 32
+#define SSM_VB_THREADS_G1 128
 #endif
 #ifndef SSM_VB_THREADS_G2
-#define SSM_VB_THREADS_G2 128
+#define SSM_VB_THREADS_G2 64
 #endif
 #ifndef SSM_VB_THREADS_G4
 #define SSM_VB_THREADS_G4 128
@@ -450,6 +454,7 @@ inline cudaError_t launch_mode(ScanArgs a, int64_t units, unsigned nseg, cudaStr
 #ifdef SSM_VPB_MAX
     if (vmax > SSM_VPB_MAX) vmax = SSM_VPB_MAX;
 #endif
+    if (G == 4) vmax = 1;  // one block per unit measured faster for four lanes (see SSM_VB_THREADS_G*)
     if (TPB > 32 && vmax > 15) vmax = 15;  // hardware barriers 1..15
     if ((size_t)vmax * Lay::SMEM > (size_t)optin) vmax = (int)((size_t)optin / Lay::SMEM);
     if (MODE != kFull) vmax = 1;

@@ -52,7 +52,7 @@ constexpr uint32_t kTileBytes = kQ * 128;  // 128 rows x 128 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
 // shared memory: 1024-byte aligned 16 KB tiles
-enum Tile { kC0, kC1, kB0, kB1, kX, kZ, kM0, kM1, kXh, kXl, kH, kNumTiles };
+enum Tile { kC0, kC1, kB0, kB1, kX, kZ, kM0, kM1, kXh, kXl, kH, kHl, kNumTiles };
 constexpr uint32_t kSmemBytes = kNumTiles * kTileBytes + 1024;
 
 // TMEM columns (fp32): C B^T, Y_diag, Y_off, chunk state
@@ -91,6 +91,25 @@ __device__ __forceinline__ void store_piece(unsigned char *tile, int row, int pi
     w.z = pack_bf16x2(v[4], v[5]);
     w.w = pack_bf16x2(v[6], v[7]);
     *reinterpret_cast<uint4 *>(tile + sw128_offset(row, piece)) = w;
+}
+
+// The carried state's copy for C H^T: bf16(H) in `hi` and the bf16 rounding
+// of H - bf16(H) in `lo` (rows n = r, this thread's 32 of the 64 channels),
+// so that the product with C keeps ~2^-17 relative accuracy; one bf16 term
+// would put ~1e-2 of error into the output when the state is large.
+__device__ __forceinline__ void store_state_split(unsigned char *hi, unsigned char *lo, int r, int half,
+                                                  const float (&H)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float vh[8], vl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            vh[i] = __bfloat162float(__float2bfloat16_rn(H[8 * j + i]));
+            vl[i] = H[8 * j + i] - vh[i];
+        }
+        store_piece(hi, r, 4 * half + j, vh);
+        store_piece(lo, r, 4 * half + j, vl);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -142,13 +161,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
     const int64_t sbase = ((b * a.heads + h) * kP + 32 * half) * N + r;
 #pragma unroll
     for (int i = 0; i < 32; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
-        store_piece(tile(kH), r, 4 * half + j, v);
-    }
+    store_state_split(tile(kH), tile(kHl), r, half, H);
     fence_proxy_async();
     __syncthreads();
 
@@ -211,11 +224,12 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
                 const uint64_t bd = desc_sw128(smem_u32(tile(kB0 + k / 4)) + (k % 4) * 32, 16, 1024);
                 mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
             }
-            for (int k = 0; k < ksteps; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(tile(kC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(tile(kH)) + k * 2048, 16, 1024);
-                mma_bf16(tm + kColYoff, ad, bd, id_yo, k > 0);
-            }
+            for (int part = 0; part < 2; ++part)
+                for (int k = 0; k < ksteps; ++k) {
+                    const uint64_t ad = desc_sw128(smem_u32(tile(kC0 + k / 4)) + (k % 4) * 32, 16, 1024);
+                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kHl : kH)) + k * 2048, 16, 1024);
+                    mma_bf16(tm + kColYoff, ad, bd, id_yo, part > 0 || k > 0);
+                }
             mma_commit(&bar_mma1);
         }
 
@@ -297,13 +311,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
             const float gdec = ex2_approx(Ah * cum_end);
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
-                store_piece(tile(kH), r, 4 * half + j, v);
-            }
+            store_state_split(tile(kH), tile(kHl), r, half, H);
         }
         // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(Z), into tile kZ
         wait(&bar_mma3, par);
@@ -364,7 +372,8 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
 // element-wise phases overlap: C B^T and C H^T run while the threads form
 // w o X; B^T (w o X) runs while they mask C B^T; M X runs while they update
 // the carried state.
-enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kNumTiles2 };
+enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kHl2,
+             kNumTiles2 };
 constexpr uint32_t kSmemBytes2 = kNumTiles2 * kTileBytes + 1024;
 constexpr uint32_t kColM = 320;  // bf16 M as the A operand: 64 columns (two values per column)
 
@@ -379,6 +388,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
     __shared__ uint64_t bar_ld[2], bar_mma1, bar_mma2, bar_mma3;
     __shared__ uint32_t s_tmem;
     __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[8];
+    __shared__ __align__(16) float s_q[kQ];  // A S_s - log2(Delta_s), log2 units (+inf where Delta_s = 0)
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -429,13 +439,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
     const int64_t sbase = ((b * a.heads + h) * kP + 32 * half) * N + r;
 #pragma unroll
     for (int i = 0; i < 32; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
-        store_piece(tile(kH2), r, 4 * half + j, v);
-    }
+    store_state_split(tile(kH2), tile(kHl2), r, half, H);
     fence_proxy_async();
     __syncthreads();
 
@@ -445,6 +449,20 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
             s_abort = 1;
         }
     };
+
+    // z (this thread's 32 channels of row r) and dt of chunk cc, into registers
+    uint4 zn[4];
+    float dtn = 0.f;
+    auto prefetch = [&](int cc) {
+        const int64_t t = (int64_t)cc * kQ + r;
+        const bool ok = cc < nchunks && t < L;
+        const int64_t gr = ((b * L + t) * a.heads + h) * kP + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            zn[j] = (zg && ok) ? __ldg(reinterpret_cast<const uint4 *>(zg + gr) + j) : make_uint4(0, 0, 0, 0);
+        dtn = ok ? __bfloat162float(dt[(b * L + t) * a.heads + h]) : 0.f;
+    };
+    prefetch(0);
 
     int c = 0;
     for (; c < nchunks; ++c) {
@@ -456,16 +474,18 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         // 1. the next chunk's tiles into the other stage (its last readers,
         // the previous chunk's products and threads, are done)
         if (tid == 0 && c + 1 < nchunks) issue(c + 1);
-        // 2. z of row r (this thread's half of the head's channels) into
-        // registers, Delta and its running sum
+        // 2. this chunk's z and dt of row r (prefetched one chunk ahead, so no
+        // global-memory latency sits on the chunk's chain); Delta and its
+        // running sum
         uint4 zr[4];
-        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 32 * half;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            zr[j] = (zg && valid) ? __ldg(reinterpret_cast<const uint4 *>(zg + grow) + j) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 4; ++j) zr[j] = zn[j];
+        const float dt_raw = dtn;
+        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 32 * half;
+        prefetch(c + 1);
         float dl = 0.f;
         if (valid) {
-            const float sv = __bfloat162float(dt[(b * L + trow) * a.heads + h]) + bias;
+            const float sv = dt_raw + bias;
             dl = a.softplus ? softplus<false>(sv) : sv;
         }
         float cum = dl;
@@ -480,6 +500,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         if (half == 0) {
             s_dl[r] = dl;
             s_cum[r] = cum;
+            s_q[r] = dl > 0.f ? fmaf(Ah, cum, -lg2_approx(dl)) : __int_as_float(0x7f800000);
         }
         wait(&bar_ld[st], (uint32_t)(c >> 1) & 1u);
         __syncthreads();
@@ -496,11 +517,12 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 const uint64_t bd = desc_sw128(smem_u32(tile(tB0 + k / 4)) + (k % 4) * 32, 16, 1024);
                 mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
             }
-            for (int k = 0; k < ksteps; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(tile(kH2)) + k * 2048, 16, 1024);
-                mma_bf16(tm + kColYoff, ad, bd, id_yo, k > 0);
-            }
+            for (int part = 0; part < 2; ++part)
+                for (int k = 0; k < ksteps; ++k) {
+                    const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
+                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kHl2 : kH2)) + k * 2048, 16, 1024);
+                    mma_bf16(tm + kColYoff, ad, bd, id_yo, part > 0 || k > 0);
+                }
             mma_commit(&bar_mma1);
         }
         // 4. w o X as bf16 high and low parts
@@ -538,20 +560,40 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         // into tensor memory (two bf16 per column)
         wait(&bar_mma1, (uint32_t)c & 1u);
         fence_after_sync();
+        // M[t, s] = CB[t, s] exp(A (S_t - S_s)) Delta_s = CB[t, s] 2^(p_t - q_s)
+        // with p_t = A S_t and q_s = A S_s - log2(Delta_s) (log2 units; a zero
+        // Delta_s gives q_s = +inf and M = 0) when Delta = softplus(.) >= 0;
+        // 32-column blocks that lie above the diagonal for the whole warp
+        // are zero without arithmetic.
         {
+            const float pt = Ah * cum;
             uint32_t packed[32];
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
+                const int sb = 64 * half + 32 * blk;
+                if (sb > (warp & 3) * 32 + 31) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) packed[16 * blk + i] = 0u;
+                    continue;
+                }
                 float cb[32];
-                tmem_ld32(tlane + kColCB + 64 * half + 32 * blk, cb);
+                tmem_ld32(tlane + kColCB + sb, cb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int s0 = 64 * half + 32 * blk + 2 * i;
-                    const float m0 = s0 <= r ? cb[2 * i] * ex2_approx(Ah * (cum - s_cum[s0])) * s_dl[s0] : 0.f;
-                    const float m1 =
-                        s0 + 1 <= r ? cb[2 * i + 1] * ex2_approx(Ah * (cum - s_cum[s0 + 1])) * s_dl[s0 + 1] : 0.f;
-                    packed[16 * blk + i] = pack_bf16x2(m0, m1);
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 q4 = *reinterpret_cast<const float4 *>(s_q + sb + 4 * i4);
+                    const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+                    float m[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s0 = sb + 4 * i4 + e;
+                        // without softplus Delta may be negative: keep the product form
+                        const float f = a.softplus ? ex2_approx(pt - qv[e])
+                                                   : ex2_approx(Ah * (cum - s_cum[s0])) * s_dl[s0];
+                        m[e] = s0 <= r ? cb[4 * i4 + e] * f : 0.f;
+                    }
+                    packed[16 * blk + 2 * i4] = pack_bf16x2(m[0], m[1]);
+                    packed[16 * blk + 2 * i4 + 1] = pack_bf16x2(m[2], m[3]);
                 }
             }
             tmem_st32(tlane + kColM + 32 * half, packed);
@@ -580,13 +622,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
             const float gdec = ex2_approx(Ah * cum_end);
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
-                store_piece(tile(kH2), r, 4 * half + j, v);
-            }
+            store_state_split(tile(kH2), tile(kHl2), r, half, H);
         }
         // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), straight to global memory
         wait(&bar_mma3, (uint32_t)c & 1u);

@@ -85,13 +85,16 @@ void scan_layout(int64_t dstate, int64_t channels, int sms, int lanes_req, int *
     if (dstate <= 16) {
         int G = lanes_req;
         if (G != 1 && G != 2 && G != 4) {
-            // One lane per channel (all 16 states) once the channels give the
-            // SMs 1.5 blocks of 128 on average (most SMs then hold two): no
-            // shuffles, ~40% fewer instructions per element, and it measured
-            // ~5% faster at the 1.4B-layer shape (32,768 channels).  Below
-            // that, four lanes per channel (4 states each) quadruple the warps
-            // that hide latency and even out the work per SM.
-            G = 2 * channels >= (int64_t)sms * ssm::kBlock * 3 ? 1 : 4;
+            // Below 1.5 blocks of 128 channels per SM, four lanes per channel
+            // (4 states each) give the warps that hide latency.  From there
+            // up to what one CTA per SM holds in 64-thread virtual blocks of
+            // two lanes per channel (8 per CTA: 256 channels per SM), two
+            // lanes: the 1.4B layer (32,768 channels) measured 164.6 Gelem/s
+            // against 156.7 with one lane.  Beyond that, one lane per channel
+            // (all 16 states, no shuffles) in 128-thread blocks.
+            if (2 * channels < (int64_t)sms * ssm::kBlock * 3) G = 4;
+            else if (channels <= (int64_t)sms * 256) G = 2;
+            else G = 1;
         }
         *g = G;
         *ns = 16 / G;
