@@ -375,9 +375,31 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__
 enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kHl2,
              kNumTiles2 };
 constexpr uint32_t kSmemBytes2 = kNumTiles2 * kTileBytes + 1024;
-constexpr uint32_t kColM = 320;  // bf16 M as the A operand: 64 columns (two values per column)
+constexpr int kThreads2 = 512;   // 16 warps: four per scheduler to hide latency
+constexpr uint32_t kColM = 320;  // M as the A operand, high part: 64 columns (two bf16 per column)
+constexpr uint32_t kColMl = 384; // low part
 
-__global__ void __launch_bounds__(kThreads, 1)
+// The carried state's two-term copy (this thread's 16 of the 64 channels of
+// state row r): pieces 2 part and 2 part + 1 of the row.
+__device__ __forceinline__ void store_state_split16(unsigned char *hi, unsigned char *lo, int r, int part,
+                                                    const float (&H)[16]) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        float vh[8], vl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            vh[i] = __bfloat162float(__float2bfloat16_rn(H[8 * j + i]));
+            vl[i] = H[8 * j + i] - vh[i];
+        }
+        store_piece(hi, r, 2 * part + j, vh);
+        store_piece(lo, r, 2 * part + j, vl);
+    }
+}
+
+// Thread (warp w, lane l) owns TMEM lane / tile row r = 32 (w % 4) + l and
+// the quarter part = w / 4 of the columns: channels [16 part, 16 part + 16)
+// of the head, mask columns [32 part, 32 part + 32).
+__global__ void __launch_bounds__(kThreads2, 1)
 ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
                          const __grid_constant__ CUtensorMap mapC, const __nv_bfloat16 *__restrict__ zg,
                          __nv_bfloat16 *__restrict__ og, const SsdArgs a) {
@@ -387,13 +409,13 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
     auto tile = [&](int i) { return sm + (uint32_t)i * kTileBytes; };
     __shared__ uint64_t bar_ld[2], bar_mma1, bar_mma2, bar_mma3;
     __shared__ uint32_t s_tmem;
-    __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[8];
+    __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[16];
     __shared__ __align__(16) float s_q[kQ];  // A S_s - log2(Delta_s), log2 units (+inf where Delta_s = 0)
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = (warp & 3) * 32 + lane;
-    const int half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;
+    const int r = quad * 32 + lane;
     const int64_t b = blockIdx.x / a.heads, h = blockIdx.x % a.heads;
     const int g = (int)(h / (a.heads / a.groups));
     const int N = a.dstate;
@@ -418,7 +440,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = s_tmem;
-    const uint32_t tlane = tm + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t tlane = tm + ((uint32_t)(quad * 32) << 16);
     const int nchunks = (int)((L + kQ - 1) / kQ);
 
     auto issue = [&](int cc) {  // thread 0: the tiles of chunk cc into stage cc & 1
@@ -434,12 +456,13 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
     };
     if (tid == 0 && nchunks > 0) issue(0);
 
-    float H[32];
+    // carried state H[n = r][p = 16 part + i], fp32
+    float H[16];
     const bool nrow = r < N;
-    const int64_t sbase = ((b * a.heads + h) * kP + 32 * half) * N + r;
+    const int64_t sbase = ((b * a.heads + h) * kP + 16 * part) * N + r;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
-    store_state_split(tile(kH2), tile(kHl2), r, half, H);
+    for (int i = 0; i < 16; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
+    store_state_split16(tile(kH2), tile(kHl2), r, part, H);
     fence_proxy_async();
     __syncthreads();
 
@@ -450,15 +473,15 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         }
     };
 
-    // z (this thread's 32 channels of row r) and dt of chunk cc, into registers
-    uint4 zn[4];
+    // z (this thread's 16 channels of row r) and dt of chunk cc, into registers
+    uint4 zn[2];
     float dtn = 0.f;
     auto prefetch = [&](int cc) {
         const int64_t t = (int64_t)cc * kQ + r;
         const bool ok = cc < nchunks && t < L;
-        const int64_t gr = ((b * L + t) * a.heads + h) * kP + 32 * half;
+        const int64_t gr = ((b * L + t) * a.heads + h) * kP + 16 * part;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
             zn[j] = (zg && ok) ? __ldg(reinterpret_cast<const uint4 *>(zg + gr) + j) : make_uint4(0, 0, 0, 0);
         dtn = ok ? __bfloat162float(dt[(b * L + t) * a.heads + h]) : 0.f;
     };
@@ -474,14 +497,11 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         // 1. the next chunk's tiles into the other stage (its last readers,
         // the previous chunk's products and threads, are done)
         if (tid == 0 && c + 1 < nchunks) issue(c + 1);
-        // 2. this chunk's z and dt of row r (prefetched one chunk ahead, so no
-        // global-memory latency sits on the chunk's chain); Delta and its
-        // running sum
-        uint4 zr[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) zr[j] = zn[j];
+        // 2. this chunk's z and dt (prefetched a chunk ahead); Delta and its
+        // running sum over the chunk
+        const uint4 zr0 = zn[0], zr1 = zn[1];
         const float dt_raw = dtn;
-        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 32 * half;
+        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 16 * part;
         prefetch(c + 1);
         float dl = 0.f;
         if (valid) {
@@ -496,8 +516,8 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         }
         if (lane == 31) s_wsum[warp] = cum;
         __syncthreads();
-        for (int w2 = 0; w2 < (warp & 3); ++w2) cum += s_wsum[(warp & ~3) + w2];
-        if (half == 0) {
+        for (int w2 = 0; w2 < quad; ++w2) cum += s_wsum[4 * part + w2];
+        if (part == 0) {
             s_dl[r] = dl;
             s_cum[r] = cum;
             s_q[r] = dl > 0.f ? fmaf(Ah, cum, -lg2_approx(dl)) : __int_as_float(0x7f800000);
@@ -507,7 +527,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         if (s_abort) break;
         const float cum_end = s_cum[kQ - 1];
 
-        // 3. C B^T and C H_prev^T
+        // 3. C B^T and C H_prev^T (two-term state copy)
         if (tid == 0) {
             fence_after_sync();
             const uint32_t id_cb = idesc_bf16(128, 128, kMajorK, kMajorK);
@@ -517,29 +537,29 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 const uint64_t bd = desc_sw128(smem_u32(tile(tB0 + k / 4)) + (k % 4) * 32, 16, 1024);
                 mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
             }
-            for (int part = 0; part < 2; ++part)
+            for (int hp = 0; hp < 2; ++hp)
                 for (int k = 0; k < ksteps; ++k) {
                     const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kHl2 : kH2)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColYoff, ad, bd, id_yo, part > 0 || k > 0);
+                    const uint64_t bd = desc_sw128(smem_u32(tile(hp ? kHl2 : kH2)) + k * 2048, 16, 1024);
+                    mma_bf16(tm + kColYoff, ad, bd, id_yo, hp > 0 || k > 0);
                 }
             mma_commit(&bar_mma1);
         }
-        // 4. w o X as bf16 high and low parts
+        // 4. w o X as bf16 high and low parts, w_s = exp(A (S_end - S_s)) Delta_s
         {
             const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 float x8[8], hi[8], lo[8];
-                load_piece(tile(tX), r, 4 * half + j, x8);
+                load_piece(tile(tX), r, 2 * part + j, x8);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float xw = w * x8[i];
                     hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
                     lo[i] = xw - hi[i];
                 }
-                store_piece(tile(kXh2), r, 4 * half + j, hi);
-                store_piece(tile(kXl2), r, 4 * half + j, lo);
+                store_piece(tile(kXh2), r, 2 * part + j, hi);
+                store_piece(tile(kXl2), r, 2 * part + j, lo);
             }
         }
         fence_proxy_async();
@@ -548,34 +568,29 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         if (tid == 0) {
             fence_after_sync();
             const uint32_t id_s = idesc_bf16(128, kP, kMajorMN, kMajorMN);
-            for (int part = 0; part < 2; ++part)
+            for (int xp = 0; xp < 2; ++xp)
                 for (int k = 0; k < kQ / 16; ++k) {
                     const uint64_t ad = desc_sw128(smem_u32(tile(tB0)) + k * 2048, kTileBytes, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kXl2 : kXh2)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColS, ad, bd, id_s, part > 0 || k > 0);
+                    const uint64_t bd = desc_sw128(smem_u32(tile(xp ? kXl2 : kXh2)) + k * 2048, 16, 1024);
+                    mma_bf16(tm + kColS, ad, bd, id_s, xp > 0 || k > 0);
                 }
             mma_commit(&bar_mma2);
         }
-        // 6. M = Lmask o C B^T o Delta_s, row t = r, columns s of this half,
-        // into tensor memory (two bf16 per column)
+        // 6. M[t, s] = CB[t, s] exp(A (S_t - S_s)) Delta_s for row t = r and the
+        // 32 columns of this part, as bf16 high and low parts in tensor memory:
+        // CB 2^(p_t - q_s), p_t = A S_t, q_s = A S_s - log2(Delta_s) when Delta
+        // is a softplus (>= 0), the product form otherwise; a block of columns
+        // above the diagonal for the whole warp is zero without arithmetic.
         wait(&bar_mma1, (uint32_t)c & 1u);
         fence_after_sync();
-        // M[t, s] = CB[t, s] exp(A (S_t - S_s)) Delta_s = CB[t, s] 2^(p_t - q_s)
-        // with p_t = A S_t and q_s = A S_s - log2(Delta_s) (log2 units; a zero
-        // Delta_s gives q_s = +inf and M = 0) when Delta = softplus(.) >= 0;
-        // 32-column blocks that lie above the diagonal for the whole warp
-        // are zero without arithmetic.
         {
-            const float pt = Ah * cum;
-            uint32_t packed[32];
+            const int sb = 32 * part;
+            uint32_t mh[16], ml[16];
+            if (sb > quad * 32 + 31) {
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                const int sb = 64 * half + 32 * blk;
-                if (sb > (warp & 3) * 32 + 31) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[16 * blk + i] = 0u;
-                    continue;
-                }
+                for (int i = 0; i < 16; ++i) mh[i] = ml[i] = 0u;
+            } else {
+                const float pt = Ah * cum;
                 float cb[32];
                 tmem_ld32(tlane + kColCB + sb, cb);
                 tmem_wait_ld();
@@ -583,61 +598,66 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 for (int i4 = 0; i4 < 8; ++i4) {
                     const float4 q4 = *reinterpret_cast<const float4 *>(s_q + sb + 4 * i4);
                     const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-                    float m[4];
+                    float m[4], mhf[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int s0 = sb + 4 * i4 + e;
-                        // without softplus Delta may be negative: keep the product form
                         const float f = a.softplus ? ex2_approx(pt - qv[e])
                                                    : ex2_approx(Ah * (cum - s_cum[s0])) * s_dl[s0];
                         m[e] = s0 <= r ? cb[4 * i4 + e] * f : 0.f;
+                        mhf[e] = __bfloat162float(__float2bfloat16_rn(m[e]));
                     }
-                    packed[16 * blk + 2 * i4] = pack_bf16x2(m[0], m[1]);
-                    packed[16 * blk + 2 * i4 + 1] = pack_bf16x2(m[2], m[3]);
+                    mh[2 * i4] = pack_bf16x2(mhf[0], mhf[1]);
+                    mh[2 * i4 + 1] = pack_bf16x2(mhf[2], mhf[3]);
+                    ml[2 * i4] = pack_bf16x2(m[0] - mhf[0], m[1] - mhf[1]);
+                    ml[2 * i4 + 1] = pack_bf16x2(m[2] - mhf[2], m[3] - mhf[3]);
                 }
             }
-            tmem_st32(tlane + kColM + 32 * half, packed);
+            tmem_st16(tlane + kColM + 16 * part, mh);
+            tmem_st16(tlane + kColMl + 16 * part, ml);
             tmem_wait_st();
         }
         fence_before_sync();
         __syncthreads();
         if (s_abort) break;
-        // 7. Y_diag = M X, M from tensor memory
+        // 7. Y_diag = M X with both parts of M read from tensor memory
         if (tid == 0) {
             fence_after_sync();
             const uint32_t id_y = idesc_bf16(128, kP, kMajorK, kMajorMN);
-            for (int k = 0; k < kQ / 16; ++k) {
-                const uint64_t bd = desc_sw128(smem_u32(tile(tX)) + k * 2048, 16, 1024);
-                mma_bf16_ts(tm + kColY, tm + kColM + 8 * k, bd, id_y, k > 0);
-            }
+            for (int mp = 0; mp < 2; ++mp)
+                for (int k = 0; k < kQ / 16; ++k) {
+                    const uint64_t bd = desc_sw128(smem_u32(tile(tX)) + k * 2048, 16, 1024);
+                    mma_bf16_ts(tm + kColY, tm + (mp ? kColMl : kColM) + 8 * k, bd, id_y, mp > 0 || k > 0);
+                }
             mma_commit(&bar_mma3);
         }
-        // 8. carried state
+        // 8. carried state: H = exp(A S_end) H + B^T (w o X), and its copy for the next chunk
         wait(&bar_mma2, (uint32_t)c & 1u);
         fence_after_sync();
         {
-            float sv[32];
-            tmem_ld32(tlane + kColS + 32 * half, sv);
+            float sv[16];
+            tmem_ld16(tlane + kColS + 16 * part, sv);
             tmem_wait_ld();
             const float gdec = ex2_approx(Ah * cum_end);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
-            store_state_split(tile(kH2), tile(kHl2), r, half, H);
+            for (int i = 0; i < 16; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
+            store_state_split16(tile(kH2), tile(kHl2), r, part, H);
         }
         // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), straight to global memory
         wait(&bar_mma3, (uint32_t)c & 1u);
         fence_after_sync();
         {
-            float yd[32], yo[32];
-            tmem_ld32(tlane + kColY + 32 * half, yd);
-            tmem_ld32(tlane + kColYoff + 32 * half, yo);
+            float yd[16], yo[16];
+            tmem_ld16(tlane + kColY + 16 * part, yd);
+            tmem_ld16(tlane + kColYoff + 16 * part, yo);
             tmem_wait_ld();
             const float et = ex2_approx(Ah * cum);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 float x8[8];
-                load_piece(tile(tX), r, 4 * half + j, x8);
-                const uint32_t zw[4] = {zr[j].x, zr[j].y, zr[j].z, zr[j].w};
+                load_piece(tile(tX), r, 2 * part + j, x8);
+                const uint4 zq = j ? zr1 : zr0;
+                const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
                 uint32_t ow[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -666,7 +686,7 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         (void)mbar_wait(&bar_mma3, (uint32_t)c & 1u, kWaitNs);
     } else if (a.state && nrow) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) a.state[sbase + (int64_t)i * N] = H[i];
+        for (int i = 0; i < 16; ++i) a.state[sbase + (int64_t)i * N] = H[i];
     }
     fence_before_sync();
     __syncthreads();
@@ -769,7 +789,7 @@ cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     const int64_t grid = a.batch * a.heads;
     if (grid > 2147483647LL) return cudaErrorInvalidConfiguration;
     if (kSsdPipelined)
-        ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads, kSmemBytes2, st>>>(
+        ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads2, kSmemBytes2, st>>>(
             mx, mb, mc, static_cast<const __nv_bfloat16 *>(a.z), static_cast<__nv_bfloat16 *>(a.out), k);
     else
         ssd_fwd_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mx, mz, mb, mc, mo, k);

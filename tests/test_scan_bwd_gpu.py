@@ -166,9 +166,10 @@ def test_bwd_is_linear_in_dout(family):
         assert e <= 1e-4, (k, e)
 
 
-def test_bwd_staged_at_a_one_lane_forward_shape(lib):
-    # 32,768 channels, where the forward scan takes the one-lane layout (its
-    # checkpoint pass keeps four lanes per channel): all gradients
-    plan = lib.scan_plan(2, 48, 16384, 16, "bf16")
-    assert plan["lanes"] == 1
-    _check("bf16", 2, 48, 16384, 16, 17, family="staged", h0_sigma=0.5)
+@pytest.mark.parametrize("dim,fwd_lanes", [(16384, 2), (20480, 1)])
+def test_bwd_staged_at_forward_shapes_with_other_layouts(lib, dim, fwd_lanes):
+    # 32,768 and 40,960 channels, where the forward scan takes two lanes and
+    # one lane per channel (its checkpoint pass keeps four): all gradients
+    plan = lib.scan_plan(2, 48, dim, 16, "bf16")
+    assert plan["lanes"] == fwd_lanes
+    _check("bf16", 2, 48, dim, 16, 17, family="staged", h0_sigma=0.5)
