@@ -17,19 +17,21 @@
 // diagonal blocks by the quadratic form, off-diagonal blocks by the carried
 // state.  Four GEMMs per chunk and head run as tcgen05.mma with bf16
 // operands in shared memory and fp32 accumulators in tensor memory:
-//   C B^T      (128 x 128, K = dstate)    -> masked in registers, bf16 M
+//   C B^T      (128 x 128, K = dstate)    -> masked in registers
 //   M X        (128 x headdim, K = 128)
 //   C H^T      (128 x headdim, K = dstate)
-//   B^T Xw     (dstate x headdim, K = 128), twice: Xw = w o X split into a
-//              bf16 high part and the bf16 rounding of the rest, so that the
-//              state keeps fp32-level accuracy (one bf16 term would leave
-//              ~3e-3 relative error in the state).
-// Tiles of C, B, X, Z come in by TMA (cp.async.bulk.tensor, 128-byte
-// swizzle, no multicast) and out leaves by TMA store.  One CTA of 256
-// threads per (b, h): thread (warp w, lane l) owns TMEM lane / tile row
-// r = 32 (w % 4) + l and column half w / 4; thread 0 issues the copies and
-// the MMAs.  Every wait is bounded; a wait that runs out sets bit 1 of the
-// device status word and the CTA stops after its in-flight work.
+//   B^T Xw     (dstate x headdim, K = 128)
+// Three of them take two-term operands -- a bf16 high part plus the bf16
+// rounding of the rest -- so that the result keeps fp32-level accuracy:
+// Xw = w o X (one bf16 term would leave ~3e-3 relative error in the state),
+// the carried state H in C H^T, and the masked matrix M (one bf16 term each
+// measured 2.4e-2 output error on the full workload, above the 2e-2 bound).
+// Tiles of C, B, X come in by TMA (cp.async.bulk.tensor, 128-byte swizzle,
+// no multicast), two chunks deep.  One CTA of 512 threads per (b, h):
+// thread (warp w, lane l) owns TMEM lane / tile row r = 32 (w % 4) + l and the
+// quarter w / 4 of the columns; thread 0 issues the copies and the MMAs.
+// Every wait is bounded; a wait that runs out sets bit 1 of the device
+// status word and the CTA stops after its in-flight work.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,13 +49,8 @@ using namespace umma;
 
 constexpr int kQ = 128;         // tokens per chunk
 constexpr int kP = 64;          // head dimension (one 128-byte swizzled row of bf16)
-constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kQ * 128;  // 128 rows x 128 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
-
-// shared memory: 1024-byte aligned 16 KB tiles
-enum Tile { kC0, kC1, kB0, kB1, kX, kZ, kM0, kM1, kXh, kXl, kH, kHl, kNumTiles };
-constexpr uint32_t kSmemBytes = kNumTiles * kTileBytes + 1024;
 
 // TMEM columns (fp32): C B^T, Y_diag, Y_off, chunk state
 constexpr uint32_t kColCB = 0, kColY = 128, kColYoff = 192, kColS = 256, kTmemCols = 512;
@@ -93,285 +90,14 @@ __device__ __forceinline__ void store_piece(unsigned char *tile, int row, int pi
     *reinterpret_cast<uint4 *>(tile + sw128_offset(row, piece)) = w;
 }
 
-// The carried state's copy for C H^T: bf16(H) in `hi` and the bf16 rounding
-// of H - bf16(H) in `lo` (rows n = r, this thread's 32 of the 64 channels),
-// so that the product with C keeps ~2^-17 relative accuracy; one bf16 term
-// would put ~1e-2 of error into the output when the state is large.
-__device__ __forceinline__ void store_state_split(unsigned char *hi, unsigned char *lo, int r, int half,
-                                                  const float (&H)[32]) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float vh[8], vl[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            vh[i] = __bfloat162float(__float2bfloat16_rn(H[8 * j + i]));
-            vl[i] = H[8 * j + i] - vh[i];
-        }
-        store_piece(hi, r, 4 * half + j, vh);
-        store_piece(lo, r, 4 * half + j, vl);
-    }
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-ssd_fwd_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapZ,
-               const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapC,
-               const __grid_constant__ CUtensorMap mapO, const SsdArgs a) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                          ~static_cast<uintptr_t>(1023));
-    auto tile = [&](int i) { return sm + (uint32_t)i * kTileBytes; };
-    __shared__ uint64_t bar_ld, bar_mma1, bar_mma2, bar_mma3;
-    __shared__ uint32_t s_tmem;
-    __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[8];
-    __shared__ int s_abort;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = (warp & 3) * 32 + lane;  // tile row and TMEM lane of this thread
-    const int half = warp >> 2;            // which half of the columns it handles
-    const int64_t b = blockIdx.x / a.heads, h = blockIdx.x % a.heads;
-    const int g = (int)(h / (a.heads / a.groups));
-    const int N = a.dstate;
-    const int ntiles = N / 64;              // dstate in 64-wide tiles
-    const int ksteps = N / 16;              // MMA K steps over dstate
-    const int64_t L = a.seqlen;
-    const float Ah = a.A[h] * kLog2e;      // decays as powers of 2
-    const float Dh = a.D ? a.D[h] : 0.f;
-    const float bias = a.dt_bias ? a.dt_bias[h] : 0.f;
-    const __nv_bfloat16 *dt = static_cast<const __nv_bfloat16 *>(a.dt);
-
-    if (tid == 0) {
-        mbar_init(&bar_ld, 1);
-        mbar_init(&bar_mma1, 1);
-        mbar_init(&bar_mma2, 1);
-        mbar_init(&bar_mma3, 1);
-        mbar_fence_init();
-        s_abort = 0;
-    }
-    if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = s_tmem;
-    const uint32_t tlane = tm + ((uint32_t)((warp & 3) * 32) << 16);
-
-    // carried state: H[n = r][p = 32 half + i] in fp32 registers, a bf16 copy
-    // (rows n, 64 p per 128-byte row) in tile kH for the C H^T product
-    float H[32];
-    const bool nrow = r < N;
-    const int64_t sbase = ((b * a.heads + h) * kP + 32 * half) * N + r;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
-    store_state_split(tile(kH), tile(kHl), r, half, H);
-    fence_proxy_async();
-    __syncthreads();
-
-    auto wait = [&](uint64_t *bar, uint32_t par) {
-        if (!mbar_wait(bar, par, kWaitNs)) {
-            atomicOr(a.status, 2u);
-            s_abort = 1;
-        }
-    };
-
-    const int nchunks = (int)((L + kQ - 1) / kQ);
-    int c = 0;
-    for (; c < nchunks; ++c) {
-        const int64_t t0 = (int64_t)c * kQ;
-        const uint32_t par = (uint32_t)c & 1u;
-        // 1. the chunk's tiles of C, B (dstate in 64-wide tiles), X and Z
-        if (tid == 0) {
-            tma_store_wait_read<0>();  // the previous out tile (in kZ) has been read
-            const uint32_t bytes = (uint32_t)(2 * ntiles + 1 + (a.has_z ? 1 : 0)) * kTileBytes;
-            mbar_expect_tx(&bar_ld, bytes);
-            for (int kt = 0; kt < ntiles; ++kt) {
-                tma_load_3d(tile(kC0 + kt), &mapC, g * N + 64 * kt, (int32_t)t0, (int32_t)b, &bar_ld);
-                tma_load_3d(tile(kB0 + kt), &mapB, g * N + 64 * kt, (int32_t)t0, (int32_t)b, &bar_ld);
-            }
-            tma_load_3d(tile(kX), &mapX, (int32_t)(h * kP), (int32_t)t0, (int32_t)b, &bar_ld);
-            if (a.has_z) tma_load_3d(tile(kZ), &mapZ, (int32_t)(h * kP), (int32_t)t0, (int32_t)b, &bar_ld);
-        }
-        // 2. Delta of row r and its running sum over the chunk (rows past the
-        // sequence get Delta = 0: no decay, no input)
-        float dl = 0.f;
-        if (t0 + r < L) {
-            const float s = __bfloat162float(dt[(b * L + t0 + r) * a.heads + h]) + bias;
-            dl = a.softplus ? softplus<false>(s) : s;
-        }
-        float cum = dl;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, cum, o);
-            if (lane >= o) cum += v;
-        }
-        if (lane == 31) s_wsum[warp] = cum;
-        __syncthreads();
-        for (int w2 = 0; w2 < (warp & 3); ++w2) cum += s_wsum[(warp & ~3) + w2];
-        if (half == 0) {
-            s_dl[r] = dl;
-            s_cum[r] = cum;
-        }
-        wait(&bar_ld, par);
-        __syncthreads();
-        if (s_abort) break;
-        const float cum_end = s_cum[kQ - 1];
-
-        // 3. C B^T and C H_prev^T
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_cb = idesc_bf16(128, 128, kMajorK, kMajorK);
-            const uint32_t id_yo = idesc_bf16(128, kP, kMajorK, kMajorMN);
-            for (int k = 0; k < ksteps; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(tile(kC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(tile(kB0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
-            }
-            for (int part = 0; part < 2; ++part)
-                for (int k = 0; k < ksteps; ++k) {
-                    const uint64_t ad = desc_sw128(smem_u32(tile(kC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kHl : kH)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColYoff, ad, bd, id_yo, part > 0 || k > 0);
-                }
-            mma_commit(&bar_mma1);
-        }
-
-        // 4. Xw = w o X, w_s = exp(A (S_end - S_s)) Delta_s, as bf16 high and low parts
-        {
-            const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float x8[8], hi[8], lo[8];
-                load_piece(tile(kX), r, 4 * half + j, x8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float xw = w * x8[i];
-                    hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
-                    lo[i] = xw - hi[i];
-                }
-                store_piece(tile(kXh), r, 4 * half + j, hi);
-                store_piece(tile(kXl), r, 4 * half + j, lo);
-            }
-        }
-        fence_proxy_async();
-        __syncthreads();
-        // 5. chunk state B^T Xw (dstate x headdim; M = 128 covers dstate 64 too,
-        // the rows past dstate are not read)
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_s = idesc_bf16(128, kP, kMajorMN, kMajorMN);
-            for (int part = 0; part < 2; ++part)
-                for (int k = 0; k < kQ / 16; ++k) {
-                    const uint64_t ad = desc_sw128(smem_u32(tile(kB0)) + k * 2048, kTileBytes, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(part ? kXl : kXh)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColS, ad, bd, id_s, part > 0 || k > 0);
-                }
-            mma_commit(&bar_mma2);
-        }
-
-        // 6. M = Lmask o C B^T o Delta_s for row t = r, columns s of this half
-        wait(&bar_mma1, par);
-        fence_after_sync();
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            float cb[32];
-            tmem_ld32(tlane + kColCB + 64 * half + 32 * blk, cb);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float m8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s = 64 * half + 32 * blk + 8 * j + i;
-                    m8[i] = s <= r ? cb[8 * j + i] * ex2_approx(Ah * (cum - s_cum[s])) * s_dl[s] : 0.f;
-                }
-                store_piece(tile(kM0 + half), r, 4 * blk + j, m8);
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (s_abort) break;
-        // 7. Y_diag = M X
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_y = idesc_bf16(128, kP, kMajorK, kMajorMN);
-            for (int k = 0; k < kQ / 16; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(tile(kM0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(tile(kX)) + k * 2048, 16, 1024);
-                mma_bf16(tm + kColY, ad, bd, id_y, k > 0);
-            }
-            mma_commit(&bar_mma3);
-        }
-
-        // 8. carried state: H = exp(A S_end) H + B^T Xw; bf16 copy for the next chunk
-        wait(&bar_mma2, par);
-        fence_after_sync();
-        {
-            float sv[32];
-            tmem_ld32(tlane + kColS + 32 * half, sv);
-            tmem_wait_ld();
-            const float gdec = ex2_approx(Ah * cum_end);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
-            store_state_split(tile(kH), tile(kHl), r, half, H);
-        }
-        // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(Z), into tile kZ
-        wait(&bar_mma3, par);
-        fence_after_sync();
-        {
-            float yd[32], yo[32];
-            tmem_ld32(tlane + kColY + 32 * half, yd);
-            tmem_ld32(tlane + kColYoff + 32 * half, yo);
-            tmem_wait_ld();
-            const float et = ex2_approx(Ah * cum);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float x8[8], z8[8], o8[8];
-                load_piece(tile(kX), r, 4 * half + j, x8);
-                if (a.has_z) load_piece(tile(kZ), r, 4 * half + j, z8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float y = fmaf(et, yo[8 * j + i], yd[8 * j + i]);
-                    y = fmaf(Dh, x8[i], y);
-                    o8[i] = a.has_z ? y * silu<false>(z8[i]) : y;
-                }
-                store_piece(tile(kZ), r, 4 * half + j, o8);
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (s_abort) break;
-        if (tid == 0) {
-            tma_store_3d(&mapO, (int32_t)(h * kP), (int32_t)t0, (int32_t)b, tile(kZ));
-            tma_store_commit();
-        }
-    }
-    if (s_abort) {
-        // let whatever was issued for chunk c finish (bounded), so that no copy
-        // or MMA still targets this CTA's shared or tensor memory
-        const uint32_t par = (uint32_t)c & 1u;
-        (void)mbar_wait(&bar_ld, par, kWaitNs);
-        (void)mbar_wait(&bar_mma1, par, kWaitNs);
-        (void)mbar_wait(&bar_mma2, par, kWaitNs);
-        (void)mbar_wait(&bar_mma3, par, kWaitNs);
-    } else if (a.state && nrow) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) a.state[sbase + (int64_t)i * N] = H[i];
-    }
-    if (tid == 0) tma_store_wait_all<0>();
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, kTmemCols);
-}
-
 // ---------------------------------------------------------------------------
-// Pipelined form: the tiles of chunk c + 1 (C, B, X; two stages) are copied
-// while chunk c computes, the masked intra-chunk matrix M stays in tensor
-// memory as the A operand of M X (no shared-memory round trip), and z / out
-// move between registers and global memory directly, so that the double
-// buffers fit in shared memory.  Inside a chunk the products and the
-// element-wise phases overlap: C B^T and C H^T run while the threads form
-// w o X; B^T (w o X) runs while they mask C B^T; M X runs while they update
-// the carried state.
+// The tiles of chunk c + 1 (C, B, X; two stages) are copied while chunk c
+// computes, the masked intra-chunk matrix M stays in tensor memory as the A
+// operand of M X (no shared-memory round trip), and z / out move between
+// registers and global memory directly, so that the double buffers fit in
+// shared memory.  Inside a chunk the products and the element-wise phases
+// overlap: C B^T and C H^T run while the threads form w o X; B^T (w o X)
+// runs while they mask C B^T; M X runs while they update the carried state.
 enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kHl2,
              kNumTiles2 };
 constexpr uint32_t kSmemBytes2 = kNumTiles2 * kTileBytes + 1024;
@@ -700,13 +426,6 @@ namespace ssm {
 
 namespace {
 
-// 1: the pipelined kernel (double-buffered tiles, M in tensor memory);
-// 0: the plain one (one chunk at a time, every tile in shared memory).
-#ifndef SSM_SSD_PIPELINED
-#define SSM_SSD_PIPELINED 1
-#endif
-constexpr bool kSsdPipelined = SSM_SSD_PIPELINED != 0;
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -753,11 +472,10 @@ bool ssd_fwd_supported(const SsdFwdArgs &a) {
 
 cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     if (!ssd_fwd_supported(a)) return cudaErrorNotSupported;
-    CUtensorMap mx, mz, mb, mc, mo;
+    CUtensorMap mx, mb, mc;
     const int64_t hp = a.heads * a.headdim, gn = a.groups * a.dstate;
     if (!encode_btw(&mx, a.x, a.batch, a.seqlen, hp) || !encode_btw(&mb, a.B, a.batch, a.seqlen, gn) ||
-        !encode_btw(&mc, a.C, a.batch, a.seqlen, gn) || !encode_btw(&mo, a.out, a.batch, a.seqlen, hp) ||
-        !encode_btw(&mz, a.z ? a.z : a.x, a.batch, a.seqlen, hp))
+        !encode_btw(&mc, a.C, a.batch, a.seqlen, gn))
         return cudaErrorInvalidValue;
     SsdArgs k{};
     k.dt = a.dt;
@@ -779,20 +497,15 @@ cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (!configured[dev & 63]) {
-        e = cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kSmemBytes2);
+        e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes2);
         if (e != cudaSuccess) return e;
         configured[dev & 63] = true;
     }
     const int64_t grid = a.batch * a.heads;
     if (grid > 2147483647LL) return cudaErrorInvalidConfiguration;
-    if (kSsdPipelined)
-        ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads2, kSmemBytes2, st>>>(
-            mx, mb, mc, static_cast<const __nv_bfloat16 *>(a.z), static_cast<__nv_bfloat16 *>(a.out), k);
-    else
-        ssd_fwd_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mx, mz, mb, mc, mo, k);
+    ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads2, kSmemBytes2, st>>>(
+        mx, mb, mc, static_cast<const __nv_bfloat16 *>(a.z), static_cast<__nv_bfloat16 *>(a.out), k);
     return cudaGetLastError();
 }
 

@@ -167,3 +167,39 @@ def test_bwd_empty_sizes_without_outputs_are_noops(b):
                 dA=None, dB=None, dC=None)
     for dims in [(0, 16, 8, 16), (2, 0, 8, 16), (2, 16, 0, 16)]:
         assert _bwd(b, dims, **none) == b.SSM_OK
+
+
+def _ssd(b, dims, io=1, ptrs=None, softplus=1):
+    # ptrs: x, dt, A, B, C, D, z, dt_bias, out, state (fake, never dereferenced)
+    p = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=None, z=None, bias=None,
+             out=0x60000, state=None)
+    p.update(ptrs or {})
+    return b.lib.ssm_ssd_scan_fwd(b.SSMSsdDims(*dims), io, p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"],
+                                  p["z"], p["bias"], softplus, p["out"], p["state"], None)
+
+
+def test_ssd_argument_validation(b):
+    # (batch, seqlen, heads, headdim, groups, dstate)
+    ok = (2, 256, 4, 64, 2, 128)
+    assert _ssd(b, ok, io=7) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, ok, io=0) == b.SSM_ERR_UNSUPPORTED          # float32: the tensor-core path is bf16
+    assert b"bf16" in b.lib.ssm_last_error()
+    assert _ssd(b, (2, 256, 4, 32, 2, 128)) == b.SSM_ERR_UNSUPPORTED   # headdim 32
+    assert _ssd(b, (2, 256, 4, 64, 2, 96)) == b.SSM_ERR_UNSUPPORTED   # dstate 96
+    assert _ssd(b, (2, 256, 4, 64, 3, 128)) == b.SSM_ERR_INVALID_ARG  # heads not a multiple of groups
+    assert _ssd(b, (2, 256, 4, 64, 0, 128)) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, (2, -1, 4, 64, 2, 128)) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, ok, softplus=2) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, ok, ptrs=dict(dt=None)) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, ok, ptrs=dict(out=None)) == b.SSM_ERR_INVALID_ARG
+    assert _ssd(b, ok, ptrs=dict(dt=0x20001)) == b.SSM_ERR_INVALID_ARG   # dt not aligned to bf16
+    assert _ssd(b, ok, ptrs=dict(x=0x10008)) == b.SSM_ERR_UNSUPPORTED    # x not 16-byte aligned (TMA)
+    assert _ssd(b, ok, ptrs=dict(z=0x70004)) == b.SSM_ERR_UNSUPPORTED
+    # empty problems: nothing to compute, nothing enqueued
+    for dims in [(0, 256, 4, 64, 2, 128), (2, 0, 4, 64, 2, 128), (2, 256, 0, 64, 2, 128)]:
+        assert _ssd(b, dims, ptrs=dict(x=None, out=None)) == b.SSM_OK
+
+
+def test_build_info(b):
+    info = b.build_info()
+    assert 0 <= info["sfu_decays_per_16"] <= 16 and info["sfu_decays_per_16"] % 4 == 0
