@@ -442,9 +442,12 @@ def run_scan(args, rank, world, dev):
 
     e2e = None
     if cfg.elements <= 1 << 28:
-        # end to end through the public call with host buffers: pinned host
-        # inputs copied in, the scan, the output and the final state copied
-        # back, every step
+        # End to end through the public call with host buffers: every step
+        # copies this rank's pinned host inputs in, scans, and copies the
+        # output and the final state back.  The batch rows are independent
+        # scans, so the step is pipelined by row as a user would run it: row
+        # b + 1's host->device copy (one stream) overlaps row b's scan (the
+        # compute stream) and row b - 1's device->host copy (a third stream).
         host = {k: v.cpu().pin_memory() for k, v in d.items()}
         host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         host_state = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
@@ -452,19 +455,39 @@ def run_scan(args, rank, world, dev):
         h2d = sum(v.numel() * v.element_size() for v in host.values()) + host_state0.numel() * 4
         d2h = host_out.numel() * host_out.element_size() + host_state.numel() * 4
         e2e_steps = max(3, min(args.steps, 20))
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        rows = cfg.batch
+        ev_in = [torch.cuda.Event() for _ in range(rows)]
+        ev_done = [torch.cuda.Event() for _ in range(rows)]
 
         def e2e_step():
-            for k in d:
-                d[k].copy_(host[k], non_blocking=True)
-            state.copy_(host_state0, non_blocking=True)
-            lib.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                                   delta_bias=d["delta_bias"], out=out, last_state=state, stream=stream)
-            host_out.copy_(out, non_blocking=True)
-            host_state.copy_(state, non_blocking=True)
+            s_in.wait_stream(stream)  # the previous step is done with the buffers
+            with torch.cuda.stream(s_in):
+                for k in ("A", "D", "delta_bias"):
+                    d[k].copy_(host[k], non_blocking=True)
+                for b in range(rows):
+                    for k in I.SEQ_NAMES:
+                        d[k][b].copy_(host[k][b], non_blocking=True)
+                    state[b].copy_(host_state0[b], non_blocking=True)
+                    ev_in[b].record(s_in)
+            for b in range(rows):
+                stream.wait_event(ev_in[b])
+                sl = slice(b, b + 1)
+                lib.selective_scan_fwd(d["u"][sl], d["delta"][sl], d["A"], d["B"][sl], d["C"][sl], D=d["D"],
+                                       z=d["z"][sl], delta_bias=d["delta_bias"], out=out[sl],
+                                       last_state=state[sl], stream=stream)
+                ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                for b in range(rows):
+                    s_out.wait_event(ev_done[b])
+                    host_out[b].copy_(out[b], non_blocking=True)
+                    host_state[b].copy_(state[b], non_blocking=True)
+            stream.wait_stream(s_out)  # the step ends when its results are on the host
 
         e2e_ms = _e2e(e2e_step, e2e_steps, stream, dev, world)
         e2e = {"value": gcfg.elements / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
-               "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "steps": e2e_steps}
+               "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "steps": e2e_steps,
+               "pipeline": "by batch row: copy in / scan / copy out on three streams"}
 
     if rank == 0:
         peaks = measured_peaks()

@@ -14,13 +14,14 @@
 // holding complex states [q NS, q NS + NS); a block of 128 threads covers 32
 // channels of one batch row; B and C of a chunk of 32 steps are widened to
 // fp32 pairs in shared memory; u, delta, z of four steps are loaded ahead of
-// their arithmetic.  Per state and step the decay takes one exponential (SFU
-// in the fast tier) and a sine and cosine of Delta Im A.  The fp32 tier calls
-// sincosf.  The fast tier reduces the angle to [-pi, pi] (Cody and Waite: 2 pi
-// split into a 9-bit head and a tail) and uses the Taylor series below 1/4,
-// where the SFU sine's absolute error (~4e-7) would be a large relative phase
-// error that adds up over a state's memory of ~1/(Delta |Re A|) steps, and the
-// SFU sine and cosine above it.
+// their arithmetic.  Per state and step the decay takes one exponential and a
+// sine and cosine of Delta Im A.  The fp32 tier calls sincosf.  The fast tier
+// reduces the angle to [-pi, pi] (round to nearest by the 1.5 2^23 addition,
+// then Cody and Waite's two-part 2 pi) and takes the SFU's sine and cosine,
+// whose absolute error (<= 2^-21.4 on [-pi, pi]) is a phase error of that
+// size per step; over a state's memory of ~1/(Delta |Re A|) steps it stays
+// far inside the bf16 tier's 1e-3 state bound.  The complex products run on
+// fp32 pairs (f32x2): (re, im) of a state is one register pair.
 #include "scan_kernels.cuh"
 
 namespace ssm {
@@ -42,22 +43,11 @@ __device__ __forceinline__ void phase(float x, float &s, float &c) {
         sincosf(x, &s, &c);
         return;
     }
-    const float k = rintf(x * kInvTwoPi);
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23: x * (1 / 2 pi) + kRound - kRound = rint(x / 2 pi)
+    const float k = fmaf(x, kInvTwoPi, kRound) - kRound;
     const float r = fmaf(-k, kTwoPiLo, fmaf(-k, kTwoPiHi, x));
-    const float r2 = r * r;
-    // sin r = r (1 - r^2/6 (1 - r^2/20 (1 - r^2/42))), cos r = 1 - r^2/2 (1 - r^2/12
-    // (1 - r^2/30 (1 - r^2/56))): truncation below 1e-10 for |r| < 1/4
-    const float ps = r * fmaf(-r2 * (1.f / 6.f), fmaf(-r2 * (1.f / 20.f), fmaf(-r2, 1.f / 42.f, 1.f), 1.f), 1.f);
-    const float pc = fmaf(-r2 * 0.5f,
-                          fmaf(-r2 * (1.f / 12.f), fmaf(-r2 * (1.f / 30.f), fmaf(-r2, 1.f / 56.f, 1.f), 1.f), 1.f),
-                          1.f);
-    float ms, mc;
-    __sincosf(r, &ms, &mc);
-    const bool small = fabsf(r) < 0.25f;
-    s = small ? ps : ms;
-    c = small ? pc : mc;
+    __sincosf(r, &s, &c);
 }
-
 
 template <typename IO, int NS, bool PRECISE>
 __global__ void __launch_bounds__(kBlock)
@@ -116,19 +106,42 @@ scan_fwd_complex_kernel(const ScanArgs args) {
         auto step = [&](int r, float uv, float s, float zv) {
             const float dl = args.softplus ? softplus<PRECISE>(s) : s;
             const float du = dl * uv;
-            float yp = 0.f;
+            float yp;
+            if (PRECISE) {
+                yp = 0.f;
 #pragma unroll
-            for (int i = 0; i < NS; ++i) {
-                const float2 bv = sB[r][q * NS + i], cv = sC[r][q * NS + i];
-                const float e = decay<PRECISE>(dl, are[i]);
-                float sn, cs;
-                phase<PRECISE>(dl * aim[i], sn, cs);
-                const float ar = e * cs, ai = e * sn;
-                const float nr = fmaf(ar, hr[i], fmaf(-ai, hi[i], du * bv.x));
-                const float ni = fmaf(ar, hi[i], fmaf(ai, hr[i], du * bv.y));
-                hr[i] = nr;
-                hi[i] = ni;
-                yp = fmaf(cv.x, nr, fmaf(-cv.y, ni, yp));
+                for (int i = 0; i < NS; ++i) {
+                    const float2 bv = sB[r][q * NS + i], cv = sC[r][q * NS + i];
+                    const float e = decay<PRECISE>(dl, are[i]);
+                    float sn, cs;
+                    phase<PRECISE>(dl * aim[i], sn, cs);
+                    const float ar = e * cs, ai = e * sn;
+                    const float nr = fmaf(ar, hr[i], fmaf(-ai, hi[i], du * bv.x));
+                    const float ni = fmaf(ar, hi[i], fmaf(ai, hr[i], du * bv.y));
+                    hr[i] = nr;
+                    hi[i] = ni;
+                    yp = fmaf(cv.x, nr, fmaf(-cv.y, ni, yp));
+                }
+            } else {
+                // states as (re, im) pairs: h <- (ar, ar) h + (-ai, ai) (im, re) + du (br, bi);
+                // readout Re(C h) = cr hr - ci hi summed on a pair
+                const float2 du2 = make_float2(du, du);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < NS; ++i) {
+                    const float2 bv = sB[r][q * NS + i], cv = sC[r][q * NS + i];
+                    const float e = ex2_approx(dl * are[i]);
+                    float sn, cs;
+                    phase<false>(dl * aim[i], sn, cs);
+                    const float2 h2 = make_float2(hr[i], hi[i]);
+                    float2 t = mul2(du2, bv);
+                    t = fma2(make_float2(-e * sn, e * sn), make_float2(hi[i], hr[i]), t);
+                    t = fma2(make_float2(e * cs, e * cs), h2, t);
+                    hr[i] = t.x;
+                    hi[i] = t.y;
+                    acc = fma2(make_float2(cv.x, -cv.y), t, acc);
+                }
+                yp = acc.x + acc.y;
             }
             float y = group_sum<G>(yp);
             if (q == 0) {
