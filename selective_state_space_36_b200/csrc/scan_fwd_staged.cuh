@@ -125,18 +125,19 @@ __device__ __forceinline__ void store_vals(IO *p, const float (&v)[CPL]) {
 template <int TPB, int MODE>
 __device__ __forceinline__ void vblock_sync(int vb) {
     if (TPB == 32) __syncwarp();
-    else if (MODE != kFull) __syncthreads();
+    else if (MODE != kFull && MODE != kCkpt) __syncthreads();
     else asm volatile("bar.sync %0, %1;" ::"r"(vb + 1), "n"(TPB) : "memory");
 }
 
-// Threads a CTA of the staged kernel may have.  Only the one-pass mode packs
-// several virtual blocks per CTA: up to 512 threads for layouts whose lanes
-// hold at most 8 states (they stay below 128 registers), else 256, so that
-// ptxas may give every thread up to 255 registers.  The other modes launch
-// one 128-thread block per unit.
+// Threads a CTA of the staged kernel may have.  The one-pass modes (the scan
+// and the backward's checkpoint pass) pack several virtual blocks per CTA: up
+// to 512 threads for layouts whose lanes hold at most 8 states (they stay
+// below 128 registers), else 256, so that ptxas may give every thread up to
+// 255 registers.  The split passes launch one 128-thread block per unit.
 template <int G, int NS, int CPL, int MODE>
 struct StagedMaxThreads {
-    static constexpr int value = MODE != kFull ? kBlock : (G > 1 && NS * CPL <= 8 ? 512 : 256);
+    static constexpr int value =
+        (MODE != kFull && MODE != kCkpt) ? kBlock : (G > 1 && NS * CPL <= 8 ? 512 : 256);
 };
 
 template <typename IO, int NS, int G, int CPL, bool PRECISE, int MODE, bool ZOH, int TPB>
@@ -457,7 +458,7 @@ inline cudaError_t launch_mode(ScanArgs a, int64_t units, unsigned nseg, cudaStr
     if (G == 4) vmax = 1;  // one block per unit measured faster for four lanes (see SSM_VB_THREADS_G*)
     if (TPB > 32 && vmax > 15) vmax = 15;  // hardware barriers 1..15
     if ((size_t)vmax * Lay::SMEM > (size_t)optin) vmax = (int)((size_t)optin / Lay::SMEM);
-    if (MODE != kFull) vmax = 1;
+    if (MODE != kFull && MODE != kCkpt) vmax = 1;
     if (vmax < 1) return cudaErrorInvalidConfiguration;
     // the shared-memory opt-in is a per-device function attribute: set it once per device
     static std::atomic<unsigned long long> configured{0};
@@ -496,7 +497,8 @@ inline cudaError_t launch_z(const ScanArgs &a, int variant, cudaStream_t st) {
         return launch_mode<IO, NS, G, CPL, kFull, ZOH, TPBS>(a, a.batch * ((a.dim + CPBS - 1) / CPBS), 1, st);
     if (variant == kVariantCkpt) {
         if (CPL != 1 || ZOH) return cudaErrorInvalidConfiguration;
-        return launch_mode<IO, NS, G, 1, kCkpt, false, kBlock>(a, units, 1, st);
+        constexpr int CPBC = StagedLayout<IO, NS, G, 1, TPBS>::CPB;
+        return launch_mode<IO, NS, G, 1, kCkpt, false, TPBS>(a, a.batch * ((a.dim + CPBC - 1) / CPBC), 1, st);
     }
     cudaError_t e = launch_mode<IO, NS, G, CPL, kSegAgg, ZOH, kBlock>(a, units, (unsigned)(a.nseg - 1), st);
     if (e != cudaSuccess) return e;
