@@ -13,8 +13,8 @@
 // Layout as the generic real kernel: G = 4 lanes share a channel, lane q
 // holding complex states [q NS, q NS + NS); a block of 128 threads covers 32
 // channels of one batch row; B and C of a chunk of 32 steps are widened to
-// fp32 pairs in shared memory; u, delta, z of four steps are loaded ahead of
-// their arithmetic.  Per state and step the decay takes one exponential and a
+// fp32 pairs in shared memory; u, delta, z of kCAhead steps are loaded ahead
+// of their arithmetic.  Per state and step the decay takes one exponential and a
 // sine and cosine of Delta Im A.  The fp32 tier calls sincosf.  The fast tier
 // reduces the angle to [-pi, pi] (round to nearest by the 1.5 2^23 addition,
 // then Cody and Waite's two-part 2 pi) and takes the SFU's sine and cosine,
@@ -31,7 +31,13 @@ namespace {
 constexpr int kCG = 4;                 // lanes per channel
 constexpr int kCCPB = kBlock / kCG;    // channels per block
 constexpr int kCChunk = 32;            // steps of B, C staged at once
-constexpr int kCAhead = 4;             // steps whose u, delta, z are loaded together
+// Steps whose u, delta, z are loaded together, ahead of their arithmetic:
+// with 4 the loads' latency was exposed (ncu: long-scoreboard stalls 3.55 per
+// issued instruction at the 130M layer).
+#ifndef SSM_COMPLEX_AHEAD
+#define SSM_COMPLEX_AHEAD 16
+#endif
+constexpr int kCAhead = SSM_COMPLEX_AHEAD;
 
 constexpr float kInvTwoPi = 0.15915494309189535f;
 constexpr float kTwoPiHi = 6.28125f;               // 9 significant bits: k * kTwoPiHi is exact
