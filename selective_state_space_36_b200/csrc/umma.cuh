@@ -195,12 +195,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 // Waits for the phase with the given parity to complete, for at most
 // `limit_ns` nanoseconds of the global timer; false if the wait ran out.
+// The timer is read every 64 polls only: many threads may be waiting.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_timer_ns() - t0 > limit_ns) return false;
-    return true;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // --------------------------------------------------------------------- TMA
