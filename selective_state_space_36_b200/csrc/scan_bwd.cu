@@ -283,48 +283,52 @@ scan_bwd_kernel(const ScanBwdArgs args) {
 // The first pass is the staged forward kernel in checkpoint mode, which
 // stores the state entering every KC-th step.  This kernel walks the chunks of
 // T steps of its (batch row, 32-channel) tile from the last to the first; the
-// copies of the next chunk (u, delta, z, dout tiles and the B, C rows) are in
-// flight while the current one is processed.  Within a chunk it takes the
-// sub-chunks of KC steps from last to first:
+// copies of the next two chunks (u, delta, z, dout tiles and the B, C rows)
+// are in flight while the current one is processed.  Within a chunk it takes
+// the sub-chunks of KC steps from last to first:
 //   scalars    lane q of a channel's group of 4 computes Delta, Delta u,
 //              sigmoid(z) and dy = dout silu(z) for steps k0 + 4 j + q and the
 //              values travel to the other lanes by shuffles;
-//   recompute  from the checkpoint, the KC states and decays of this lane's
-//              4 states (kept in registers);
-//   reverse    the adjoint recurrence over the KC steps; the per-step partial
-//              sums of dDelta, sum_n lambda B and y are reduce-scattered back
-//              to the owning lanes, which finish du, ddelta, dz and write them
-//              into the consumed input rows of the tile (u, delta, z) -- the
-//              chunk's gradients then leave in 16-byte pieces;
-//   dB, dC     as in the generic kernel: a [KC][channel][state] tile in shared
-//              memory, summed over the 32 channels and added with vector
-//              atomics.
-// Thread groups that share the channel sum of the dB/dC tile (1: 64 threads
-// sum all 32 channels; 2: all 128 threads, 16 channels each, two atomic adds
-// per output -- measured 13 % slower at the 1.4B-layer shape: twice the
-// global atomics and more register spills).
-#ifndef SSM_BWD_RED_SPLIT
-#define SSM_BWD_RED_SPLIT 1
+//   recompute  from the checkpoint, the KC states of this lane's 4 states
+//              (kept in registers; the decays are recomputed in the reverse
+//              sweep rather than kept, which leaves room for four blocks per
+//              SM);
+//   reverse    the adjoint recurrence over the KC steps, G steps at a time;
+//              after each group of G steps the per-step partial sums of
+//              dDelta, sum_n lambda B and y are reduce-scattered to the owning
+//              lanes, which finish du, ddelta, dz and write them into the
+//              consumed input rows of the tile (u, delta, z) -- the chunk's
+//              gradients then leave in 16-byte pieces;
+//   dB, dC     a [KC][channel][state] tile in shared memory, summed over the
+//              32 channels by all 128 threads (two threads per output quad,
+//              16 channels each, joined by a shuffle) and added to global
+//              memory with one vector atomic per quad.
+#ifndef SSM_BWD_MIN_BLOCKS_BF16
+#define SSM_BWD_MIN_BLOCKS_BF16 4
 #endif
 
 template <typename IO>
 struct BwdStagedLayout {
     static constexpr int G = 4, NS = 4, NSP = 16, CPB = kBlock / G;
-    static constexpr int T = sizeof(IO) == 2 ? 32 : 16;   // steps per staged chunk
+    static constexpr int T = 16;                          // steps per staged chunk
     static constexpr int KC = kCkptEvery;                 // steps per sub-chunk (checkpoint spacing)
-    static constexpr int S = 2;                           // pipeline stages
-    static constexpr int ROW = CPB + 32 / (int)sizeof(IO);  // tile row, padded by 32 bytes
+    static constexpr int S = 3;                           // pipeline stages
+    static constexpr int ROW = CPB + 8;                   // tile row, padded against bank conflicts
     static constexpr int TILE = T * ROW;
     static constexpr int RAW = T * NSP;                   // raw B or C rows (elements)
     static constexpr size_t STAGE_BYTES = (4 * (size_t)TILE + 2 * RAW) * sizeof(IO);
     static constexpr size_t BC_BYTES = 2 * (size_t)T * NSP * sizeof(float);
     // reduction tile [2 (dC, dB)][KC][CPB][NSP]; each step's slab is padded by
-    // 16 floats so that the reading threads of a quarter-warp (4 state
-    // columns x 2 steps) fall in different banks
+    // 16 floats
     static constexpr int KSTRIDE = CPB * NSP + 16;
     static constexpr size_t RED_BYTES = 2 * (size_t)KC * KSTRIDE * sizeof(float);
     static constexpr size_t SMEM = S * STAGE_BYTES + BC_BYTES + RED_BYTES;
+    // blocks per SM the kernel is compiled for: four for the bf16 tier
+    // (65536 / (128 x 4) = 128 registers per thread, 53 KB of shared memory
+    // per block), three for fp32 I/O (larger tiles)
+    static constexpr int MIN_BLOCKS = sizeof(IO) == 2 ? SSM_BWD_MIN_BLOCKS_BF16 : 3;
     static_assert(T % KC == 0 && KC % G == 0, "chunks hold whole sub-chunks of whole step groups");
+    static_assert((ROW * sizeof(IO)) % 16 == 0, "tile rows leave in 16-byte pieces");
 };
 
 template <int K, int G>
@@ -337,7 +341,7 @@ __device__ __forceinline__ void exchange_one(const float (&own)[K / G], float (&
 }
 
 template <typename IO, bool PRECISE>
-__global__ void __launch_bounds__(kBlock, 3)
+__global__ void __launch_bounds__(kBlock, BwdStagedLayout<IO>::MIN_BLOCKS)
 scan_bwd_staged_kernel(const ScanBwdArgs args) {
     using io = io_traits<IO>;
     using Lay = BwdStagedLayout<IO>;
@@ -401,8 +405,9 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
         }
     };
 
-    // per-lane constants: A pairs (scaled for the decay, and as given)
-    float2 Aw2[NS / 2], An2[NS / 2];
+    // per-lane constants: A pairs, scaled for the decay (the fast tier's
+    // log2(e) factor comes off the dDelta sums once per step, below)
+    float2 Aw2[NS / 2];
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) {
         float v[2];
@@ -411,9 +416,9 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             const int n = q * NS + 2 * p + e;
             v[e] = (active && n < N) ? args.A[d * N + n] : 0.f;
         }
-        An2[p] = make_float2(v[0], v[1]);
         Aw2[p] = make_float2(scale_A<PRECISE>(v[0]), scale_A<PRECISE>(v[1]));
     }
+    constexpr float kAUnscale = PRECISE ? 1.f : kLn2;
     const float bias = (active && args.bias) ? args.bias[d] : 0.f;
     const float dskip = (active && args.Dskip) ? args.Dskip[d] : 0.f;
     const float *ck_lane = args.ckpt + (b * nck * Dm + d) * N + q * NS;
@@ -422,16 +427,6 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) { lam2[p] = make_float2(0.f, 0.f); dA2[p] = make_float2(0.f, 0.f); }
     float dD_acc = 0.f, dbias_acc = 0.f;
-    // the checkpoint of the first sub-chunk processed (the last one in time)
-    float2 hc_next[NS / 2];
-    {
-        const float *cp = ck_lane + (nck - 1) * Dm * N;
-#pragma unroll
-        for (int p = 0; p < NS / 2; ++p) {
-            const int n = q * NS + 2 * p;
-            hc_next[p] = make_float2((active && n < N) ? cp[2 * p] : 0.f, (active && n + 1 < N) ? cp[2 * p + 1] : 0.f);
-        }
-    }
 
 #pragma unroll
     for (int o = 0; o < S - 1; ++o) {
@@ -439,10 +434,12 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
         cp_async_commit();
     }
     for (int o = 0; o < nchunks; ++o) {
+        cp_async_wait<S - 2>();
+        // chunk o has landed for every thread, and every thread is done with
+        // the stage that chunk o + S - 1 goes to (it held chunk o - 1)
+        __syncthreads();
         if (o + S - 1 < nchunks) issue(o + S - 1);
         cp_async_commit();
-        cp_async_wait<S - 1>();
-        __syncthreads();
         const int64_t tc = (int64_t)(nchunks - 1 - o) * T;
         const int rows = (int)(L - tc < T ? L - tc : T);
         IO *st = stage_ptr(o % S);
@@ -476,28 +473,24 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
         // of this chunk; the constant T for full chunks).
         auto sub_chunk = [&](const int k0, const int nrows) {
             const int64_t t0 = tc + k0;
+            // the state entering the sub-chunk, loaded first so that the step
+            // scalars below cover its latency
             float2 hc[NS / 2];
-#pragma unroll
-            for (int p = 0; p < NS / 2; ++p) hc[p] = hc_next[p];
-            if (t0 >= KC) {  // prefetch the checkpoint of the sub-chunk processed next
-                const float *cp = ck_lane + (t0 / KC - 1) * Dm * N;
+            {
+                const float *cp = ck_lane + (t0 / KC) * Dm * N;
 #pragma unroll
                 for (int p = 0; p < NS / 2; ++p) {
                     const int n = q * NS + 2 * p;
-                    hc_next[p] = make_float2((active && n < N) ? cp[2 * p] : 0.f,
-                                             (active && n + 1 < N) ? cp[2 * p + 1] : 0.f);
+                    hc[p] = make_float2((active && n < N) ? __ldcs(cp + 2 * p) : 0.f,
+                                        (active && n + 1 < N) ? __ldcs(cp + 2 * p + 1) : 0.f);
                 }
             }
-            // ---- per-step scalars of the owned steps k0 + j G + q
-            float uo[KG], so[KG], zo[KG], go[KG], szo[KG], dlo[KG], duo[KG], dyo[KG];
+            // ---- per-step scalars of the owned steps k0 + j G + q (the raw
+            // inputs are read again from the tile where the end of the
+            // sub-chunk needs them)
+            float so[KG], szo[KG], dlo[KG], duo[KG], dyo[KG];
 #pragma unroll
-            for (int j = 0; j < KG; ++j) {
-                const int rr = k0 + j * G;
-                uo[j] = io::load_smem(su + rr * ROW);
-                so[j] = io::load_smem(sd + rr * ROW) + bias;
-                zo[j] = pz ? io::load_smem(sz + rr * ROW) : 0.f;
-                go[j] = io::load_smem(sg + rr * ROW);
-            }
+            for (int j = 0; j < KG; ++j) so[j] = io::load_smem(sd + (k0 + j * G) * ROW) + bias;
             if (args.softplus) {
                 if (!PRECISE && KG % 2 == 0) {
 #pragma unroll
@@ -516,23 +509,25 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             }
 #pragma unroll
             for (int j = 0; j < KG; ++j) {
-                if (k0 + j * G + q >= nrows || !active) { dlo[j] = 0.f; go[j] = 0.f; }
-                duo[j] = dlo[j] * uo[j];
+                const int rr = k0 + j * G;
+                const float uo = io::load_smem(su + rr * ROW);
+                float go = io::load_smem(sg + rr * ROW);
+                if (rr + q >= nrows || !active) { dlo[j] = 0.f; go = 0.f; }
+                duo[j] = dlo[j] * uo;
                 if (pz) {
-                    szo[j] = sigmoid_of<PRECISE>(zo[j]);
-                    dyo[j] = go[j] * zo[j] * szo[j];
+                    const float zo = io::load_smem(sz + rr * ROW);
+                    szo[j] = sigmoid_of<PRECISE>(zo);
+                    dyo[j] = go * zo * szo[j];
                 } else {
                     szo[j] = 0.f;
-                    dyo[j] = go[j];
+                    dyo[j] = go;
                 }
             }
-            float dl[KC], du[KC], dy[KC];
-            exchange_steps<KC, G>(dlo, duo, dl, du);
-            exchange_one<KC, G>(dyo, dy);
-
-            // ---- recompute the sub-chunk's states and decays
-            float2 hs[KC][NS / 2], as[KC][NS / 2];
+            // ---- recompute the sub-chunk's states
+            float2 hs[KC][NS / 2];
             {
+                float dl[KC], du[KC];
+                exchange_steps<KC, G>(dlo, duo, dl, du);
                 float2 h2[NS / 2];
 #pragma unroll
                 for (int p = 0; p < NS / 2; ++p) h2[p] = hc[p];
@@ -547,81 +542,103 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                         const float2 a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
                         h2[p] = fma2(a2, h2[p], mul2(u2, b2));
                         hs[k][p] = h2[p];
-                        as[k][p] = a2;
                     }
                 }
             }
 
-            // ---- adjoint recurrence, last step first
-            float ddl_p[KC], dub_p[KC], y_p[KC];
+            // ---- adjoint recurrence, last step first, G steps at a time (the
+            // step scalars come from their owning lanes again, rather than
+            // being held through the sweep)
+            const unsigned gbase = (threadIdx.x & 31u) & ~(unsigned)(G - 1);
+            const unsigned gmask = ((1u << G) - 1u) << gbase;
 #pragma unroll
-            for (int k = KC - 1; k >= 0; --k) {
-                const float4 bv = *reinterpret_cast<const float4 *>(fBq + (k0 + k) * NSP);
-                const float4 cv = *reinterpret_cast<const float4 *>(fCq + (k0 + k) * NSP);
-                const float2 dy2 = make_float2(dy[k], dy[k]), dl2 = make_float2(dl[k], dl[k]);
-                const float2 du2 = make_float2(du[k], du[k]);
-                float2 accy = make_float2(0.f, 0.f), accd = accy, accb = accy, pc[NS / 2], pb[NS / 2];
+            for (int jg = KG - 1; jg >= 0; --jg) {
+                float ddl_p[G], dub_p[G], y_p[G];
 #pragma unroll
-                for (int p = 0; p < NS / 2; ++p) {
-                    const float2 b2 = p ? make_float2(bv.z, bv.w) : make_float2(bv.x, bv.y);
-                    const float2 c2 = p ? make_float2(cv.z, cv.w) : make_float2(cv.x, cv.y);
-                    const float2 hprev = k > 0 ? hs[k - 1][p] : hc[p];
-                    lam2[p] = fma2(dy2, c2, lam2[p]);
-                    pc[p] = mul2(dy2, hs[k][p]);
-                    pb[p] = mul2(lam2[p], du2);
-                    accy = fma2(c2, hs[k][p], accy);
-                    accb = fma2(lam2[p], b2, accb);
-                    const float2 la = mul2(lam2[p], as[k][p]);
-                    const float2 ga = mul2(la, hprev);
-                    accd = fma2(ga, An2[p], accd);
-                    dA2[p] = fma2(ga, dl2, dA2[p]);
-                    lam2[p] = la;
+                for (int i = G - 1; i >= 0; --i) {
+                    const int k = jg * G + i;
+                    const float4 bv = *reinterpret_cast<const float4 *>(fBq + (k0 + k) * NSP);
+                    const float4 cv = *reinterpret_cast<const float4 *>(fCq + (k0 + k) * NSP);
+                    const float dyk = __shfl_sync(gmask, dyo[jg], gbase + i);
+                    const float dlk = __shfl_sync(gmask, dlo[jg], gbase + i);
+                    const float duk = __shfl_sync(gmask, duo[jg], gbase + i);
+                    const float2 dy2 = make_float2(dyk, dyk), dl2 = make_float2(dlk, dlk);
+                    const float2 du2 = make_float2(duk, duk);
+                    float2 accy = make_float2(0.f, 0.f), accd = accy, accb = accy, pc[NS / 2], pb[NS / 2];
+#pragma unroll
+                    for (int p = 0; p < NS / 2; ++p) {
+                        const float2 b2 = p ? make_float2(bv.z, bv.w) : make_float2(bv.x, bv.y);
+                        const float2 c2 = p ? make_float2(cv.z, cv.w) : make_float2(cv.x, cv.y);
+                        const float2 hprev = k > 0 ? hs[k - 1][p] : hc[p];
+                        // the decay of step k, as the recomputation took it
+                        float2 a2;
+                        if (PRECISE) {
+                            const float2 x2 = mul2(dl2, Aw2[p]);
+                            a2 = make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
+                        } else {
+                            a2 = decay2_fresh(dl2, Aw2[p]);
+                        }
+                        lam2[p] = fma2(dy2, c2, lam2[p]);
+                        pc[p] = mul2(dy2, hs[k][p]);
+                        pb[p] = mul2(lam2[p], du2);
+                        accy = fma2(c2, hs[k][p], accy);
+                        accb = fma2(lam2[p], b2, accb);
+                        const float2 la = mul2(lam2[p], a2);
+                        const float2 ga = mul2(la, hprev);
+                        accd = fma2(ga, Aw2[p], accd);
+                        dA2[p] = fma2(ga, dl2, dA2[p]);
+                        lam2[p] = la;
+                    }
+                    *reinterpret_cast<float4 *>(sredq + k * KSTRIDE) =
+                        make_float4(pc[0].x, pc[0].y, pc[1].x, pc[1].y);
+                    *reinterpret_cast<float4 *>(sredq + (KC + k) * KSTRIDE) =
+                        make_float4(pb[0].x, pb[0].y, pb[1].x, pb[1].y);
+                    ddl_p[i] = (accd.x + accd.y) * kAUnscale;
+                    dub_p[i] = accb.x + accb.y;
+                    y_p[i] = accy.x + accy.y;
                 }
-                *reinterpret_cast<float4 *>(sredq + k * KSTRIDE) = make_float4(pc[0].x, pc[0].y, pc[1].x, pc[1].y);
-                *reinterpret_cast<float4 *>(sredq + (KC + k) * KSTRIDE) =
-                    make_float4(pb[0].x, pb[0].y, pb[1].x, pb[1].y);
-                ddl_p[k] = accd.x + accd.y;
-                dub_p[k] = accb.x + accb.y;
-                y_p[k] = accy.x + accy.y;
-            }
-            float ddl_o[KG], dub_o[KG], y_o[KG];
-            reduce_scatter_steps<KC, G>(ddl_p, ddl_o, q);
-            reduce_scatter_steps<KC, G>(dub_p, dub_o, q);
-            reduce_scatter_steps<KC, G>(y_p, y_o, q);
-#pragma unroll
-            for (int j = 0; j < KG; ++j) {
-                const int rr = k0 + j * G;
+                // lane q keeps the sums of step jg G + q (the step it owns)
+                // and finishes that step's du, ddelta, dz
+                float r[1];
+                reduce_scatter_steps<G, G>(ddl_p, r, q);
+                const float ddl_o = r[0];
+                reduce_scatter_steps<G, G>(dub_p, r, q);
+                const float dub = r[0];
+                reduce_scatter_steps<G, G>(y_p, r, q);
+                const float y_o = r[0];
+                const int rr = k0 + jg * G;
                 if (rr + q < nrows && active) {
-                    const float dub = dub_o[j];
-                    const float ddl = fmaf(uo[j], dub, ddl_o[j]);
-                    const float dd = args.softplus ? ddl * sigmoid_of<PRECISE>(so[j]) : ddl;
-                    io::store_smem(su + rr * ROW, fmaf(dyo[j], dskip, dlo[j] * dub));
+                    const float uo = io::load_smem(su + rr * ROW);
+                    const float ddl = fmaf(uo, dub, ddl_o);
+                    const float dd = args.softplus ? ddl * sigmoid_of<PRECISE>(so[jg]) : ddl;
+                    io::store_smem(su + rr * ROW, fmaf(dyo[jg], dskip, dlo[jg] * dub));
                     io::store_smem(sd + rr * ROW, dd);
                     if (pz) {
-                        const float y = fmaf(dskip, uo[j], y_o[j]);
-                        io::store_smem(sz + rr * ROW, go[j] * y * szo[j] * (1.f + zo[j] * (1.f - szo[j])));
+                        const float zo = io::load_smem(sz + rr * ROW), go = io::load_smem(sg + rr * ROW);
+                        const float y = fmaf(dskip, uo, y_o);
+                        io::store_smem(sz + rr * ROW, go * y * szo[jg] * (1.f + zo * (1.f - szo[jg])));
                     }
                     dbias_acc += dd;
-                    dD_acc = fmaf(dyo[j], uo[j], dD_acc);
+                    dD_acc = fmaf(dyo[jg], uo, dD_acc);
                 }
             }
-            // ---- dB, dC of the sub-chunk: sum the tile over the block's
-            // channels (SPLIT groups of threads each sum CPB / SPLIT channels
-            // and add their partial sums)
+            // ---- dB, dC of the sub-chunk: 64 (which, step, quad) sums over
+            // the block's 32 channels, two threads (adjacent lanes) per sum,
+            // 16 channels each; the odd thread starts one channel later so
+            // that the two halves of a quarter-warp fall in different banks
             __syncthreads();
-            constexpr int SPLIT = kBlock / (2 * KC * NQ) < SSM_BWD_RED_SPLIT ? kBlock / (2 * KC * NQ)
-                                                                             : SSM_BWD_RED_SPLIT;
-            if (tid < SPLIT * 2 * KC * NQ) {
-                const int task = tid % (2 * KC * NQ), part = tid / (2 * KC * NQ);
+            {
+                const int task = tid >> 1, part = tid & 1;
                 const int nq = task % NQ;
                 const int kk = (task / NQ) % KC;
                 const int which = task / (NQ * KC);  // 0: dC, 1: dB
                 const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) + nq +
-                                    part * (CPB / SPLIT) * NQ;
+                                    part * (CPB / 2) * NQ;
                 float2 a01 = make_float2(0.f, 0.f), a23 = a01, b01 = a01, b23 = a01;
 #pragma unroll
-                for (int cc = 0; cc < CPB / SPLIT; cc += 2) {
-                    const float4 v = col[cc * NQ], w = col[(cc + 1) * NQ];
+                for (int cc = 0; cc < CPB / 2; cc += 2) {
+                    const float4 v = col[((cc + part) & (CPB / 2 - 1)) * NQ];
+                    const float4 w = col[((cc + 1 + part) & (CPB / 2 - 1)) * NQ];
                     a01 = add2(a01, make_float2(v.x, v.y));
                     a23 = add2(a23, make_float2(v.z, v.w));
                     b01 = add2(b01, make_float2(w.x, w.y));
@@ -629,8 +646,12 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                 }
                 a01 = add2(a01, b01);
                 a23 = add2(a23, b23);
+                a01.x += __shfl_xor_sync(0xffffffffu, a01.x, 1);
+                a01.y += __shfl_xor_sync(0xffffffffu, a01.y, 1);
+                a23.x += __shfl_xor_sync(0xffffffffu, a23.x, 1);
+                a23.y += __shfl_xor_sync(0xffffffffu, a23.y, 1);
                 const int n = nq * 4;
-                if (k0 + kk < nrows && n < N) {
+                if (part == 0 && k0 + kk < nrows && n < N) {
                     float *dst = (which ? args.dB : args.dC) + (b * L + t0 + kk) * N + n;
                     if (args.vec_red) {
                         atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(a01.x, a01.y, a23.x, a23.y));
@@ -645,12 +666,13 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             __syncthreads();
         };
         if (rows == T) {
-#pragma unroll
+#pragma unroll 1
             for (int sc = T / KC - 1; sc >= 0; --sc) sub_chunk(sc * KC, T);
         } else {
             for (int sc = (rows + KC - 1) / KC - 1; sc >= 0; --sc) sub_chunk(sc * KC, rows);
         }
-        // ---- the chunk's du, ddelta, dz leave in 16-byte pieces
+        // ---- the chunk's du, ddelta, dz leave in 16-byte pieces (the stage
+        // is reused S chunks later, after the barrier at the top of the loop)
         for (int p = tid; p < T * ROWV; p += kBlock) {
             const int r = p / ROWV, v = p % ROWV;
             const int64_t col = d0 + v * EPV;
@@ -663,7 +685,6 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                     __stcs(reinterpret_cast<uint4 *>(gdz + go), *reinterpret_cast<const uint4 *>(st + 2 * TILE + so));
             }
         }
-        __syncthreads();  // the stage is free for the next copies
     }
     cp_async_wait<0>();
     // dD and dbias were accumulated by the owner of each step: sum the group

@@ -144,6 +144,21 @@ __device__ __forceinline__ float decay_of(float x) {
     return ex2_approx(x);
 }
 
+// Fast-tier decay pair exp2(Delta * Aw) evaluated anew, bit for bit what
+// mul2 + decay_of<false> give.  The statement is volatile so that the
+// compiler does not merge it with an earlier evaluation of the same decays: a
+// kernel that recomputes decays instead of keeping them (to save the registers
+// that would hold them) gets the recomputation it asked for.
+__device__ __forceinline__ float2 decay2_fresh(float2 dl2, float2 aw2) {
+    float2 r;
+    asm volatile(
+        "{\n.reg .b64 ra, rb, rd;\n.reg .f32 x0, x1;\nmov.b64 ra, {%2,%3};\nmov.b64 rb, {%4,%5};\n"
+        "mul.rn.f32x2 rd, ra, rb;\nmov.b64 {x0,x1}, rd;\nex2.approx.ftz.f32 %0, x0;\nex2.approx.ftz.f32 %1, x1;\n}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(dl2.x), "f"(dl2.y), "f"(aw2.x), "f"(aw2.y));
+    return r;
+}
+
 // ------------------------------------------------- packed fp32 pairs (f32x2)
 // One instruction operates on two fp32 lanes held in a register pair; each
 // lane is rounded exactly like the scalar instruction (round to nearest even).
