@@ -52,8 +52,7 @@ constexpr int kP = 64;          // head dimension (one 128-byte swizzled row of 
 constexpr uint32_t kTileBytes = kQ * 128;  // 128 rows x 128 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
-// TMEM columns (fp32): C B^T, Y_diag, Y_off, chunk state
-constexpr uint32_t kColCB = 0, kColY = 128, kColYoff = 192, kColS = 256, kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;  // tensor-memory columns allocated per CTA
 
 struct SsdArgs {
     const void *dt;
@@ -77,6 +76,14 @@ __device__ __forceinline__ void load_piece(const unsigned char *tile, int row, i
         v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
     }
 }
+// Read-only global load as a volatile statement: it stays where it is written
+// (a prefetch a whole chunk ahead of its use) instead of being moved next to
+// the use by the compiler.
+__device__ __forceinline__ float ld_nc_bf16(const __nv_bfloat16 *p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return __uint_as_float((uint32_t)v << 16);
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
@@ -91,19 +98,31 @@ __device__ __forceinline__ void store_piece(unsigned char *tile, int row, int pi
 }
 
 // ---------------------------------------------------------------------------
-// The tiles of chunk c + 1 (C, B, X; two stages) are copied while chunk c
-// computes, the masked intra-chunk matrix M stays in tensor memory as the A
-// operand of M X (no shared-memory round trip), and z / out move between
-// registers and global memory directly, so that the double buffers fit in
-// shared memory.  Inside a chunk the products and the element-wise phases
-// overlap: C B^T and C H^T run while the threads form w o X; B^T (w o X)
-// runs while they mask C B^T; M X runs while they update the carried state.
+// Warp-specialised layout.  One CTA per (b, h): 16 element-wise warps
+// (512 threads) and one warp whose elected thread issues every TMA copy and
+// every tensor-core product.  The two sides meet only at mbarriers: the
+// products signal the element-wise warps through tcgen05.commit, the
+// element-wise warps signal the issuing thread with one arrival per warp.
+// The issuing thread therefore never waits behind element-wise work, and the
+// next chunk's C B^T runs while the current chunk updates its state and
+// writes its output.
+//
+// Shared memory: two stages of C, B, X tiles (TMA, two chunks deep), the
+// two-term w o X tiles and the two-term carried state.  The w o X high-part
+// tile is reused twice per chunk once B^T (w o X) has read it: z arrives in it
+// by TMA, each thread overwrites its own z pieces with its out pieces, and a
+// TMA store writes the 128 x 64 out tile (rows past the sequence are clipped).
+//
+// Tensor memory (fp32 columns): C B^T 128 | C [Hh | Hl]^T 128 (both terms of
+// the state in one N = 128 product, summed when read) | chunk state 64 | Y 64
+// | M high 64 | M low 64 (two bf16 per column).
 enum Tile2 { kC0s0, kC1s0, kB0s0, kB1s0, kXs0, kC0s1, kC1s1, kB0s1, kB1s1, kXs1, kXh2, kXl2, kH2, kHl2,
              kNumTiles2 };
 constexpr uint32_t kSmemBytes2 = kNumTiles2 * kTileBytes + 1024;
-constexpr int kThreads2 = 512;   // 16 warps: four per scheduler to hide latency
-constexpr uint32_t kColM = 320;  // M as the A operand, high part: 64 columns (two bf16 per column)
-constexpr uint32_t kColMl = 384; // low part
+constexpr int kEw = 512;               // element-wise threads: four warps per scheduler
+constexpr int kThreads2 = kEw + 32;    // plus the issuing warp
+constexpr uint32_t kTCB = 0, kTYo = 128, kTS = 256, kTY = 320, kTM = 384, kTMl = 448;
+static_assert(kHl2 == kH2 + 1 && kXl2 == kXh2 + 1, "two-term halves are adjacent tiles");
 
 // The carried state's two-term copy (this thread's 16 of the 64 channels of
 // state row r): pieces 2 part and 2 part + 1 of the row.
@@ -122,297 +141,437 @@ __device__ __forceinline__ void store_state_split16(unsigned char *hi, unsigned 
     }
 }
 
-// Thread (warp w, lane l) owns TMEM lane / tile row r = 32 (w % 4) + l and
-// the quarter part = w / 4 of the columns: channels [16 part, 16 part + 16)
-// of the head, mask columns [32 part, 32 part + 32).
+// Barrier among the 512 element-wise threads only (named barrier 1).
+__device__ __forceinline__ void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEw) : "memory"); }
+
+// Element-wise thread (warp w < 16, lane l) owns TMEM lane / tile row
+// r = 32 (w % 4) + l and the quarter part = w / 4 of the columns: channels
+// [16 part, 16 part + 16) of the head, mask columns [32 part, 32 part + 32).
+template <int NT>  // dstate / 64: 64-column tiles of B and C
 __global__ void __launch_bounds__(kThreads2, 1)
 ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-                         const __grid_constant__ CUtensorMap mapC, const __nv_bfloat16 *__restrict__ zg,
-                         __nv_bfloat16 *__restrict__ og, const SsdArgs a) {
+                         const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapO,
+                         const __grid_constant__ CUtensorMap mapZ, const SsdArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                           ~static_cast<uintptr_t>(1023));
     auto tile = [&](int i) { return sm + (uint32_t)i * kTileBytes; };
-    __shared__ uint64_t bar_ld[2], bar_mma1, bar_mma2, bar_mma3;
+    // products -> element-wise warps
+    __shared__ uint64_t bar_ld[2], bar_z, bar_cb, bar_ch, bar_s, bar_y, bar_fin;
+    // element-wise warps -> issuing thread (one arrival per warp)
+    __shared__ uint64_t bar_h, bar_wx, bar_m, bar_cbfree, bar_yfree;
     __shared__ uint32_t s_tmem;
-    __shared__ float s_dl[kQ], s_cum[kQ], s_wsum[16];
-    __shared__ __align__(16) float s_q[kQ];  // A S_s - log2(Delta_s), log2 units (+inf where Delta_s = 0)
-    __shared__ int s_abort;
+    // per step s of the chunk: Delta_s, the running sum S_s, and
+    // v_s = exp(A (S_J - S_s)) Delta_s with S_J the running sum at the end of
+    // the 32-step block J that holds s
+    __shared__ __align__(16) float s_dl[kQ];
+    __shared__ __align__(16) float s_cum[kQ];
+    __shared__ __align__(16) float s_v[kQ];
+    __shared__ float s_wsum[4];
+    __shared__ int s_abort, s_abort_ew;  // s_abort_ew: the element-wise warps' copy, taken between barriers
 
+    constexpr int ksteps = 4 * NT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, part = warp >> 2;
+    const int quad = warp & 3, part = (warp >> 2) & 3;
     const int r = quad * 32 + lane;
     const int64_t b = blockIdx.x / a.heads, h = blockIdx.x % a.heads;
     const int g = (int)(h / (a.heads / a.groups));
     const int N = a.dstate;
-    const int ntiles = N / 64, ksteps = N / 16;
     const int64_t L = a.seqlen;
     const float Ah = a.A[h] * kLog2e;
     const float Dh = a.D ? a.D[h] : 0.f;
     const float bias = a.dt_bias ? a.dt_bias[h] : 0.f;
     const __nv_bfloat16 *dt = static_cast<const __nv_bfloat16 *>(a.dt);
+    const bool has_z = a.has_z != 0;
 
     if (tid == 0) {
-        mbar_init(&bar_ld[0], 1);
-        mbar_init(&bar_ld[1], 1);
-        mbar_init(&bar_mma1, 1);
-        mbar_init(&bar_mma2, 1);
-        mbar_init(&bar_mma3, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&bar_ld[i], 1);
+        mbar_init(&bar_z, 1);
+        mbar_init(&bar_cb, 1);
+        mbar_init(&bar_ch, 1);
+        mbar_init(&bar_s, 1);
+        mbar_init(&bar_y, 1);
+        mbar_init(&bar_fin, 1);
+        mbar_init(&bar_h, kEw / 32);
+        mbar_init(&bar_wx, kEw / 32);
+        mbar_init(&bar_m, kEw / 32);
+        mbar_init(&bar_cbfree, kEw / 32);
+        mbar_init(&bar_yfree, kEw / 32);
         mbar_fence_init();
         s_abort = 0;
+        s_abort_ew = 0;
     }
     if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = s_tmem;
-    const uint32_t tlane = tm + ((uint32_t)(quad * 32) << 16);
     const int nchunks = (int)((L + kQ - 1) / kQ);
-
-    auto issue = [&](int cc) {  // thread 0: the tiles of chunk cc into stage cc & 1
-        const int st = cc & 1;
-        const int base = st ? kC0s1 : kC0s0;
-        mbar_expect_tx(&bar_ld[st], (uint32_t)(2 * ntiles + 1) * kTileBytes);
-        const int32_t t0 = cc * kQ;
-        for (int kt = 0; kt < ntiles; ++kt) {
-            tma_load_3d(tile(base + kt), &mapC, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
-            tma_load_3d(tile(base + 2 + kt), &mapB, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
-        }
-        tma_load_3d(tile(base + 4), &mapX, (int32_t)(h * kP), t0, (int32_t)b, &bar_ld[st]);
-    };
-    if (tid == 0 && nchunks > 0) issue(0);
-
-    // carried state H[n = r][p = 16 part + i], fp32
-    float H[16];
-    const bool nrow = r < N;
-    const int64_t sbase = ((b * a.heads + h) * kP + 16 * part) * N + r;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
-    store_state_split16(tile(kH2), tile(kHl2), r, part, H);
-    fence_proxy_async();
-    __syncthreads();
-
     auto wait = [&](uint64_t *bar, uint32_t par) {
         if (!mbar_wait(bar, par, kWaitNs)) {
             atomicOr(a.status, 2u);
             s_abort = 1;
+            return false;
         }
+        return true;
     };
 
-    // z (this thread's 16 channels of row r) and dt of chunk cc, into registers
-    uint4 zn[2];
-    float dtn = 0.f;
-    auto prefetch = [&](int cc) {
-        const int64_t t = (int64_t)cc * kQ + r;
-        const bool ok = cc < nchunks && t < L;
-        const int64_t gr = ((b * L + t) * a.heads + h) * kP + 16 * part;
+    if (warp == kEw / 32) {
+        // ------------------------------------------------- the issuing warp
+        // The whole warp runs the loop (descriptors and waits warp-uniform);
+        // one elected lane issues the copies, the products and the commits.
+        const uint32_t el = elect_one();
+        const uint64_t dK = desc_sw128(smem_u32(sm), 16, 1024);
+        const uint64_t dMN2 = desc_sw128(smem_u32(sm), kTileBytes, 1024);
+        auto at = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
+        auto wait_w = [&](uint64_t *bar, uint32_t par) {  // the same answer in every lane
+            const bool ok1 = __all_sync(0xffffffffu, mbar_wait(bar, par, kWaitNs));
+            if (!ok1 && el) {
+                atomicOr(a.status, 2u);
+                s_abort = 1;
+            }
+            return ok1;
+        };
+        int ld_issued0 = 0, ld_issued1 = 0, z_issued = 0;
+        auto issue = [&](int cc) {  // the C, B, X tiles of chunk cc into stage cc & 1
+            const int st = cc & 1;
+            if (el) {
+                const int base = st ? kC0s1 : kC0s0;
+                mbar_expect_tx(&bar_ld[st], (uint32_t)(2 * NT + 1) * kTileBytes);
+                const int32_t t0 = cc * kQ;
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-            zn[j] = (zg && ok) ? __ldg(reinterpret_cast<const uint4 *>(zg + gr) + j) : make_uint4(0, 0, 0, 0);
-        dtn = ok ? __bfloat162float(dt[(b * L + t) * a.heads + h]) : 0.f;
-    };
-    prefetch(0);
+                for (int kt = 0; kt < NT; ++kt) {
+                    tma_load_3d(tile(base + kt), &mapC, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
+                    tma_load_3d(tile(base + 2 + kt), &mapB, g * N + 64 * kt, t0, (int32_t)b, &bar_ld[st]);
+                }
+                tma_load_3d(tile(base + 4), &mapX, (int32_t)(h * kP), t0, (int32_t)b, &bar_ld[st]);
+            }
+            if (st) ++ld_issued1; else ++ld_issued0;
+        };
+        auto mma_cb = [&](int cc) {  // C B^T of chunk cc
+            const int tC0 = (cc & 1) ? kC0s1 : kC0s0;
+            constexpr uint32_t id_cb = idesc_bf16(128, 128, kMajorK, kMajorK);
+            const uint64_t dC = at(dK, (uint32_t)tC0 * kTileBytes), dB = at(dK, (uint32_t)(tC0 + 2) * kTileBytes);
+#pragma unroll
+            for (int k = 0; k < ksteps; ++k) {
+                const uint32_t o = (k / 4) * kTileBytes + (k % 4) * 32;
+                mma_bf16_if(el, tm + kTCB, at(dC, o), at(dB, o), id_cb, k > 0);
+            }
+            mma_commit_if(el, &bar_cb);
+        };
+        bool ok = true;
+        if (nchunks > 0) issue(0);
+        if (nchunks > 1) issue(1);
+        if (nchunks > 0) {
+            ok = wait_w(&bar_ld[0], 0u);
+            if (ok) {
+                fence_after_sync();
+                mma_cb(0);
+            }
+        }
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int st = c & 1;
+            const uint32_t par = (uint32_t)c & 1u;
+            const int tC0 = st ? kC0s1 : kC0s0, tB0 = tC0 + 2, tX = tC0 + 4;
+            // C [Hh | Hl]^T with the state entering chunk c
+            if (!(ok = wait_w(&bar_h, par))) break;
+            fence_after_sync();
+            {
+                constexpr uint32_t id_yo = idesc_bf16(128, 128, kMajorK, kMajorMN);
+                const uint64_t dC = at(dK, (uint32_t)tC0 * kTileBytes), dH = at(dMN2, (uint32_t)kH2 * kTileBytes);
+#pragma unroll
+                for (int k = 0; k < ksteps; ++k)
+                    mma_bf16_if(el, tm + kTYo, at(dC, (k / 4) * kTileBytes + (k % 4) * 32), at(dH, k * 2048), id_yo,
+                                k > 0);
+                mma_commit_if(el, &bar_ch);
+            }
+            // chunk state B^T (w o X), both terms accumulated
+            if (!(ok = wait_w(&bar_wx, par))) break;
+            fence_after_sync();
+            {
+                constexpr uint32_t id_s = idesc_bf16(128, kP, kMajorMN, kMajorMN);
+                const uint64_t dB2 = at(dMN2, (uint32_t)tB0 * kTileBytes);
+#pragma unroll
+                for (int xp = 0; xp < 2; ++xp)
+#pragma unroll
+                    for (int k = 0; k < kQ / 16; ++k)
+                        mma_bf16_if(el, tm + kTS, at(dB2, k * 2048), at(dK, (kXh2 + xp) * kTileBytes + k * 2048),
+                                    id_s, xp > 0 || k > 0);
+                mma_commit_if(el, &bar_s);
+            }
+            // Y_diag = M X, both terms of M from tensor memory
+            if (!(ok = wait_w(&bar_m, par))) break;
+            fence_after_sync();
+            {
+                constexpr uint32_t id_y = idesc_bf16(128, kP, kMajorK, kMajorMN);
+                const uint64_t dX = at(dK, (uint32_t)tX * kTileBytes);
+#pragma unroll
+                for (int mp = 0; mp < 2; ++mp)
+#pragma unroll
+                    for (int k = 0; k < kQ / 16; ++k)
+                        mma_bf16_ts_if(el, tm + kTY, tm + (mp ? kTMl : kTM) + 8 * k, at(dX, k * 2048), id_y,
+                                       mp > 0 || k > 0);
+                mma_commit_if(el, &bar_y);
+            }
+            // z of chunk c into the w o X high-part tile once B^T (w o X) has read it
+            if (has_z) {
+                if (!(ok = wait_w(&bar_s, par))) break;
+                if (el) {
+                    mbar_expect_tx(&bar_z, kTileBytes);
+                    tma_load_3d(tile(kXh2), &mapZ, (int32_t)(h * kP), c * kQ, (int32_t)b, &bar_z);
+                }
+                ++z_issued;
+            }
+            // C B^T of the next chunk once this chunk's mask has read C B^T
+            if (c + 1 < nchunks) {
+                if (!(ok = wait_w(&bar_cbfree, par))) break;
+                if (!(ok = wait_w(&bar_ld[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u))) break;
+                fence_after_sync();
+                mma_cb(c + 1);
+            }
+            // chunk c is fully consumed (its C H^T / Y columns are free): its
+            // out tile, written over X in the stage, leaves by TMA store, and
+            // once the store has read it the stage takes chunk c + 2
+            if (!(ok = wait_w(&bar_yfree, par))) break;
+            if (el) {
+                tma_store_3d(&mapO, (int32_t)(h * kP), c * kQ, (int32_t)b, tile(tX));
+                tma_store_commit();
+                tma_store_wait_read<0>();
+            }
+            __syncwarp();
+            if (c + 2 < nchunks) issue(c + 2);
+        }
+        if (el) tma_store_wait_all<0>();
+        // whatever was issued completes before the CTA's memory goes away
+        mma_commit_if(el, &bar_fin);
+        (void)mbar_wait(&bar_fin, 0u, kWaitNs);
+        if (ld_issued0 > 0) (void)mbar_wait(&bar_ld[0], (uint32_t)(ld_issued0 - 1) & 1u, kWaitNs);
+        if (ld_issued1 > 0) (void)mbar_wait(&bar_ld[1], (uint32_t)(ld_issued1 - 1) & 1u, kWaitNs);
+        if (z_issued > 0) (void)mbar_wait(&bar_z, (uint32_t)(z_issued - 1) & 1u, kWaitNs);
+        __syncwarp();
+    } else {
+        // ------------------------------------------- the element-wise warps
+        const uint32_t tlane = tm + ((uint32_t)(quad * 32) << 16);
+        auto signal = [&](uint64_t *bar) {  // one arrival per warp, after the warp's writes
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        // carried state H[n = r][p = 16 part + i], fp32
+        float H[16];
+        const bool nrow = r < N;
+        const int64_t sbase = ((b * a.heads + h) * kP + 16 * part) * N + r;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) H[i] = (a.state && nrow) ? a.state[sbase + (int64_t)i * N] : 0.f;
+        store_state_split16(tile(kH2), tile(kHl2), r, part, H);
+        fence_proxy_async();
+        signal(&bar_h);
 
-    int c = 0;
-    for (; c < nchunks; ++c) {
-        const int st = c & 1;
-        const int64_t t0 = (int64_t)c * kQ;
-        const int64_t trow = t0 + r;
-        const bool valid = trow < L;
-        const int tC0 = st ? kC0s1 : kC0s0, tB0 = tC0 + 2, tX = tC0 + 4;
-        // 1. the next chunk's tiles into the other stage (its last readers,
-        // the previous chunk's products and threads, are done)
-        if (tid == 0 && c + 1 < nchunks) issue(c + 1);
-        // 2. this chunk's z and dt (prefetched a chunk ahead); Delta and its
-        // running sum over the chunk
-        const uint4 zr0 = zn[0], zr1 = zn[1];
-        const float dt_raw = dtn;
-        const int64_t grow = ((b * L + trow) * a.heads + h) * kP + 16 * part;
-        prefetch(c + 1);
-        float dl = 0.f;
-        if (valid) {
-            const float sv = dt_raw + bias;
-            dl = a.softplus ? softplus<false>(sv) : sv;
-        }
-        float cum = dl;
+        // Delta = softplus(dt + bias) of chunk cc and its running sum over the
+        // chunk (warps of part 0; dt is loaded a chunk ahead), in two halves
+        // around a barrier: the in-warp scan, then the warps' offsets and the
+        // tables s_dl, s_cum, s_q.  Chunk c + 1's tables are formed while chunk
+        // c waits for its last products (they are no longer read by then).
+        float dtn = 0.f;
+        auto prefetch_dt = [&](int cc) {
+            const int64_t t = (int64_t)cc * kQ + r;
+            dtn = (cc < nchunks && t < L) ? ld_nc_bf16(dt + (b * L + t) * a.heads + h) : 0.f;
+        };
+        auto scan_a = [&](int cc, float &dl, float &cum) {
+            dl = 0.f;
+            if ((int64_t)cc * kQ + r < L) {
+                const float sv = dtn + bias;
+                dl = a.softplus ? softplus<false>(sv) : sv;
+            }
+            prefetch_dt(cc + 1);
+            cum = dl;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, cum, o);
-            if (lane >= o) cum += v;
-        }
-        if (lane == 31) s_wsum[warp] = cum;
-        __syncthreads();
-        for (int w2 = 0; w2 < quad; ++w2) cum += s_wsum[4 * part + w2];
-        if (part == 0) {
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, cum, o);
+                if (lane >= o) cum += v;
+            }
+            if (lane == 31) s_wsum[quad] = cum;
+        };
+        auto scan_b = [&](float dl, float cum) {
+            for (int w2 = 0; w2 < quad; ++w2) cum += s_wsum[w2];
+            const float send = __shfl_sync(0xffffffffu, cum, 31);
             s_dl[r] = dl;
             s_cum[r] = cum;
-            s_q[r] = dl > 0.f ? fmaf(Ah, cum, -lg2_approx(dl)) : __int_as_float(0x7f800000);
+            s_v[r] = ex2_approx(Ah * (send - cum)) * dl;
+        };
+        {
+            float dl0 = 0.f, cum0 = 0.f;
+            if (part == 0) {
+                prefetch_dt(0);
+                scan_a(0, dl0, cum0);
+            }
+            ew_sync();
+            if (part == 0) scan_b(dl0, cum0);
+            ew_sync();
         }
-        wait(&bar_ld[st], (uint32_t)(c >> 1) & 1u);
-        __syncthreads();
-        if (s_abort) break;
-        const float cum_end = s_cum[kQ - 1];
 
-        // 3. C B^T and C H_prev^T (two-term state copy)
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_cb = idesc_bf16(128, 128, kMajorK, kMajorK);
-            const uint32_t id_yo = idesc_bf16(128, kP, kMajorK, kMajorMN);
-            for (int k = 0; k < ksteps; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(tile(tB0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                mma_bf16(tm + kColCB, ad, bd, id_cb, k > 0);
-            }
-            for (int hp = 0; hp < 2; ++hp)
-                for (int k = 0; k < ksteps; ++k) {
-                    const uint64_t ad = desc_sw128(smem_u32(tile(tC0 + k / 4)) + (k % 4) * 32, 16, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(hp ? kHl2 : kH2)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColYoff, ad, bd, id_yo, hp > 0 || k > 0);
-                }
-            mma_commit(&bar_mma1);
-        }
-        // 4. w o X as bf16 high and low parts, w_s = exp(A (S_end - S_s)) Delta_s
-        {
-            const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
+        int c = 0;
+        for (; c < nchunks; ++c) {
+            const int st = c & 1;
+            const uint32_t par = (uint32_t)c & 1u;
+            const int tX = (st ? kC0s1 : kC0s0) + 4;
+            // 1. this chunk's Delta tables (complete since the barrier that
+            // ended the previous chunk)
+            const float dl = s_dl[r], cum = s_cum[r];
+            const float cum_end = s_cum[kQ - 1];
+
+            // 2. w o X as bf16 high and low parts, w_s = exp(A (S_end - S_s)) Delta_s
+            wait(&bar_ld[st], (uint32_t)(c >> 1) & 1u);
+            {
+                const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float x8[8], hi[8], lo[8];
-                load_piece(tile(tX), r, 2 * part + j, x8);
+                for (int j = 0; j < 2; ++j) {
+                    float x8[8], hi[8], lo[8];
+                    load_piece(tile(tX), r, 2 * part + j, x8);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float xw = w * x8[i];
-                    hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
-                    lo[i] = xw - hi[i];
-                }
-                store_piece(tile(kXh2), r, 2 * part + j, hi);
-                store_piece(tile(kXl2), r, 2 * part + j, lo);
-            }
-        }
-        fence_proxy_async();
-        __syncthreads();
-        // 5. chunk state B^T (w o X)
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_s = idesc_bf16(128, kP, kMajorMN, kMajorMN);
-            for (int xp = 0; xp < 2; ++xp)
-                for (int k = 0; k < kQ / 16; ++k) {
-                    const uint64_t ad = desc_sw128(smem_u32(tile(tB0)) + k * 2048, kTileBytes, 1024);
-                    const uint64_t bd = desc_sw128(smem_u32(tile(xp ? kXl2 : kXh2)) + k * 2048, 16, 1024);
-                    mma_bf16(tm + kColS, ad, bd, id_s, xp > 0 || k > 0);
-                }
-            mma_commit(&bar_mma2);
-        }
-        // 6. M[t, s] = CB[t, s] exp(A (S_t - S_s)) Delta_s for row t = r and the
-        // 32 columns of this part, as bf16 high and low parts in tensor memory:
-        // CB 2^(p_t - q_s), p_t = A S_t, q_s = A S_s - log2(Delta_s) when Delta
-        // is a softplus (>= 0), the product form otherwise; a block of columns
-        // above the diagonal for the whole warp is zero without arithmetic.
-        wait(&bar_mma1, (uint32_t)c & 1u);
-        fence_after_sync();
-        {
-            const int sb = 32 * part;
-            uint32_t mh[16], ml[16];
-            if (sb > quad * 32 + 31) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) mh[i] = ml[i] = 0u;
-            } else {
-                const float pt = Ah * cum;
-                float cb[32];
-                tmem_ld32(tlane + kColCB + sb, cb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 q4 = *reinterpret_cast<const float4 *>(s_q + sb + 4 * i4);
-                    const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-                    float m[4], mhf[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s0 = sb + 4 * i4 + e;
-                        const float f = a.softplus ? ex2_approx(pt - qv[e])
-                                                   : ex2_approx(Ah * (cum - s_cum[s0])) * s_dl[s0];
-                        m[e] = s0 <= r ? cb[4 * i4 + e] * f : 0.f;
-                        mhf[e] = __bfloat162float(__float2bfloat16_rn(m[e]));
+                    for (int i = 0; i < 8; ++i) {
+                        const float xw = w * x8[i];
+                        hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
+                        lo[i] = xw - hi[i];
                     }
+                    store_piece(tile(kXh2), r, 2 * part + j, hi);
+                    store_piece(tile(kXl2), r, 2 * part + j, lo);
+                }
+            }
+            fence_proxy_async();
+            signal(&bar_wx);
+
+            // 3. M[t, s] = CB[t, s] exp(A (S_t - S_s)) Delta_s for row t = r and
+            // the 32 columns of this part (block J = part), as bf16 high and
+            // low parts in tensor memory.  Blocks above the diagonal (J > the
+            // row block) are zero without arithmetic; below it the decay
+            // separates exactly, exp(A (S_t - S_J)) v_s, both factors at most
+            // one (the running sum grows), so a row takes one exponential per
+            // block; the diagonal block takes exp(A (S_t - S_s)) Delta_s per
+            // element and the causal select s <= t.
+            wait(&bar_cb, par);
+            fence_after_sync();
+            {
+                const int sb = 32 * part;
+                uint32_t mh[16], ml[16];
+                auto split4 = [&](int i4, const float (&m)[4]) {
+                    float mhf[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) mhf[e] = __bfloat162float(__float2bfloat16_rn(m[e]));
                     mh[2 * i4] = pack_bf16x2(mhf[0], mhf[1]);
                     mh[2 * i4 + 1] = pack_bf16x2(mhf[2], mhf[3]);
                     ml[2 * i4] = pack_bf16x2(m[0] - mhf[0], m[1] - mhf[1]);
                     ml[2 * i4 + 1] = pack_bf16x2(m[2] - mhf[2], m[3] - mhf[3]);
-                }
-            }
-            tmem_st16(tlane + kColM + 16 * part, mh);
-            tmem_st16(tlane + kColMl + 16 * part, ml);
-            tmem_wait_st();
-        }
-        fence_before_sync();
-        __syncthreads();
-        if (s_abort) break;
-        // 7. Y_diag = M X with both parts of M read from tensor memory
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_y = idesc_bf16(128, kP, kMajorK, kMajorMN);
-            for (int mp = 0; mp < 2; ++mp)
-                for (int k = 0; k < kQ / 16; ++k) {
-                    const uint64_t bd = desc_sw128(smem_u32(tile(tX)) + k * 2048, 16, 1024);
-                    mma_bf16_ts(tm + kColY, tm + (mp ? kColMl : kColM) + 8 * k, bd, id_y, mp > 0 || k > 0);
-                }
-            mma_commit(&bar_mma3);
-        }
-        // 8. carried state: H = exp(A S_end) H + B^T (w o X), and its copy for the next chunk
-        wait(&bar_mma2, (uint32_t)c & 1u);
-        fence_after_sync();
-        {
-            float sv[16];
-            tmem_ld16(tlane + kColS + 16 * part, sv);
-            tmem_wait_ld();
-            const float gdec = ex2_approx(Ah * cum_end);
+                };
+                if (part > quad) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
-            store_state_split16(tile(kH2), tile(kHl2), r, part, H);
-        }
-        // 9. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), straight to global memory
-        wait(&bar_mma3, (uint32_t)c & 1u);
-        fence_after_sync();
-        {
-            float yd[16], yo[16];
-            tmem_ld16(tlane + kColY + 16 * part, yd);
-            tmem_ld16(tlane + kColYoff + 16 * part, yo);
-            tmem_wait_ld();
-            const float et = ex2_approx(Ah * cum);
+                    for (int i = 0; i < 16; ++i) mh[i] = ml[i] = 0u;
+                    fence_before_sync();
+                    signal(&bar_cbfree);
+                } else {
+                    float cb[32];
+                    tmem_ld32(tlane + kTCB + sb, cb);
+                    tmem_wait_ld();
+                    fence_before_sync();
+                    signal(&bar_cbfree);
+                    if (part < quad) {
+                        const float u = ex2_approx(Ah * (cum - s_cum[sb + 31]));
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float x8[8];
-                load_piece(tile(tX), r, 2 * part + j, x8);
-                const uint4 zq = j ? zr1 : zr0;
-                const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
-                uint32_t ow[4];
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(s_v + sb + 4 * i4);
+                            const float m[4] = {cb[4 * i4] * (u * v4.x), cb[4 * i4 + 1] * (u * v4.y),
+                                                cb[4 * i4 + 2] * (u * v4.z), cb[4 * i4 + 3] * (u * v4.w)};
+                            split4(i4, m);
+                        }
+                    } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float y0 = fmaf(Dh, x8[2 * i], fmaf(et, yo[8 * j + 2 * i], yd[8 * j + 2 * i]));
-                    float y1 = fmaf(Dh, x8[2 * i + 1], fmaf(et, yo[8 * j + 2 * i + 1], yd[8 * j + 2 * i + 1]));
-                    if (zg) {
-                        y0 *= silu<false>(__uint_as_float(zw[i] << 16));
-                        y1 *= silu<false>(__uint_as_float(zw[i] & 0xffff0000u));
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 c4 = *reinterpret_cast<const float4 *>(s_cum + sb + 4 * i4);
+                            const float4 d4 = *reinterpret_cast<const float4 *>(s_dl + sb + 4 * i4);
+                            const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, ds[4] = {d4.x, d4.y, d4.z, d4.w};
+                            float m[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int s0 = sb + 4 * i4 + e;
+                                const float f = ex2_approx(Ah * (cum - cs[e])) * ds[e];
+                                m[e] = s0 <= r ? cb[4 * i4 + e] * f : 0.f;
+                            }
+                            split4(i4, m);
+                        }
                     }
-                    ow[i] = pack_bf16x2(y0, y1);
                 }
-                if (valid) reinterpret_cast<uint4 *>(og + grow)[j] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                tmem_st16(tlane + kTM + 16 * part, mh);
+                tmem_st16(tlane + kTMl + 16 * part, ml);
+                tmem_wait_st();
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (s_abort) break;
-    }
-    if (s_abort) {
-        // let whatever was issued finish (bounded) before the memory goes away
-        (void)mbar_wait(&bar_ld[c & 1], (uint32_t)(c >> 1) & 1u, kWaitNs);
-        if (c + 1 < nchunks) (void)mbar_wait(&bar_ld[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u, kWaitNs);
-        (void)mbar_wait(&bar_mma1, (uint32_t)c & 1u, kWaitNs);
-        (void)mbar_wait(&bar_mma2, (uint32_t)c & 1u, kWaitNs);
-        (void)mbar_wait(&bar_mma3, (uint32_t)c & 1u, kWaitNs);
-    } else if (a.state && nrow) {
+            fence_before_sync();
+            signal(&bar_m);
+
+            // 4. carried state: H = exp(A S_end) H + B^T (w o X) once C H^T has
+            // read the previous copy, and its copy for the next chunk
+            wait(&bar_s, par);
+            wait(&bar_ch, par);
+            fence_after_sync();
+            {
+                float sv[16];
+                tmem_ld16(tlane + kTS + 16 * part, sv);
+                tmem_wait_ld();
+                const float gdec = ex2_approx(Ah * cum_end);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a.state[sbase + (int64_t)i * N] = H[i];
+                for (int i = 0; i < 16; ++i) H[i] = fmaf(gdec, H[i], sv[i]);
+                store_state_split16(tile(kH2), tile(kHl2), r, part, H);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            signal(&bar_h);
+            if (c + 1 < nchunks) {
+                float ndl = 0.f, ncum = 0.f;
+                if (part == 0) scan_a(c + 1, ndl, ncum);
+                ew_sync();
+                if (part == 0) scan_b(ndl, ncum);
+            }
+
+            // 5. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), written over
+            // this thread's X pieces in the stage's X tile (M X has read it);
+            // the issuing warp stores the tile by TMA
+            if (has_z) wait(&bar_z, par);
+            wait(&bar_y, par);
+            fence_after_sync();
+            {
+                float yd[16], yh[16], yl[16];
+                tmem_ld16(tlane + kTY + 16 * part, yd);
+                tmem_ld16(tlane + kTYo + 16 * part, yh);
+                tmem_ld16(tlane + kTYo + 64 + 16 * part, yl);
+                tmem_wait_ld();
+                const float et = ex2_approx(Ah * cum);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float x8[8], z8[8], o8[8];
+                    load_piece(tile(tX), r, 2 * part + j, x8);
+                    if (has_z) load_piece(tile(kXh2), r, 2 * part + j, z8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int k = 8 * j + i;
+                        float y = fmaf(Dh, x8[i], fmaf(et, yh[k] + yl[k], yd[k]));
+                        if (has_z) y *= silu<false>(z8[i]);
+                        o8[i] = y;
+                    }
+                    store_piece(tile(tX), r, 2 * part + j, o8);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            signal(&bar_yfree);
+            // the next chunk's tables are complete; the abort flag is read
+            // once, between barriers, so that every element-wise thread takes
+            // the same branch
+            if (tid == 0) s_abort_ew = *reinterpret_cast<volatile int *>(&s_abort);
+            ew_sync();
+            if (s_abort_ew) break;
+        }
+        if (!s_abort && a.state && nrow) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a.state[sbase + (int64_t)i * N] = H[i];
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -472,10 +631,13 @@ bool ssd_fwd_supported(const SsdFwdArgs &a) {
 
 cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     if (!ssd_fwd_supported(a)) return cudaErrorNotSupported;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, mo, mz;
     const int64_t hp = a.heads * a.headdim, gn = a.groups * a.dstate;
+    // without a gate the z map is never read; it is encoded over x so that
+    // the kernel parameter is a valid map
     if (!encode_btw(&mx, a.x, a.batch, a.seqlen, hp) || !encode_btw(&mb, a.B, a.batch, a.seqlen, gn) ||
-        !encode_btw(&mc, a.C, a.batch, a.seqlen, gn))
+        !encode_btw(&mc, a.C, a.batch, a.seqlen, gn) || !encode_btw(&mo, a.out, a.batch, a.seqlen, hp) ||
+        !encode_btw(&mz, a.z ? a.z : a.x, a.batch, a.seqlen, hp))
         return cudaErrorInvalidValue;
     SsdArgs k{};
     k.dt = a.dt;
@@ -497,15 +659,18 @@ cudaError_t launch_ssd_fwd(const SsdFwdArgs &a, cudaStream_t st) {
     e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (!configured[dev & 63]) {
-        e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes2);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(ssd_fwd_pipelined_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kSmemBytes2);
         if (e != cudaSuccess) return e;
         configured[dev & 63] = true;
     }
     const int64_t grid = a.batch * a.heads;
     if (grid > 2147483647LL) return cudaErrorInvalidConfiguration;
-    ssd_fwd_pipelined_kernel<<<(unsigned)grid, kThreads2, kSmemBytes2, st>>>(
-        mx, mb, mc, static_cast<const __nv_bfloat16 *>(a.z), static_cast<__nv_bfloat16 *>(a.out), k);
+    auto kern = a.dstate == 128 ? ssd_fwd_pipelined_kernel<2> : ssd_fwd_pipelined_kernel<1>;
+    kern<<<(unsigned)grid, kThreads2, kSmemBytes2, st>>>(mx, mb, mc, mo, mz, k);
     return cudaGetLastError();
 }
 
