@@ -88,6 +88,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
 }
+// Two-term bf16 split of a pair of floats: the high parts (rounded to
+// nearest) and the bf16 rounding of the remainders, two per word.
+__device__ __forceinline__ void split_pair(float a0, float a1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16x2(a0, a1);
+    lo = pack_bf16x2(a0 - __uint_as_float(hi << 16), a1 - __uint_as_float(hi & 0xffff0000u));
+}
+// The split of eight floats into piece `piece` of row `row` of two tiles.
+__device__ __forceinline__ void store_piece_split(unsigned char *hi_tile, unsigned char *lo_tile, int row, int piece,
+                                                  const float (&v)[8]) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_pair(v[2 * i], v[2 * i + 1], h[i], l[i]);
+    const uint32_t off = sw128_offset(row, piece);
+    *reinterpret_cast<uint4 *>(hi_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
 __device__ __forceinline__ void store_piece(unsigned char *tile, int row, int piece, const float (&v)[8]) {
     uint4 w;
     w.x = pack_bf16x2(v[0], v[1]);
@@ -130,19 +146,18 @@ __device__ __forceinline__ void store_state_split16(unsigned char *hi, unsigned 
                                                     const float (&H)[16]) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        float vh[8], vl[8];
+        float v[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            vh[i] = __bfloat162float(__float2bfloat16_rn(H[8 * j + i]));
-            vl[i] = H[8 * j + i] - vh[i];
-        }
-        store_piece(hi, r, 2 * part + j, vh);
-        store_piece(lo, r, 2 * part + j, vl);
+        for (int i = 0; i < 8; ++i) v[i] = H[8 * j + i];
+        store_piece_split(hi, lo, r, 2 * part + j, v);
     }
 }
 
-// Barrier among the 512 element-wise threads only (named barrier 1).
+// Barrier among the 512 element-wise threads only (named barrier 1), and
+// among the four element-wise warps that form the running sums (named
+// barrier 2).
 __device__ __forceinline__ void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEw) : "memory"); }
+__device__ __forceinline__ void scan_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Element-wise thread (warp w < 16, lane l) owns TMEM lane / tile row
 // r = 32 (w % 4) + l and the quarter part = w / 4 of the columns: channels
@@ -299,6 +314,16 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                                     id_s, xp > 0 || k > 0);
                 mma_commit_if(el, &bar_s);
             }
+            // z of chunk c into the w o X high-part tile once B^T (w o X) has read it
+            // (before M X: the copy's latency then overlaps the mask)
+            if (has_z) {
+                if (!(ok = wait_w(&bar_s, par))) break;
+                if (el) {
+                    mbar_expect_tx(&bar_z, kTileBytes);
+                    tma_load_3d(tile(kXh2), &mapZ, (int32_t)(h * kP), c * kQ, (int32_t)b, &bar_z);
+                }
+                ++z_issued;
+            }
             // Y_diag = M X, both terms of M from tensor memory
             if (!(ok = wait_w(&bar_m, par))) break;
             fence_after_sync();
@@ -312,15 +337,6 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                         mma_bf16_ts_if(el, tm + kTY, tm + (mp ? kTMl : kTM) + 8 * k, at(dX, k * 2048), id_y,
                                        mp > 0 || k > 0);
                 mma_commit_if(el, &bar_y);
-            }
-            // z of chunk c into the w o X high-part tile once B^T (w o X) has read it
-            if (has_z) {
-                if (!(ok = wait_w(&bar_s, par))) break;
-                if (el) {
-                    mbar_expect_tx(&bar_z, kTileBytes);
-                    tma_load_3d(tile(kXh2), &mapZ, (int32_t)(h * kP), c * kQ, (int32_t)b, &bar_z);
-                }
-                ++z_issued;
             }
             // C B^T of the next chunk once this chunk's mask has read C B^T
             if (c + 1 < nchunks) {
@@ -367,18 +383,22 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
         signal(&bar_h);
 
         // Delta = softplus(dt + bias) of chunk cc and its running sum over the
-        // chunk (warps of part 0; dt is loaded a chunk ahead), in two halves
-        // around a barrier: the in-warp scan, then the warps' offsets and the
-        // tables s_dl, s_cum, s_q.  Chunk c + 1's tables are formed while chunk
-        // c waits for its last products (they are no longer read by then).
+        // chunk.  Four warps whose mask blocks all lie above the diagonal
+        // (warps 4, 8, 12, 9: no mask arithmetic) do it for rows
+        // sr = 32 k + lane, k = 0..3, while the other warps mask: dt a chunk
+        // ahead, the in-warp scan, a barrier among the four, the warps'
+        // offsets and v; the tables s_dl, s_cum, s_v are replaced once every
+        // warp is done with the current ones.
+        const int scan_k = warp == 4 ? 0 : warp == 8 ? 1 : warp == 12 ? 2 : warp == 9 ? 3 : -1;
+        const int sr = 32 * scan_k + lane;
         float dtn = 0.f;
         auto prefetch_dt = [&](int cc) {
-            const int64_t t = (int64_t)cc * kQ + r;
+            const int64_t t = (int64_t)cc * kQ + sr;
             dtn = (cc < nchunks && t < L) ? ld_nc_bf16(dt + (b * L + t) * a.heads + h) : 0.f;
         };
         auto scan_a = [&](int cc, float &dl, float &cum) {
             dl = 0.f;
-            if ((int64_t)cc * kQ + r < L) {
+            if ((int64_t)cc * kQ + sr < L) {
                 const float sv = dtn + bias;
                 dl = a.softplus ? softplus<false>(sv) : sv;
             }
@@ -389,25 +409,27 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 const float v = __shfl_up_sync(0xffffffffu, cum, o);
                 if (lane >= o) cum += v;
             }
-            if (lane == 31) s_wsum[quad] = cum;
+            if (lane == 31) s_wsum[scan_k] = cum;
         };
-        auto scan_b = [&](float dl, float cum) {
-            for (int w2 = 0; w2 < quad; ++w2) cum += s_wsum[w2];
+        auto scan_b = [&](float dl, float &cum, float &v) {
+            for (int w2 = 0; w2 < scan_k; ++w2) cum += s_wsum[w2];
             const float send = __shfl_sync(0xffffffffu, cum, 31);
-            s_dl[r] = dl;
-            s_cum[r] = cum;
-            s_v[r] = ex2_approx(Ah * (send - cum)) * dl;
+            v = ex2_approx(Ah * (send - cum)) * dl;
         };
-        {
-            float dl0 = 0.f, cum0 = 0.f;
-            if (part == 0) {
-                prefetch_dt(0);
-                scan_a(0, dl0, cum0);
-            }
-            ew_sync();
-            if (part == 0) scan_b(dl0, cum0);
-            ew_sync();
+        auto publish = [&](float dl, float cum, float v) {
+            s_dl[sr] = dl;
+            s_cum[sr] = cum;
+            s_v[sr] = v;
+        };
+        float ndl = 0.f, ncum = 0.f, nv = 0.f;  // the next chunk's row sr (scan warps)
+        if (scan_k >= 0) {
+            prefetch_dt(0);
+            scan_a(0, ndl, ncum);
+            scan_sync();
+            scan_b(ndl, ncum, nv);
+            publish(ndl, ncum, nv);
         }
+        ew_sync();
 
         int c = 0;
         for (; c < nchunks; ++c) {
@@ -425,16 +447,11 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 const float w = ex2_approx(Ah * (cum_end - cum)) * dl;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    float x8[8], hi[8], lo[8];
+                    float x8[8];
                     load_piece(tile(tX), r, 2 * part + j, x8);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float xw = w * x8[i];
-                        hi[i] = __bfloat162float(__float2bfloat16_rn(xw));
-                        lo[i] = xw - hi[i];
-                    }
-                    store_piece(tile(kXh2), r, 2 * part + j, hi);
-                    store_piece(tile(kXl2), r, 2 * part + j, lo);
+                    for (int i = 0; i < 8; ++i) x8[i] *= w;
+                    store_piece_split(tile(kXh2), tile(kXl2), r, 2 * part + j, x8);
                 }
             }
             fence_proxy_async();
@@ -454,13 +471,8 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
                 const int sb = 32 * part;
                 uint32_t mh[16], ml[16];
                 auto split4 = [&](int i4, const float (&m)[4]) {
-                    float mhf[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) mhf[e] = __bfloat162float(__float2bfloat16_rn(m[e]));
-                    mh[2 * i4] = pack_bf16x2(mhf[0], mhf[1]);
-                    mh[2 * i4 + 1] = pack_bf16x2(mhf[2], mhf[3]);
-                    ml[2 * i4] = pack_bf16x2(m[0] - mhf[0], m[1] - mhf[1]);
-                    ml[2 * i4 + 1] = pack_bf16x2(m[2] - mhf[2], m[3] - mhf[3]);
+                    split_pair(m[0], m[1], mh[2 * i4], ml[2 * i4]);
+                    split_pair(m[2], m[3], mh[2 * i4 + 1], ml[2 * i4 + 1]);
                 };
                 if (part > quad) {
 #pragma unroll
@@ -505,6 +517,13 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
             }
             fence_before_sync();
             signal(&bar_m);
+            // the next chunk's Delta and running sum (scan warps), kept in
+            // registers until every warp is done with this chunk's tables
+            if (scan_k >= 0 && c + 1 < nchunks) {
+                scan_a(c + 1, ndl, ncum);
+                scan_sync();
+                scan_b(ndl, ncum, nv);
+            }
 
             // 4. carried state: H = exp(A S_end) H + B^T (w o X) once C H^T has
             // read the previous copy, and its copy for the next chunk
@@ -523,12 +542,6 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
             fence_proxy_async();
             fence_before_sync();
             signal(&bar_h);
-            if (c + 1 < nchunks) {
-                float ndl = 0.f, ncum = 0.f;
-                if (part == 0) scan_a(c + 1, ndl, ncum);
-                ew_sync();
-                if (part == 0) scan_b(ndl, ncum);
-            }
 
             // 5. out = (Y_diag + exp(A S_t) Y_off + D X) silu(z), written over
             // this thread's X pieces in the stage's X tile (M X has read it);
@@ -536,6 +549,10 @@ ssd_fwd_pipelined_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_
             if (has_z) wait(&bar_z, par);
             wait(&bar_y, par);
             fence_after_sync();
+            // M X has completed, so every warp has signalled the end of its
+            // mask and no longer reads this chunk's tables: the next chunk's
+            // replace them (visible after the barrier that ends the chunk)
+            if (scan_k >= 0 && c + 1 < nchunks) publish(ndl, ncum, nv);
             {
                 float yd[16], yh[16], yl[16];
                 tmem_ld16(tlane + kTY + 16 * part, yd);
