@@ -15,19 +15,22 @@
 //   * One thread per CTA issues the unit's cp.async.bulk copies (TMA, one
 //     per array) into a ring of kStages shared-memory buffers, kAhead units
 //     ahead; they complete on the buffer's mbarrier (transaction bytes).
-//   * The CTA updates the unit in place (a thread owns 4-state slices; the
-//     lanes of a channel sum their partial y with shuffles), writes out into
-//     the buffer, and the same thread writes state and out back with bulk
-//     stores.  A buffer is refilled only after the stores that last read it
-//     have finished reading (cp.async.bulk.wait_group.read).
+//   * Each thread updates its 4-state slices of the unit in registers and
+//     writes them straight back to global memory (16-byte streaming stores;
+//     a warp's 32 slices are 512 contiguous bytes); the lanes of a channel
+//     sum their partial y with shuffles and the first writes out.  A warp
+//     arrives on the buffer's "empty" mbarrier once it has read the buffer,
+//     and the refill waits for all warps' arrivals: no CTA-wide barrier per
+//     unit.
 //   * A CTA takes a contiguous run of units in chunk-major order (consecutive
 //     units cover the same channels of successive batch rows), so A and D stay
 //     in registers and are reloaded only when the channel chunk changes.
 // The grid is persistent: up to three 256-thread CTAs per SM.  Every wait on
-// an mbarrier gives up after 200 ms (read from the global timer), sets bit 0
-// of a device status word and leaves the CTA through a block barrier, after
-// letting the copies it already issued land; the host reads the word with
-// ssm_get_device_status.
+// an mbarrier gives up after 200 ms (read from the global timer) and sets bit
+// 0 of a device status word; the warp that saw it (the answer is made
+// warp-uniform) leaves its loop, and the thread that issues the loads first
+// lets the loads it issued land (each wait again bounded); the host reads
+// the word with ssm_get_device_status.
 #include <atomic>
 
 #include "scan_kernels.cuh"
@@ -70,6 +73,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
                  : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
@@ -104,27 +110,16 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_addr(src)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
-// Shared-memory layout of one stage: the unit's state, then x, dt, z and
-// out for its channels, then the batch row's B and C.
+// Shared-memory layout of one stage: the unit's state, then x, dt and z
+// for its channels, then the batch row's B and C.
 template <typename IO, int N>
 struct BulkStage {
     static constexpr int CH = kUnitFloats / N;                       // channels per unit
     static constexpr size_t STATE = (size_t)kUnitFloats * 4;
     static constexpr size_t VEC = (size_t)CH * sizeof(IO);           // one per-channel array
     static constexpr size_t ROW = (size_t)N * sizeof(IO);            // one B or C row
-    static constexpr size_t X = STATE, DT = X + VEC, Z = DT + VEC, OUT = Z + VEC, B = OUT + VEC, C = B + ROW;
+    static constexpr size_t X = STATE, DT = X + VEC, Z = DT + VEC, B = Z + VEC, C = B + ROW;
     static constexpr size_t BYTES = (C + ROW + 127) / 128 * 128;
     static_assert(VEC % 16 == 0 && ROW % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
@@ -134,15 +129,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_units, uint32_t missing_bytes) {
     using io = io_traits<IO>;
     constexpr int N = 4 * G4;                 // states per channel
+    constexpr int kWarps = kThreads / 32;
     using SL = BulkStage<IO, N>;
     constexpr int CH = SL::CH;
     extern __shared__ __align__(128) unsigned char smem[];  // [kStages][SL::BYTES]
-    __shared__ __align__(8) uint64_t bars[kStages];
-    __shared__ int s_abort;
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int64_t Dm = args.dim, Bt = args.batch;
     const IO *pz = static_cast<const IO *>(args.z);
+    IO *pout = static_cast<IO *>(args.out);
     // this CTA's units: a contiguous run, chunk-major (unit u = chunk u / batch,
     // batch row u % batch), so that consecutive units share A and D
     const int64_t per = (total_units + gridDim.x - 1) / gridDim.x;
@@ -151,9 +147,11 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
 
     if (tid == 0) {
 #pragma unroll
-        for (int st = 0; st < kStages; ++st) mbar_init(&bars[st], 1);
+        for (int st = 0; st < kStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], kWarps);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        s_abort = 0;
     }
     __syncthreads();
 
@@ -168,7 +166,7 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
         int nch;
         geom(k, b, c0, nch);
         unsigned char *stg = smem + (size_t)(k % kStages) * SL::BYTES;
-        uint64_t *bar = &bars[k % kStages];
+        uint64_t *bar = &full[k % kStages];
         const uint32_t sb = (uint32_t)nch * N * 4, vb = (uint32_t)nch * sizeof(IO), rb = (uint32_t)SL::ROW;
         const int64_t ch = b * Dm + c0;
         mbar_arrive_expect_tx(bar, sb + vb * (pz ? 3 : 2) + 2 * rb + missing_bytes);
@@ -179,18 +177,27 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
         bulk_load(stg + SL::B, static_cast<const IO *>(args.B) + b * N, rb, bar);
         bulk_load(stg + SL::C, static_cast<const IO *>(args.C) + b * N, rb, bar);
     };
+    int64_t issued = 0;  // thread 0: units whose loads were issued
     if (tid == 0)
-        for (int64_t k = 0; k < kAhead && k < mine; ++k) issue(k);
+        for (; issued < kAhead && issued < mine; ++issued) issue(issued);
 
     float4 av[kPerThread];
     float dv[kPerThread];
     int64_t a_chunk = -1;
-    for (int64_t k = 0; k < mine; ++k) {
+    bool abort = false;
+    int64_t k = 0;
+    for (; k < mine; ++k) {
         if (tid == 0 && k + kAhead < mine) {
-            // the buffer being refilled last held unit k + kAhead - kStages; at
-            // most kStages - kAhead - 1 stores were committed after its stores
-            bulk_wait_read<kStages - kAhead - 1>();
-            issue(k + kAhead);
+            // the buffer being refilled last held unit k + kAhead - kStages:
+            // every warp has arrived once it had read that unit
+            const int64_t j = k + kAhead;
+            if (j >= kStages && !mbar_wait_bounded(&empty[j % kStages], (uint32_t)((j / kStages - 1) & 1))) {
+                atomicOr(&g_device_status, 1u);
+                abort = true;
+            } else {
+                issue(j);
+                issued = j + 1;
+            }
         }
         int64_t b, c0;
         int nch;
@@ -208,9 +215,13 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
             }
         }
         const int st = (int)(k % kStages);
-        if (!mbar_wait_bounded(&bars[st], (uint32_t)((k / kStages) & 1))) {
+        if (!abort && !mbar_wait_bounded(&full[st], (uint32_t)((k / kStages) & 1))) {
             atomicOr(&g_device_status, 1u);
-            s_abort = 1;
+            abort = true;
+        }
+        if (__any_sync(0xffffffffu, abort)) {  // the whole warp leaves together
+            abort = true;
+            break;
         }
         unsigned char *stg = smem + (size_t)st * SL::BYTES;
         float4 *unit = reinterpret_cast<float4 *>(stg);
@@ -219,7 +230,7 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
         const IO *szz = reinterpret_cast<const IO *>(stg + SL::Z);
         const IO *sB = reinterpret_cast<const IO *>(stg + SL::B);
         const IO *sC = reinterpret_cast<const IO *>(stg + SL::C);
-        IO *so = reinterpret_cast<IO *>(stg + SL::OUT);
+        const int64_t ch = b * Dm + c0;
 #pragma unroll
         for (int i = 0; i < kPerThread; ++i) {
             const int sl = tid + i * kThreads;
@@ -241,32 +252,25 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
             }
             y = group_sum<G4>(y);
             if (ok) {
-                unit[sl] = make_float4(h[0], h[1], h[2], h[3]);
+                __stcs(reinterpret_cast<float4 *>(args.state + (ch + c) * N + q * 4), make_float4(h[0], h[1], h[2], h[3]));
                 if (q == 0) {
                     y = fmaf(dv[i], xv, y);
                     if (pz) y *= silu<PRECISE>(io::load_smem(szz + c));
-                    io::store_smem(so + c, y);
+                    io::store(pout + ch + c, y);
                 }
             }
         }
-        // the bulk stores read what the threads wrote through the generic proxy
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        __syncthreads();
-        if (s_abort) {
-            // let the loads already issued land before the buffers go away
-            if (tid == 0)
-                for (int64_t j = k + 1; j <= k + kAhead && j < mine; ++j)
-                    (void)mbar_wait_bounded(&bars[j % kStages], (uint32_t)((j / kStages) & 1));
-            break;
-        }
-        if (tid == 0) {
-            const int64_t ch = b * Dm + c0;
-            bulk_store(args.state + ch * N, unit, (uint32_t)nch * N * 4);
-            bulk_store(static_cast<IO *>(args.out) + ch, so, (uint32_t)nch * sizeof(IO));
-            bulk_commit();
-        }
+        // this warp is done reading the buffer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
-    if (tid == 0) bulk_wait_all();
+    if (tid == 0 && abort) {
+        // let the loads already issued land before the buffers go away
+        for (int64_t j = k; j < issued; ++j)
+            (void)mbar_wait_bounded(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+    }
+    // no warp leaves while loads it did not wait for may still be landing
+    __syncthreads();
 }
 
 template <typename IO, int G4>
