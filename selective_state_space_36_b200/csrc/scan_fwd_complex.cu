@@ -22,6 +22,9 @@
 // size per step; over a state's memory of ~1/(Delta |Re A|) steps it stays
 // far inside the bf16 tier's 1e-3 state bound.  The complex products run on
 // fp32 pairs (f32x2): (re, im) of a state is one register pair.
+#include <atomic>
+
+#include "cp_async.cuh"
 #include "scan_kernels.cuh"
 
 namespace ssm {
@@ -186,6 +189,218 @@ scan_fwd_complex_kernel(const ScanArgs args) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Staged kernel for the common case (bf16 I/O, N = 16, rows of 16-byte
+// multiples): the same four-lane layout with every input brought through
+// shared memory, as in the real staged scan.  Chunks of T = 32 steps of the
+// (batch row, 32-channel) tile move by cp.async three stages deep (u, delta,
+// z tiles and the raw B, C rows); B and C are widened once per chunk to fp32
+// pairs, C with its imaginary part negated so that Re(C h) is one f32x2 FMA.
+// Per 8-step block lane q computes Delta, Delta u of steps 4 j + q (softplus
+// on pairs) and the values go to the other lanes by shuffles; each lane then
+// runs its 4 complex states over the 8 steps, and the per-step partial
+// readouts are reduce-scattered back to the owning lanes, which finish out and
+// write it over the consumed u row of the tile; the chunk's out leaves in
+// 16-byte stores.
+struct CxLayout {
+    static constexpr int G = 4, NS = 4, NSP = 16, CPB = kBlock / G;
+    static constexpr int T = 32, K = 8, KG = K / G, S = 3;
+    static constexpr int ROW = CPB + 8;                     // bf16 tile row, padded by 16 bytes
+    static constexpr int TILE = T * ROW;                    // elements
+    static constexpr int RAW = T * NSP * 2;                 // raw B or C chunk (elements)
+    static constexpr size_t STAGE_BYTES = (3 * (size_t)TILE + 2 * RAW) * 2;
+    static constexpr size_t W_BYTES = 2 * (size_t)T * NSP * sizeof(float2);  // widened B, C
+    static constexpr size_t SMEM = S * STAGE_BYTES + W_BYTES;
+};
+
+__global__ void __launch_bounds__(kBlock, 4)
+scan_fwd_complex_staged_kernel(const ScanArgs args) {
+    using io = io_traits<__nv_bfloat16>;
+    using Lay = CxLayout;
+    constexpr int G = Lay::G, NS = Lay::NS, NSP = Lay::NSP, CPB = Lay::CPB;
+    constexpr int T = Lay::T, K = Lay::K, KG = Lay::KG, S = Lay::S, ROW = Lay::ROW, TILE = Lay::TILE;
+    constexpr int EPV = 8;             // bf16 elements per 16-byte piece
+    constexpr int ROWV = CPB / EPV;    // pieces per tile row
+    extern __shared__ __align__(16) unsigned char smem[];
+    float2 *wB = reinterpret_cast<float2 *>(smem + S * Lay::STAGE_BYTES);  // [T][NSP]
+    float2 *wC = wB + T * NSP;                                              // [T][NSP], (re, -im)
+
+    const int64_t L = args.seqlen, Dm = args.dim;
+    const int tid = threadIdx.x, q = tid % G, grp = tid / G;
+    const int64_t tiles = (Dm + CPB - 1) / CPB;
+    const int64_t b = blockIdx.x / tiles;
+    const int64_t d0 = (blockIdx.x % tiles) * CPB;
+    const int64_t d = d0 + grp;
+    const bool active = d < Dm;
+    const int nchunks = (int)((L + T - 1) / T);
+    using bf = __nv_bfloat16;
+    const bf *pu = static_cast<const bf *>(args.u);
+    const bf *pd = static_cast<const bf *>(args.delta);
+    const bf *pz = static_cast<const bf *>(args.z);
+    const bf *pB = static_cast<const bf *>(args.B);
+    const bf *pC = static_cast<const bf *>(args.C);
+    bf *po = static_cast<bf *>(args.out);
+
+    auto stage_ptr = [&](int s) { return reinterpret_cast<bf *>(smem + s * Lay::STAGE_BYTES); };
+    auto issue = [&](int c) {  // chunk c into stage c % S
+        const int64_t tc = (int64_t)c * T;
+        const int rows = (int)(L - tc < T ? L - tc : T);
+        bf *st = stage_ptr(c % S);
+        bf *su = st, *sd = st + TILE, *sz = st + 2 * TILE, *rb = st + 3 * TILE, *rc = rb + Lay::RAW;
+        for (int p = tid; p < T * ROWV; p += kBlock) {
+            const int r = p / ROWV, v = p % ROWV;
+            const int64_t col = d0 + v * EPV;
+            const bool ok = r < rows && col < Dm;
+            const int64_t go = ok ? (b * L + tc + r) * Dm + col : 0;
+            const int so = r * ROW + v * EPV;
+            cp_async16(su + so, pu + go, ok);
+            cp_async16(sd + so, pd + go, ok);
+            if (pz) cp_async16(sz + so, pz + go, ok);
+        }
+        const int pieces = rows * NSP * 2 / EPV;  // the chunk's B/C rows are contiguous
+        const int64_t gbc = (b * L + tc) * NSP * 2;
+        for (int p = tid; p < pieces; p += kBlock) {
+            cp_async16(rb + p * EPV, pB + gbc + p * EPV, true);
+            cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
+        }
+    };
+
+    // per-lane constants: A of this lane's 4 states (Re scaled for the decay)
+    float are[NS], aim[NS];
+    float2 h2[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int64_t n = (int64_t)(d * NSP + q * NS + i);
+        are[i] = active ? scale_A<false>(args.A[2 * n]) : 0.f;
+        aim[i] = active ? args.A[2 * n + 1] : 0.f;
+        const bool h0 = active && args.last_state;
+        h2[i] = make_float2(h0 ? args.last_state[2 * (b * Dm * NSP + n)] : 0.f,
+                            h0 ? args.last_state[2 * (b * Dm * NSP + n) + 1] : 0.f);
+    }
+    const float bias = (active && args.bias) ? args.bias[d] : 0.f;
+    const float dskip = (active && args.Dskip) ? args.Dskip[d] : 0.f;
+
+#pragma unroll
+    for (int c = 0; c < S - 1; ++c) {
+        if (c < nchunks) issue(c);
+        cp_async_commit();
+    }
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<S - 2>();
+        // chunk c has landed for every thread, and every thread is done with
+        // the stage that chunk c + S - 1 goes to and with the widened rows
+        __syncthreads();
+        if (c + S - 1 < nchunks) issue(c + S - 1);
+        cp_async_commit();
+        const int64_t tc = (int64_t)c * T;
+        const int rows = (int)(L - tc < T ? L - tc : T);
+        bf *st = stage_ptr(c % S);
+        {
+            const bf *rb = st + 3 * TILE, *rc = rb + Lay::RAW;
+            for (int i = 4 * tid; i < T * NSP * 2; i += 4 * kBlock) {  // 2 complex values per thread and pass
+                float v[4], w[4];
+                const bool ok = i / (NSP * 2) < rows;
+                io::load4_smem(rb + i, v);
+                io::load4_smem(rc + i, w);
+                float4 *db = reinterpret_cast<float4 *>(wB) + i / 4, *dc = reinterpret_cast<float4 *>(wC) + i / 4;
+                *db = ok ? make_float4(v[0], v[1], v[2], v[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+                *dc = ok ? make_float4(w[0], -w[1], w[2], -w[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        __syncthreads();
+        bf *su = st + grp + q * ROW, *sd = st + TILE + grp + q * ROW, *sz = st + 2 * TILE + grp + q * ROW;
+        const float4 *wBq = reinterpret_cast<const float4 *>(wB + q * NS);
+        const float4 *wCq = reinterpret_cast<const float4 *>(wC + q * NS);
+
+        auto block = [&](const int k0, const int nrows) {
+            // the step scalars of the owned steps k0 + j G + q
+            float uo[KG], zo[KG], dlo[KG], duo[KG];
+            float so[KG];
+#pragma unroll
+            for (int j = 0; j < KG; ++j) {
+                const int rr = k0 + j * G;
+                uo[j] = io::load_smem(su + rr * ROW);
+                so[j] = io::load_smem(sd + rr * ROW) + bias;
+                zo[j] = pz ? io::load_smem(sz + rr * ROW) : 0.f;
+            }
+            if (args.softplus) {
+                const float2 sp = softplus2_fast(make_float2(so[0], so[1]));
+                dlo[0] = sp.x;
+                dlo[1] = sp.y;
+            } else {
+#pragma unroll
+                for (int j = 0; j < KG; ++j) dlo[j] = so[j];
+            }
+#pragma unroll
+            for (int j = 0; j < KG; ++j) {
+                if (k0 + j * G + q >= nrows || !active) dlo[j] = 0.f;
+                duo[j] = dlo[j] * uo[j];
+            }
+            float dl[K], du[K];
+            exchange_steps<K, G>(dlo, duo, dl, du);
+            float yp[K];
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int row = (k0 + k) * (NSP / 2);  // float4 index of the row (2 complex values each)
+                const float2 du2 = make_float2(du[k], du[k]);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i2 = 0; i2 < NS / 2; ++i2) {
+                    const float4 b4 = wBq[row + i2], c4 = wCq[row + i2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int i = 2 * i2 + e2;
+                        const float2 bv = e2 ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
+                        const float2 cv = e2 ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+                        const float e = ex2_approx(dl[k] * are[i]);
+                        float sn, cs;
+                        phase<false>(dl[k] * aim[i], sn, cs);
+                        const float ec = e * cs, es = e * sn;
+                        float2 t = fma2(make_float2(ec, ec), h2[i], mul2(du2, bv));
+                        t.x = fmaf(-es, h2[i].y, t.x);
+                        t.y = fmaf(es, h2[i].x, t.y);
+                        h2[i] = t;
+                        acc = fma2(cv, t, acc);  // (cr hr, -ci hi)
+                    }
+                }
+                yp[k] = acc.x + acc.y;
+            }
+            float yo[KG];
+            reduce_scatter_steps<K, G>(yp, yo, q);
+#pragma unroll
+            for (int j = 0; j < KG; ++j) {
+                const int rr = k0 + j * G;
+                float y = fmaf(dskip, uo[j], yo[j]);
+                if (pz) y *= silu<false>(zo[j]);
+                io::store_smem(su + rr * ROW, y);  // out over the consumed u
+            }
+        };
+        if (rows == T) {
+#pragma unroll 1
+            for (int k0 = 0; k0 < T; k0 += K) block(k0, T);
+        } else {
+            for (int k0 = 0; k0 < rows; k0 += K) block(k0, rows);
+        }
+        __syncthreads();
+        // the chunk's out leaves in 16-byte pieces
+        for (int p = tid; p < T * ROWV; p += kBlock) {
+            const int r = p / ROWV, v = p % ROWV;
+            const int64_t col = d0 + v * EPV;
+            if (r < rows && col < Dm)
+                __stcs(reinterpret_cast<uint4 *>(po + (b * L + tc + r) * Dm + col),
+                       *reinterpret_cast<const uint4 *>(st + r * ROW + v * EPV));
+        }
+    }
+    cp_async_wait<0>();
+    if (!active || !args.last_state) return;
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int64_t n = (int64_t)(d * NSP + q * NS + i);
+        args.last_state[2 * (b * Dm * NSP + n)] = h2[i].x;
+        args.last_state[2 * (b * Dm * NSP + n) + 1] = h2[i].y;
+    }
+}
+
 template <typename IO, int NS>
 cudaError_t launch_ns(const ScanArgs &a, cudaStream_t st) {
     constexpr bool P = std::is_same<IO, float>::value;
@@ -198,7 +413,29 @@ cudaError_t launch_ns(const ScanArgs &a, cudaStream_t st) {
 
 int64_t scan_complex_channels_per_block() { return kCCPB; }
 
+bool scan_complex_staged_eligible(const ScanArgs &a, bool bf16) {
+    auto al = [](const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) % 16) == 0; };
+    return bf16 && a.dstate == CxLayout::NSP && (a.dim * 2) % 16 == 0 && al(a.u) && al(a.delta) && al(a.z) &&
+           al(a.B) && al(a.C) && al(a.out);
+}
+
 cudaError_t launch_scan_complex(const ScanArgs &a, bool bf16, cudaStream_t st) {
+    if (scan_complex_staged_eligible(a, bf16)) {
+        static std::atomic<unsigned long long> configured{0};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const unsigned long long bit = 1ull << (dev & 63);
+        if (!(configured.load(std::memory_order_relaxed) & bit)) {
+            e = cudaFuncSetAttribute(scan_fwd_complex_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)CxLayout::SMEM);
+            if (e != cudaSuccess) return e;
+            configured.fetch_or(bit, std::memory_order_relaxed);
+        }
+        const int64_t tiles = (a.dim + CxLayout::CPB - 1) / CxLayout::CPB;
+        scan_fwd_complex_staged_kernel<<<dim3((unsigned)(a.batch * tiles)), kBlock, CxLayout::SMEM, st>>>(a);
+        return cudaGetLastError();
+    }
     const int ns = a.dstate <= 16 ? 4 : (a.dstate <= 32 ? 8 : 16);
     if (bf16) {
         if (ns == 4) return launch_ns<__nv_bfloat16, 4>(a, st);

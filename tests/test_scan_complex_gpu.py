@@ -112,3 +112,32 @@ def test_complex_mamba130m_shape(lib):
     # the 130M-layer shape with S4D-Lin A, against the oracle on 64 channels
     cfg = I.MAMBA130M.with_(dim=64)
     _check(lib, "bf16", cfg.batch, cfg.seqlen, cfg.dim, cfg.dstate, cfg.seed)
+
+
+# The staged kernel (bf16, N = 16, dim a multiple of 8): several chunks of
+# 32 steps, ragged chunk and tile tails, channels past the last full tile.
+@pytest.mark.parametrize("batch,L,dim", [(1, 1, 8), (2, 31, 40), (1, 33, 64), (2, 100, 72), (1, 257, 96)])
+def test_complex_staged_shapes(lib, batch, L, dim):
+    _check(lib, "bf16", batch, L, dim, 16, 70 + L, h0_sigma=0.4)
+
+
+@pytest.mark.parametrize("opt", [dict(has_z=False), dict(has_d=False), dict(has_bias=False),
+                                 dict(has_z=False, has_d=False, has_bias=False), dict(h0_sigma=None),
+                                 # Delta as given: small steps of either sign, no bias
+                                 dict(softplus=False, has_bias=False, delta_sigma=0.05)])
+def test_complex_staged_optional_inputs(lib, opt):
+    _check(lib, "bf16", 2, 77, 48, 16, 9, **opt)
+
+
+def test_complex_staged_resume_equals_one_pass(lib):
+    # splits at multiples of 8 steps keep every step's owning lane, so the
+    # two calls reproduce the one-pass result bit for bit
+    cfg = I.ScanConfig("cx", 2, 136, 64, 16, io="bf16", seed=14, h0_sigma=0.5)
+    x = I.complex_scan_inputs(cfg)
+    out_full, st_full = _gpu(lib, x, "bf16")
+    for cut in (40, 64):
+        o1, st = _gpu(lib, I.complex_scan_inputs(cfg, 0, cut), "bf16")
+        o2, st = _gpu(lib, I.complex_scan_inputs(cfg, cut, 136), "bf16", state=st)
+        got = np.concatenate([T.from_dev(o1), T.from_dev(o2)], axis=1)
+        assert np.array_equal(got, T.from_dev(out_full))
+        assert torch.equal(st, st_full)
