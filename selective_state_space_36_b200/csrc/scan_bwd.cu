@@ -359,7 +359,10 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
 
     const int64_t L = args.seqlen, Dm = args.dim;
     const int N = args.dstate;
-    const int tid = threadIdx.x, q = tid % G, grp = tid / G;
+    // lane c + 8 q of warp w: state slot q of channel 8 w + c (the 8 lanes of
+    // a quarter-warp hold 8 channels and read the same B/C address)
+    constexpr int LS = 8;  // lane stride of a channel's group
+    const int tid = threadIdx.x, q = (tid & 31) / LS, grp = (tid >> 5) * LS + (tid & (LS - 1));
     const int64_t tiles = (Dm + CPB - 1) / CPB;
     const int64_t b = blockIdx.x / tiles;
     const int64_t d0 = (blockIdx.x % tiles) * CPB;
@@ -467,7 +470,7 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
         IO *su = st + grp + q * ROW, *sd = st + TILE + grp + q * ROW;
         IO *sz = st + 2 * TILE + grp + q * ROW, *sg = st + 3 * TILE + grp + q * ROW;
         const float *fBq = fB + q * NS, *fCq = fC + q * NS;
-        float *sredq = sred + grp * NSP + q * NS;
+        float *sredq = sred + q * (CPB * NS) + grp * NS;  // [q][channel][4] slabs
 
         // One sub-chunk of KC steps starting at chunk row k0 (nrows: the rows
         // of this chunk; the constant T for full chunks).
@@ -527,7 +530,7 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             float2 hs[KC][NS / 2];
             {
                 float dl[KC], du[KC];
-                exchange_steps<KC, G>(dlo, duo, dl, du);
+                exchange_steps<KC, G, LS>(dlo, duo, dl, du);
                 float2 h2[NS / 2];
 #pragma unroll
                 for (int p = 0; p < NS / 2; ++p) h2[p] = hc[p];
@@ -549,8 +552,7 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             // ---- adjoint recurrence, last step first, G steps at a time (the
             // step scalars come from their owning lanes again, rather than
             // being held through the sweep)
-            const unsigned gbase = (threadIdx.x & 31u) & ~(unsigned)(G - 1);
-            const unsigned gmask = ((1u << G) - 1u) << gbase;
+            const unsigned gbase = LaneGroup<G, LS>::base(), gmask = LaneGroup<G, LS>::mask();
 #pragma unroll
             for (int jg = KG - 1; jg >= 0; --jg) {
                 float ddl_p[G], dub_p[G], y_p[G];
@@ -559,9 +561,9 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                     const int k = jg * G + i;
                     const float4 bv = *reinterpret_cast<const float4 *>(fBq + (k0 + k) * NSP);
                     const float4 cv = *reinterpret_cast<const float4 *>(fCq + (k0 + k) * NSP);
-                    const float dyk = __shfl_sync(gmask, dyo[jg], gbase + i);
-                    const float dlk = __shfl_sync(gmask, dlo[jg], gbase + i);
-                    const float duk = __shfl_sync(gmask, duo[jg], gbase + i);
+                    const float dyk = __shfl_sync(gmask, dyo[jg], gbase + i * LS);
+                    const float dlk = __shfl_sync(gmask, dlo[jg], gbase + i * LS);
+                    const float duk = __shfl_sync(gmask, duo[jg], gbase + i * LS);
                     const float2 dy2 = make_float2(dyk, dyk), dl2 = make_float2(dlk, dlk);
                     const float2 du2 = make_float2(duk, duk);
                     float2 accy = make_float2(0.f, 0.f), accd = accy, accb = accy, pc[NS / 2], pb[NS / 2];
@@ -600,11 +602,11 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
                 // lane q keeps the sums of step jg G + q (the step it owns)
                 // and finishes that step's du, ddelta, dz
                 float r[1];
-                reduce_scatter_steps<G, G>(ddl_p, r, q);
+                reduce_scatter_steps<G, G, LS>(ddl_p, r, q);
                 const float ddl_o = r[0];
-                reduce_scatter_steps<G, G>(dub_p, r, q);
+                reduce_scatter_steps<G, G, LS>(dub_p, r, q);
                 const float dub = r[0];
-                reduce_scatter_steps<G, G>(y_p, r, q);
+                reduce_scatter_steps<G, G, LS>(y_p, r, q);
                 const float y_o = r[0];
                 const int rr = k0 + jg * G;
                 if (rr + q < nrows && active) {
@@ -624,21 +626,23 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
             }
             // ---- dB, dC of the sub-chunk: 64 (which, step, quad) sums over
             // the block's 32 channels, two threads (adjacent lanes) per sum,
-            // 16 channels each; the odd thread starts one channel later so
-            // that the two halves of a quarter-warp fall in different banks
+            // 16 channels each; thread (quad nq, half part) starts 2 nq + part
+            // channels in, so that the 8 threads of a quarter-warp fall in 8
+            // different banks
             __syncthreads();
             {
                 const int task = tid >> 1, part = tid & 1;
                 const int nq = task % NQ;
                 const int kk = (task / NQ) % KC;
                 const int which = task / (NQ * KC);  // 0: dC, 1: dB
-                const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) + nq +
-                                    part * (CPB / 2) * NQ;
+                const float4 *col = reinterpret_cast<const float4 *>(sred + (which * KC + kk) * KSTRIDE) +
+                                    nq * CPB + part * (CPB / 2);
+                const int rot = 2 * nq + part;
                 float2 a01 = make_float2(0.f, 0.f), a23 = a01, b01 = a01, b23 = a01;
 #pragma unroll
                 for (int cc = 0; cc < CPB / 2; cc += 2) {
-                    const float4 v = col[((cc + part) & (CPB / 2 - 1)) * NQ];
-                    const float4 w = col[((cc + 1 + part) & (CPB / 2 - 1)) * NQ];
+                    const float4 v = col[(cc + rot) & (CPB / 2 - 1)];
+                    const float4 w = col[(cc + 1 + rot) & (CPB / 2 - 1)];
                     a01 = add2(a01, make_float2(v.x, v.y));
                     a23 = add2(a23, make_float2(v.z, v.w));
                     b01 = add2(b01, make_float2(w.x, w.y));
@@ -688,8 +692,8 @@ scan_bwd_staged_kernel(const ScanBwdArgs args) {
     }
     cp_async_wait<0>();
     // dD and dbias were accumulated by the owner of each step: sum the group
-    dD_acc = group_sum<G>(dD_acc);
-    dbias_acc = group_sum<G>(dbias_acc);
+    dD_acc = group_sum<G, LS>(dD_acc);
+    dbias_acc = group_sum<G, LS>(dbias_acc);
     if (!active) return;
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) {

@@ -252,14 +252,33 @@ __device__ __forceinline__ float scale_A(float a) {
     return PRECISE ? a : a * kLog2e;
 }
 
-// Sum of a value over the G consecutive lanes that share one channel.
-template <int G>
+// The G lanes that share one channel: lanes base + i STRIDE, i < G, of the
+// warp (STRIDE 1: G consecutive lanes; STRIDE 8 with G = 4: lanes c, c + 8,
+// c + 16, c + 24, so that the 8 lanes of a quarter-warp belong to 8 channels
+// and read the same shared-memory address when they load B or C -- two L1
+// wavefronts per 128-bit load instead of four).
+template <int G, int STRIDE>
+struct LaneGroup {
+    static_assert(STRIDE == 1 || STRIDE * G == 32, "consecutive lanes, or a group spread over the warp");
+    static __device__ __forceinline__ unsigned base() {
+        const unsigned lane = threadIdx.x & 31u;
+        return STRIDE == 1 ? (lane & ~(unsigned)(G - 1)) : (lane % STRIDE);
+    }
+    static __device__ __forceinline__ unsigned mask() {
+        unsigned m = 0;
+#pragma unroll
+        for (int i = 0; i < G; ++i) m |= 1u << (i * STRIDE);
+        return G == 32 ? 0xffffffffu : (m << base());
+    }
+};
+
+// Sum of a value over the G lanes that share one channel.
+template <int G, int STRIDE = 1>
 __device__ __forceinline__ float group_sum(float v) {
     if (G > 1) {
-        const unsigned lane = threadIdx.x & 31u;
-        const unsigned mask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(unsigned)(G - 1));
+        const unsigned mask = LaneGroup<G, STRIDE>::mask();
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
+        for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o * STRIDE);
     }
     return v;
 }
@@ -304,7 +323,7 @@ __device__ __forceinline__ double group_sum_d(double v) {
 // Lane q of a group of G consecutive lanes holds the scalars of steps
 // q, q + G, q + 2G, ... (own[j] is step j G + q); afterwards every lane of
 // the group holds all K steps.
-template <int K, int G>
+template <int K, int G, int STRIDE = 1>
 __device__ __forceinline__ void exchange_steps(const float (&dlo)[K / G], const float (&duo)[K / G],
                                                float (&dl)[K], float (&du)[K]) {
     if (G == 1) {
@@ -312,13 +331,11 @@ __device__ __forceinline__ void exchange_steps(const float (&dlo)[K / G], const 
         for (int k = 0; k < K; ++k) { dl[k] = dlo[k]; du[k] = duo[k]; }
         return;
     }
-    const unsigned lane = threadIdx.x & 31u;
-    const unsigned base = lane & ~(unsigned)(G - 1);
-    const unsigned mask = ((1u << G) - 1u) << base;
+    const unsigned base = LaneGroup<G, STRIDE>::base(), mask = LaneGroup<G, STRIDE>::mask();
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-        dl[k] = __shfl_sync(mask, dlo[k / G], base + k % G);
-        du[k] = __shfl_sync(mask, duo[k / G], base + k % G);
+        dl[k] = __shfl_sync(mask, dlo[k / G], base + (k % G) * STRIDE);
+        du[k] = __shfl_sync(mask, duo[k / G], base + (k % G) * STRIDE);
     }
 }
 
@@ -326,29 +343,28 @@ __device__ __forceinline__ void exchange_steps(const float (&dlo)[K / G], const 
 // group holds the full sums of its own steps, yo[j] = sum over the group of
 // y[j G + q] (a butterfly reduce-scatter: log2 G rounds, each halving the
 // steps a lane keeps).
-template <int K, int G>
+template <int K, int G, int STRIDE = 1>
 __device__ __forceinline__ void reduce_scatter_steps(const float (&y)[K], float (&yo)[K / G], int q) {
     if (G == 1) {
 #pragma unroll
         for (int k = 0; k < K; ++k) yo[k] = y[k];
         return;
     }
-    const unsigned lane = threadIdx.x & 31u;
-    const unsigned mask = ((1u << G) - 1u) << (lane & ~(unsigned)(G - 1));
+    const unsigned mask = LaneGroup<G, STRIDE>::mask();
 #pragma unroll
     for (int j = 0; j < K / G; ++j) {
         if (G == 2) {
             const float keep = q ? y[2 * j + 1] : y[2 * j];
             const float send = q ? y[2 * j] : y[2 * j + 1];
-            yo[j] = keep + __shfl_xor_sync(mask, send, 1);
+            yo[j] = keep + __shfl_xor_sync(mask, send, STRIDE);
         } else {  // G == 4
             const bool hi = (q & 2) != 0;
             const float k0 = hi ? y[4 * j + 2] : y[4 * j + 0], k1 = hi ? y[4 * j + 3] : y[4 * j + 1];
             const float s0 = hi ? y[4 * j + 0] : y[4 * j + 2], s1 = hi ? y[4 * j + 1] : y[4 * j + 3];
-            const float m0 = k0 + __shfl_xor_sync(mask, s0, 2);
-            const float m1 = k1 + __shfl_xor_sync(mask, s1, 2);
+            const float m0 = k0 + __shfl_xor_sync(mask, s0, 2 * STRIDE);
+            const float m1 = k1 + __shfl_xor_sync(mask, s1, 2 * STRIDE);
             const bool odd = (q & 1) != 0;
-            yo[j] = (odd ? m1 : m0) + __shfl_xor_sync(mask, odd ? m0 : m1, 1);
+            yo[j] = (odd ? m1 : m0) + __shfl_xor_sync(mask, odd ? m0 : m1, STRIDE);
         }
     }
 }
