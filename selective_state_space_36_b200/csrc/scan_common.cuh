@@ -256,7 +256,7 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
 }
 
 // exchange_steps / reduce_scatter_steps for CPL channels per lane.
-template <int K, int G, int CPL>
+template <int K, int G, int CPL, int STRIDE = 1>
 __device__ __forceinline__ void exchange_steps_cpl(const float (&dlo)[K / G][CPL],
                                                    const float (&duo)[K / G][CPL],
                                                    float (&dl)[K][CPL], float (&du)[K][CPL]) {
@@ -265,13 +265,13 @@ __device__ __forceinline__ void exchange_steps_cpl(const float (&dlo)[K / G][CPL
         float a[K / G], bo[K / G], x[K], z[K];
 #pragma unroll
         for (int j = 0; j < K / G; ++j) { a[j] = dlo[j][c]; bo[j] = duo[j][c]; }
-        exchange_steps<K, G>(a, bo, x, z);
+        exchange_steps<K, G, STRIDE>(a, bo, x, z);
 #pragma unroll
         for (int k = 0; k < K; ++k) { dl[k][c] = x[k]; du[k][c] = z[k]; }
     }
 }
 
-template <int K, int G, int CPL>
+template <int K, int G, int CPL, int STRIDE = 1>
 __device__ __forceinline__ void reduce_scatter_steps_cpl(const float (&y)[K][CPL], float (&yo)[K / G][CPL],
                                                          int q) {
 #pragma unroll
@@ -279,7 +279,7 @@ __device__ __forceinline__ void reduce_scatter_steps_cpl(const float (&y)[K][CPL
         float a[K], o[K / G];
 #pragma unroll
         for (int k = 0; k < K; ++k) a[k] = y[k][c];
-        reduce_scatter_steps<K, G>(a, o, q);
+        reduce_scatter_steps<K, G, STRIDE>(a, o, q);
 #pragma unroll
         for (int j = 0; j < K / G; ++j) yo[j][c] = o[j];
     }

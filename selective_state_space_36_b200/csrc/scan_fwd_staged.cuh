@@ -169,8 +169,14 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     const int64_t L = args.seqlen, Dm = args.dim;
     const int N = args.dstate;
     const int tid = threadIdx.x % TPB;
-    const int q = tid % G;
-    const int grp = tid / G;
+    // With four lanes per channel they sit 8 apart (lane c + 8 q of a warp:
+    // state slice q of the warp's channel c), so that the 8 lanes of a
+    // quarter-warp read one B/C address (two L1 wavefronts per 128-bit load
+    // instead of four); with one or two lanes they are adjacent.
+    constexpr int LS = G == 4 ? 8 : 1;
+    static_assert(G != 4 || TPB % 32 == 0, "four-lane groups spread over whole warps");
+    const int q = G == 4 ? (tid & 31) / LS : tid % G;
+    const int grp = G == 4 ? (tid >> 5) * LS + (tid & (LS - 1)) : tid / G;
     const int64_t tiles = (Dm + CPB - 1) / CPB;
     const int64_t b = unit / tiles;
     const int64_t d0 = (unit % tiles) * CPB;
@@ -343,7 +349,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                     }
                 }
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
-                exchange_steps_cpl<KSTEP, G, CPL>(dlo, duo, dl, du);
+                exchange_steps_cpl<KSTEP, G, CPL, LS>(dlo, duo, dl, du);
                 recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, MODE != kCkpt>(
                     dl, du, fBq + r0 * NSP, fCq + r0 * NSP, NSP, A2, h2, y, invA2);
                 if (MODE == kCkpt) {
@@ -355,7 +361,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                         for (int cc = 0; cc < CPL; ++cc) dsum[cc] += (double)dlo[j][cc];
                 } else {
                     float yo[KG][CPL];
-                    reduce_scatter_steps_cpl<KSTEP, G, CPL>(y, yo, q);
+                    reduce_scatter_steps_cpl<KSTEP, G, CPL, LS>(y, yo, q);
 #pragma unroll
                     for (int j = 0; j < KG; ++j) {
                         const int rr = r0 + j * G;
@@ -385,7 +391,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     cp_async_wait<0>();
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
-        const double ds = MODE == kSegAgg ? group_sum_d<G>(dsum[c]) : 0.0;
+        const double ds = MODE == kSegAgg ? group_sum_d<G, LS>(dsum[c]) : 0.0;
         float h[NS];
 #pragma unroll
         for (int p = 0; p < NS / 2; ++p) {

@@ -309,13 +309,12 @@ __device__ __forceinline__ float2 zoh_phi2(float2 z, float2 a, float2 inv_a, flo
 }
 __device__ __forceinline__ float zoh_phi_precise(float z) { return z == 0.f ? 1.f : expm1f(z) / z; }
 
-template <int G>
+template <int G, int STRIDE = 1>
 __device__ __forceinline__ double group_sum_d(double v) {
     if (G > 1) {
-        const unsigned lane = threadIdx.x & 31u;
-        const unsigned mask = ((1u << G) - 1u) << (lane & ~(unsigned)(G - 1));
+        const unsigned mask = LaneGroup<G, STRIDE>::mask();
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
+        for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o * STRIDE);
     }
     return v;
 }
