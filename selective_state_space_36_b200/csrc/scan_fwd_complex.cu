@@ -226,7 +226,10 @@ scan_fwd_complex_staged_kernel(const ScanArgs args) {
     float2 *wC = wB + T * NSP;                                              // [T][NSP], (re, -im)
 
     const int64_t L = args.seqlen, Dm = args.dim;
-    const int tid = threadIdx.x, q = tid % G, grp = tid / G;
+    // lane c + 8 q of warp w: complex states [4 q, 4 q + 4) of channel 8 w + c
+    // (a quarter-warp's 8 lanes read one B/C address)
+    constexpr int LS = 8;
+    const int tid = threadIdx.x, q = (tid & 31) / LS, grp = (tid >> 5) * LS + (tid & (LS - 1));
     const int64_t tiles = (Dm + CPB - 1) / CPB;
     const int64_t b = blockIdx.x / tiles;
     const int64_t d0 = (blockIdx.x % tiles) * CPB;
@@ -337,7 +340,7 @@ scan_fwd_complex_staged_kernel(const ScanArgs args) {
                 duo[j] = dlo[j] * uo[j];
             }
             float dl[K], du[K];
-            exchange_steps<K, G>(dlo, duo, dl, du);
+            exchange_steps<K, G, LS>(dlo, duo, dl, du);
             float yp[K];
 #pragma unroll
             for (int k = 0; k < K; ++k) {
@@ -366,7 +369,7 @@ scan_fwd_complex_staged_kernel(const ScanArgs args) {
                 yp[k] = acc.x + acc.y;
             }
             float yo[KG];
-            reduce_scatter_steps<K, G>(yp, yo, q);
+            reduce_scatter_steps<K, G, LS>(yp, yo, q);
 #pragma unroll
             for (int j = 0; j < KG; ++j) {
                 const int rr = k0 + j * G;
