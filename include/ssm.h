@@ -345,10 +345,10 @@ ssm_status ssm_selective_state_update(ssm_dims dims, ssm_dtype io, float *state,
  * Supported: io = SSM_BF16, headdim = 64, dstate = 64 or 128, heads a
  * multiple of groups, x, z, B, C, out 16-byte aligned (SSM_ERR_UNSUPPORTED
  * otherwise).  Arithmetic: products on the tensor cores with bf16 operands
- * and fp32 accumulation; the masked intra-chunk matrix is rounded to bf16;
- * the state is carried in fp32, and both products that involve it (the
- * chunk's state update and the inter-chunk output) take a two-term operand,
- * a bf16 high part plus the bf16 rounding of the rest.  A wait inside
+ * and fp32 accumulation; the state is carried in fp32; three operands take
+ * two terms, a bf16 high part plus the bf16 rounding of the rest: the masked
+ * intra-chunk matrix, the weighted x of the chunk's state update, and the
+ * carried state in the inter-chunk output.  A wait inside
  * the kernel that runs out (2 s) sets bit 1 of the device status word
  * (ssm_get_device_status); the outputs are then not valid.
  */

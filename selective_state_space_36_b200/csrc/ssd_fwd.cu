@@ -19,19 +19,21 @@
 // operands in shared memory and fp32 accumulators in tensor memory:
 //   C B^T      (128 x 128, K = dstate)    -> masked in registers
 //   M X        (128 x headdim, K = 128)
-//   C H^T      (128 x headdim, K = dstate)
+//   C H^T      (128 x headdim, K = dstate; both terms of H as one N = 128 product)
 //   B^T Xw     (dstate x headdim, K = 128)
 // Three of them take two-term operands -- a bf16 high part plus the bf16
 // rounding of the rest -- so that the result keeps fp32-level accuracy:
 // Xw = w o X (one bf16 term would leave ~3e-3 relative error in the state),
 // the carried state H in C H^T, and the masked matrix M (one bf16 term each
 // measured 2.4e-2 output error on the full workload, above the 2e-2 bound).
-// Tiles of C, B, X come in by TMA (cp.async.bulk.tensor, 128-byte swizzle,
-// no multicast), two chunks deep.  One CTA of 512 threads per (b, h):
-// thread (warp w, lane l) owns TMEM lane / tile row r = 32 (w % 4) + l and the
-// quarter w / 4 of the columns; thread 0 issues the copies and the MMAs.
-// Every wait is bounded; a wait that runs out sets bit 1 of the device
-// status word and the CTA stops after its in-flight work.
+// Tiles of C, B, X and z come in by TMA (cp.async.bulk.tensor, 128-byte
+// swizzle, no multicast), C, B, X two chunks deep, and out leaves by TMA
+// store.  One CTA per (b, h), warp specialised: 16 element-wise warps (thread
+// (warp w, lane l) owns TMEM lane / tile row r = 32 (w % 4) + l and the
+// quarter w / 4 of the columns) and one warp that issues the copies and the
+// products (see the layout notes above the kernel).  Every wait is bounded; a
+// wait that runs out sets bit 1 of the device status word and the CTA stops
+// after its in-flight work.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
