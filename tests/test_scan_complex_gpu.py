@@ -141,3 +141,28 @@ def test_complex_staged_resume_equals_one_pass(lib):
         got = np.concatenate([T.from_dev(o1), T.from_dev(o2)], axis=1)
         assert np.array_equal(got, T.from_dev(out_full))
         assert torch.equal(st, st_full)
+
+
+@pytest.mark.slow
+def test_complex_mamba130m_full_sampled_channels(lib):
+    """The benchmark's launch (batch 8, L 2048, dim 1536, N 16, bf16: the
+    staged kernel) against the oracle on 12 channels spread over the 48
+    32-channel tiles, every batch row."""
+    cfg = I.MAMBA130M.with_(h0_sigma=0.3)
+    x = I.complex_scan_inputs(cfg)
+    out, state = _gpu(lib, x, "bf16")
+    sel = np.array([0, 1, 31, 100, 257, 511, 640, 777, 1023, 1200, 1502, 1535])
+    xs = dict(x)
+    for k in ("u", "delta", "z"):
+        xs[k] = np.ascontiguousarray(x[k][:, :, sel])
+    for k in ("D", "delta_bias"):
+        xs[k] = np.ascontiguousarray(x[k][sel])
+    xs["A"] = np.ascontiguousarray(x["A"][sel])
+    xs["h0"] = np.ascontiguousarray(x["h0"][:, sel])
+    ref_out, ref_state = _oracle(xs, "bf16")
+    idx = torch.as_tensor(sel, device="cuda")
+    T.check_out(T.from_dev(out[:, :, idx]), ref_out, "bf16")
+    st = T.from_dev(state[:, idx])
+    got_state = st[..., 0] + 1j * st[..., 1]
+    T.check_state(np.abs(got_state - ref_state) + np.abs(ref_state), np.abs(ref_state), "bf16",
+                  what="last_state (complex)")
