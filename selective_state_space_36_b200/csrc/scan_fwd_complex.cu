@@ -202,9 +202,15 @@ scan_fwd_complex_kernel(const ScanArgs args) {
 // readouts are reduce-scattered back to the owning lanes, which finish out and
 // write it over the consumed u row of the tile; the chunk's out leaves in
 // 16-byte stores.
+#ifndef SSM_COMPLEX_LANES
+#define SSM_COMPLEX_LANES 4
+#endif
+template <int GL>  // lanes per channel: 4 (4 complex states each) or 8 (2 each)
 struct CxLayout {
-    static constexpr int G = 4, NS = 4, NSP = 16, CPB = kBlock / G;
+    static constexpr int G = GL, NS = 16 / GL, NSP = 16, CPB = kBlock / G;
     static constexpr int T = 32, K = 8, KG = K / G, S = 3;
+    static constexpr int LS = 32 / G;                       // lane stride of a channel's group
+    static constexpr int MIN_BLOCKS = G == 8 ? 6 : 4;
     static constexpr int ROW = CPB + 8;                     // bf16 tile row, padded by 16 bytes
     static constexpr int TILE = T * ROW;                    // elements
     static constexpr int RAW = T * NSP * 2;                 // raw B or C chunk (elements)
@@ -213,10 +219,11 @@ struct CxLayout {
     static constexpr size_t SMEM = S * STAGE_BYTES + W_BYTES;
 };
 
-__global__ void __launch_bounds__(kBlock, 4)
+template <int GL>
+__global__ void __launch_bounds__(kBlock, CxLayout<GL>::MIN_BLOCKS)
 scan_fwd_complex_staged_kernel(const ScanArgs args) {
     using io = io_traits<__nv_bfloat16>;
-    using Lay = CxLayout;
+    using Lay = CxLayout<GL>;
     constexpr int G = Lay::G, NS = Lay::NS, NSP = Lay::NSP, CPB = Lay::CPB;
     constexpr int T = Lay::T, K = Lay::K, KG = Lay::KG, S = Lay::S, ROW = Lay::ROW, TILE = Lay::TILE;
     constexpr int EPV = 8;             // bf16 elements per 16-byte piece
@@ -226,9 +233,9 @@ scan_fwd_complex_staged_kernel(const ScanArgs args) {
     float2 *wC = wB + T * NSP;                                              // [T][NSP], (re, -im)
 
     const int64_t L = args.seqlen, Dm = args.dim;
-    // lane c + 8 q of warp w: complex states [4 q, 4 q + 4) of channel 8 w + c
-    // (a quarter-warp's 8 lanes read one B/C address)
-    constexpr int LS = 8;
+    // lane c + LS q of warp w: complex states [NS q, NS q + NS) of channel
+    // LS w + c (a quarter-warp's 8 lanes read at most two B/C addresses)
+    constexpr int LS = Lay::LS;
     const int tid = threadIdx.x, q = (tid & 31) / LS, grp = (tid >> 5) * LS + (tid & (LS - 1));
     const int64_t tiles = (Dm + CPB - 1) / CPB;
     const int64_t b = blockIdx.x / tiles;
@@ -327,9 +334,14 @@ scan_fwd_complex_staged_kernel(const ScanArgs args) {
                 zo[j] = pz ? io::load_smem(sz + rr * ROW) : 0.f;
             }
             if (args.softplus) {
-                const float2 sp = softplus2_fast(make_float2(so[0], so[1]));
-                dlo[0] = sp.x;
-                dlo[1] = sp.y;
+                if constexpr (KG == 2) {
+                    const float2 sp = softplus2_fast(make_float2(so[0], so[1]));
+                    dlo[0] = sp.x;
+                    dlo[1] = sp.y;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < KG; ++j) dlo[j] = softplus<false>(so[j]);
+                }
             } else {
 #pragma unroll
                 for (int j = 0; j < KG; ++j) dlo[j] = so[j];
@@ -418,25 +430,26 @@ int64_t scan_complex_channels_per_block() { return kCCPB; }
 
 bool scan_complex_staged_eligible(const ScanArgs &a, bool bf16) {
     auto al = [](const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) % 16) == 0; };
-    return bf16 && a.dstate == CxLayout::NSP && (a.dim * 2) % 16 == 0 && al(a.u) && al(a.delta) && al(a.z) &&
-           al(a.B) && al(a.C) && al(a.out);
+    return bf16 && a.dstate == CxLayout<SSM_COMPLEX_LANES>::NSP && (a.dim * 2) % 16 == 0 && al(a.u) &&
+           al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out);
 }
 
 cudaError_t launch_scan_complex(const ScanArgs &a, bool bf16, cudaStream_t st) {
     if (scan_complex_staged_eligible(a, bf16)) {
+        using Lay = CxLayout<SSM_COMPLEX_LANES>;
+        auto kern = scan_fwd_complex_staged_kernel<SSM_COMPLEX_LANES>;
         static std::atomic<unsigned long long> configured{0};
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
         const unsigned long long bit = 1ull << (dev & 63);
         if (!(configured.load(std::memory_order_relaxed) & bit)) {
-            e = cudaFuncSetAttribute(scan_fwd_complex_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)CxLayout::SMEM);
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM);
             if (e != cudaSuccess) return e;
             configured.fetch_or(bit, std::memory_order_relaxed);
         }
-        const int64_t tiles = (a.dim + CxLayout::CPB - 1) / CxLayout::CPB;
-        scan_fwd_complex_staged_kernel<<<dim3((unsigned)(a.batch * tiles)), kBlock, CxLayout::SMEM, st>>>(a);
+        const int64_t tiles = (a.dim + Lay::CPB - 1) / Lay::CPB;
+        kern<<<dim3((unsigned)(a.batch * tiles)), kBlock, Lay::SMEM, st>>>(a);
         return cudaGetLastError();
     }
     const int ns = a.dstate <= 16 ? 4 : (a.dstate <= 32 ? 8 : 16);

@@ -356,6 +356,24 @@ __device__ __forceinline__ void reduce_scatter_steps(const float (&y)[K], float 
             const float keep = q ? y[2 * j + 1] : y[2 * j];
             const float send = q ? y[2 * j] : y[2 * j + 1];
             yo[j] = keep + __shfl_xor_sync(mask, send, STRIDE);
+        } else if (G > 4) {
+            // log2 G butterfly rounds on the group's G values of block j:
+            // in the round of distance o a lane keeps the half of its values
+            // selected by bit o of q and adds its partner's copy of that half
+            float v[G];
+#pragma unroll
+            for (int i = 0; i < G; ++i) v[i] = y[G * j + i];
+#pragma unroll
+            for (int o = G / 2, n = G; o >= 1; o >>= 1, n >>= 1) {
+                const bool hi = (q & o) != 0;
+#pragma unroll
+                for (int i = 0; i < n / 2; ++i) {
+                    const float keep = hi ? v[n / 2 + i] : v[i];
+                    const float send = hi ? v[i] : v[n / 2 + i];
+                    v[i] = keep + __shfl_xor_sync(mask, send, o * STRIDE);
+                }
+            }
+            yo[j] = v[0];
         } else {  // G == 4
             const bool hi = (q & 2) != 0;
             const float k0 = hi ? y[4 * j + 2] : y[4 * j + 0], k1 = hi ? y[4 * j + 3] : y[4 * j + 1];
