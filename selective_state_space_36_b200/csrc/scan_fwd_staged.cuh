@@ -17,7 +17,10 @@
 // out move CPL channels per access (one channel per lane is the default: at
 // the benchmark shapes halving the warps costs more than the traffic saved).
 // Tile rows are padded by 32 bytes so that the G rows the lanes of a group
-// read at once fall in different banks.
+// read at once fall in different banks.  With four lanes per channel the
+// lanes of a group sit 8 apart in the warp, so that the 8 lanes of a
+// quarter-warp read one B/C address (two L1 wavefronts per 128-bit load, not
+// four).
 //
 // The waits are cp.async.wait_group (hardware-tracked completion of this
 // thread's own copies) followed by a block barrier: there is no polling loop.
@@ -415,11 +418,12 @@ scan_fwd_staged_kernel(const ScanArgs args) {
 // Threads of a virtual block of the one-pass scan, by lanes per channel.
 // Measured on B200 (Gelem/s; 1.4B layer = 32,768 channels, 130M layer =
 // 12,288 channels): two lanes per channel in 64-thread virtual blocks, seven
-// per CTA, 164.6 at the 1.4B layer (one lane: 156.7 in one-warp virtual
-// blocks, 155.9 in 128-thread blocks); four lanes in 128-thread blocks, one
-// per CTA, 122.6 at the 130M layer (packed three per CTA: 113.6; 32- or
-// 64-thread virtual blocks: 104-108, each re-widening the B/C rows for fewer
-// channels).
+// per CTA, 164.6 at the 1.4B layer with 16-step blocks, 167.5-167.9 with
+// 8-step blocks (one lane: 156.7 in one-warp virtual blocks, 155.9 in
+// 128-thread blocks); four lanes in 128-thread blocks, one per CTA, 122.6 at
+// the 130M layer, 125-130 once a channel's lanes sat 8 apart (packed three per
+// CTA: 113.6; 32- or 64-thread virtual blocks: 104-108, each re-widening the
+// B/C rows for fewer channels).
 #ifndef SSM_VB_THREADS_G1
 #define SSM_VB_THREADS_G1 128
 #endif

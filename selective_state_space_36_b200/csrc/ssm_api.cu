@@ -89,8 +89,10 @@ void scan_layout(int64_t dstate, int64_t channels, int sms, int lanes_req, int *
             // (4 states each) give the warps that hide latency.  From there
             // up to what one CTA per SM holds in 64-thread virtual blocks of
             // two lanes per channel (8 per CTA: 256 channels per SM), two
-            // lanes: the 1.4B layer (32,768 channels) measured 164.6 Gelem/s
-            // against 156.7 with one lane.  Beyond that, one lane per channel
+            // lanes: the 1.4B layer (32,768 channels) measured 165.3 Gelem/s
+            // against 161.5 with one lane and 163.6 with four (the same box,
+            // 16-step blocks; two lanes 167.9 with their 8-step blocks).
+            // Beyond that, one lane per channel
             // (all 16 states, no shuffles) in 128-thread blocks.
             if (2 * channels < (int64_t)sms * ssm::kBlock * 3) G = 4;
             else if (channels <= (int64_t)sms * 256) G = 2;
