@@ -388,7 +388,9 @@ typedef struct {
     int32_t sfu_decays_per_16; /* of every 16 decays exp(Delta A) of the bf16 (fast) scan
                                   tier, how many the SFU computes; the rest are computed
                                   on the FMA pipe by a polynomial */
-    int32_t reserved[7];
+    int32_t split_pass1_sfu_decays_per_16; /* the same for the first pass of the
+                                  sequence split (segment aggregates) */
+    int32_t reserved[6];
 } ssm_build_info;
 
 void ssm_get_build_info(ssm_build_info *info);

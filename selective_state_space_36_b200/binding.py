@@ -55,7 +55,8 @@ class SSMSsdDims(ctypes.Structure):
 
 
 class SSMBuildInfo(ctypes.Structure):
-    _fields_ = [("sfu_decays_per_16", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+    _fields_ = [("sfu_decays_per_16", ctypes.c_int32), ("split_pass1_sfu_decays_per_16", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 class SSMError(RuntimeError):
@@ -343,7 +344,8 @@ def build_info() -> dict:
     """Build parameters of the loaded library (ssm_get_build_info)."""
     info = SSMBuildInfo()
     lib.ssm_get_build_info(ctypes.byref(info))
-    return {"sfu_decays_per_16": int(info.sfu_decays_per_16)}
+    return {"sfu_decays_per_16": int(info.sfu_decays_per_16),
+            "split_pass1_sfu_decays_per_16": int(info.split_pass1_sfu_decays_per_16)}
 
 
 def scan_plan(batch: int, seqlen: int, dim: int, dstate: int, io: str = "bf16",

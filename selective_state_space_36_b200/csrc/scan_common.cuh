@@ -192,7 +192,8 @@ __device__ __forceinline__ void recur_block(const float (&dl)[K], const float (&
 
 // The same for a lane that holds NS states of each of CPL channels: step k's
 // B and C values are read once and used for every channel.
-template <int K, int NS, int CPL, bool PRECISE, bool ZOH = false, bool READOUT = true>
+template <int K, int NS, int CPL, bool PRECISE, bool ZOH = false, bool READOUT = true,
+          int POLY = SSM_POLY_PAIRS>
 __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const float (&du)[K][CPL],
                                                 const float *Bs, const float *Cs, int stride,
                                                 const float2 (&A2)[CPL][NS / 2],
@@ -225,7 +226,7 @@ __device__ __forceinline__ void recur_block_cpl(const float (&dl)[K][CPL], const
                 for (int c = 0; c < CPL; ++c) {
                     if (!PRECISE) {
                         const float2 x2 = mul2(d2[c], A2[c][p]);
-                        const float2 a2 = poly_pair(p) ? exp2_poly2(x2)
+                        const float2 a2 = poly_pair<POLY>(p) ? exp2_poly2(x2)
                                                        : make_float2(decay_of<PRECISE>(x2.x), decay_of<PRECISE>(x2.y));
                         float2 bu = mul2(u2[c], b2);
                         if (ZOH)

@@ -164,6 +164,9 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     // the checkpoint pass stores a state every kCkptEvery steps: its step
     // blocks are that long
     constexpr int KSTEP = MODE == kCkpt ? kCkptEvery : KStep<G, CPL>::value;
+    // the checkpoint pass and the split's first pass produce states only:
+    // no C rows staged, no readout
+    constexpr bool kReadout = MODE != kCkpt && MODE != kSegAgg;
     constexpr int KG = KSTEP / G;         // steps whose scalar work this lane does
     static_assert(T % KSTEP == 0, "a chunk holds whole step blocks");
     // A CTA holds blockDim.x / TPB virtual blocks.  Virtual block vb of CTA
@@ -234,7 +237,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
         const int64_t gbc = (b * L + tc) * N;
         for (int p = tid; p < pieces; p += TPB) {
             cp_async16(rb + p * EPV, pB + gbc + p * EPV, true);
-            if (MODE != kCkpt) cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
+            if (kReadout) cp_async16(rc + p * EPV, pC + gbc + p * EPV, true);
         }
     };
 
@@ -281,7 +284,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 float v[4];
                 io::load4_smem(rb + i, v);
                 *reinterpret_cast<float4 *>(fB + i) = make_float4(v[0], v[1], v[2], v[3]);
-                if (MODE != kCkpt) {
+                if (kReadout) {
                     io::load4_smem(rc + i, v);
                     *reinterpret_cast<float4 *>(fC + i) = make_float4(v[0], v[1], v[2], v[3]);
                 }
@@ -291,7 +294,7 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 const int r = i / NSP, n = i % NSP;
                 const bool ok = r < rows && n < N;
                 fB[i] = ok ? io::load_smem(rb + r * N + n) : 0.f;
-                if (MODE != kCkpt) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
+                if (kReadout) fC[i] = ok ? io::load_smem(rc + r * N + n) : 0.f;
             }
         }
         vblock_sync<TPB, MODE>(vb);
@@ -363,7 +366,8 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                 }
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
                 exchange_steps_cpl<KSTEP, G, CPL, LS>(dlo, duo, dl, du);
-                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, MODE != kCkpt>(
+                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, kReadout,
+                                MODE == kSegAgg ? SSM_SEGAGG_POLY_PAIRS : SSM_POLY_PAIRS>(
                     dl, du, fBq + r0 * NSP, fCq + r0 * NSP, NSP, A2, h2, y, invA2);
                 if (MODE == kCkpt) {
                     // no readout

@@ -176,6 +176,7 @@ void ssm_get_build_info(ssm_build_info *info) {
     if (!info) return;
     memset(info, 0, sizeof(*info));
     info->sfu_decays_per_16 = 16 - 4 * SSM_POLY_PAIRS;
+    info->split_pass1_sfu_decays_per_16 = 16 - 4 * SSM_SEGAGG_POLY_PAIRS;
 }
 
 }  // extern "C"

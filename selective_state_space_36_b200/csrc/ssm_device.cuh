@@ -245,7 +245,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 #ifndef SSM_POLY_PAIRS
 #define SSM_POLY_PAIRS 0
 #endif
-__device__ __forceinline__ constexpr bool poly_pair(int p) { return (p & 3) < SSM_POLY_PAIRS; }
+// The same share for the first pass of the sequence split (segment
+// aggregates, no readout), which keeps the SFU ~91 % busy: bound by its
+// throughput rather than by latency.  A quarter by default: one call at
+// L = 1,048,576, dim 1536 measured 15.35 ms with a quarter of that pass's
+// decays on the polynomial, 15.53 ms with none and 18.55 ms with half.
+#ifndef SSM_SEGAGG_POLY_PAIRS
+#define SSM_SEGAGG_POLY_PAIRS 1
+#endif
+template <int POLY>
+__device__ __forceinline__ constexpr bool poly_pair(int p) { return (p & 3) < POLY; }
 
 template <bool PRECISE>
 __device__ __forceinline__ float scale_A(float a) {

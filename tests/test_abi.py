@@ -203,3 +203,5 @@ def test_ssd_argument_validation(b):
 def test_build_info(b):
     info = b.build_info()
     assert 0 <= info["sfu_decays_per_16"] <= 16 and info["sfu_decays_per_16"] % 4 == 0
+    p1 = info["split_pass1_sfu_decays_per_16"]
+    assert 0 <= p1 <= 16 and p1 % 4 == 0
