@@ -355,14 +355,17 @@ def _scan_device_inputs(cfg: I.ScanConfig, dev, sh=None):
 
 def _time_steps(step, steps, warmup, stream, dev, world, sample_clocks=True):
     """Warm-up, then K steps bracketed by barrier + synchronize, CUDA events on
-    the launching stream around the region and around each step; max over ranks."""
+    the launching stream around the region; max over ranks.  The steps run back
+    to back, as a caller issues them: no event is recorded between them (an
+    event pair around every step added 2-6 us per step and stopped a decode
+    step's launch from overlapping the end of the step before it), so a step's
+    average duration is the region's time over K."""
     import torch
     import torch.distributed as dist
     for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev.index or 0)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -370,18 +373,15 @@ def _time_steps(step, steps, warmup, stream, dev, world, sample_clocks=True):
         sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(steps):
-        ev[i][0].record(stream)
+    for _ in range(steps):
         step()
-        ev[i][1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    elapsed_ms, launch_ms = max_over_ranks([e0.elapsed_time(e1), launch_ms], dev)
-    return elapsed_ms, launch_ms, clocks
+    elapsed_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+    return elapsed_ms, elapsed_ms / steps, clocks
 
 
 def _e2e(step_with_copies, steps, stream, dev, world):

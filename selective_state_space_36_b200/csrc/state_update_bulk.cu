@@ -25,6 +25,10 @@
 //   * A CTA takes a contiguous run of units in chunk-major order (consecutive
 //     units cover the same channels of successive batch rows), so A and D stay
 //     in registers and are reloaded only when the channel chunk changes.
+//   * The kernel is launched as a programmatic dependent of the stream's
+//     previous kernel (griddepcontrol): one decode step's launch and set-up
+//     overlap the end of the step before it, and its global accesses wait
+//     for that step's writes.
 // The grid is persistent: up to three 256-thread CTAs per SM.  Every wait on
 // an mbarrier gives up after 200 ms (read from the global timer) and sets bit
 // 0 of a device status word; the warp that saw it (the answer is made
@@ -32,6 +36,7 @@
 // lets the loads it issued land (each wait again bounded); the host reads
 // the word with ssm_get_device_status.
 #include <atomic>
+#include <utility>
 
 #include "scan_kernels.cuh"
 
@@ -40,6 +45,37 @@ namespace ssm {
 __device__ unsigned int g_device_status;
 
 namespace {
+
+// Programmatic dependent launch (sm_90 and later): the kernel may be launched
+// before the stream's previous kernel has finished, so that its launch and
+// CTA set-up overlap that kernel's end.  grid_dependency_wait() returns once
+// the previous kernel has completed and its writes are visible, and then lets
+// the next dependent launch begin.
+#ifndef SSM_PDL
+#define SSM_PDL 1
+#endif
+__device__ __forceinline__ void grid_dependency_wait() {
+#if SSM_PDL
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+#endif
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = SSM_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 #ifndef SSM_DECODE_STAGES
 #define SSM_DECODE_STAGES 4
@@ -154,6 +190,13 @@ state_update_bulk_kernel(const DecodeArgs args, int64_t chunks, int64_t total_un
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
+    // Launched as a programmatic dependent of the stream's previous kernel:
+    // the set-up above may overlap that kernel's end, but nothing in global
+    // memory is read or written before it has completed and its writes are
+    // visible (the previous decode step's state, for one).  Once every CTA of
+    // this grid runs, the next step's launch may begin (its CTAs take the
+    // SMs as these exit and wait in turn).
+    grid_dependency_wait();
 
     auto geom = [&](int64_t k, int64_t &b, int64_t &c0, int &nch) {
         const int64_t u = u0 + k;
@@ -294,8 +337,7 @@ cudaError_t launch_g(const DecodeArgs &a, uint32_t missing_bytes, cudaStream_t s
     const int64_t chunks = (a.dim + SL::CH - 1) / SL::CH;
     const int64_t total = a.batch * chunks;
     const int64_t grid = total < (int64_t)sms * kCtasPerSm ? total : (int64_t)sms * kCtasPerSm;
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(a, chunks, total, missing_bytes);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(kThreads), smem, st, a, chunks, total, missing_bytes);
 }
 
 template <typename IO>
