@@ -164,3 +164,33 @@ def test_decode_bounded_wait_sets_device_status(lib):
     T.check_out(T.from_dev(out), ref, "bf16")
     T.check_state(T.from_dev(state), h, "bf16")
     assert lib.device_status() == 0
+
+
+def test_decode_sees_the_writes_of_the_kernel_before_it(lib):
+    # The decode step is launched as a programmatic dependent of the stream's
+    # previous kernel, so its launch overlaps that kernel's end.  Here each
+    # step's state and x are written by a device kernel right before the
+    # step (alternating between two different sources); a step that read
+    # either before that kernel finished would see the previous step's
+    # values and miss the oracle.
+    cfg = I.DecodeConfig("d", 64, 2048, 16, steps=8, io="bf16", seed=21)
+    A, D, bias = I.decode_params(cfg)
+    Ad, Dd = torch.from_numpy(A).cuda(), torch.from_numpy(D).cuda()
+    rng = np.random.default_rng(7)
+    srcs = [rng.standard_normal((cfg.batch, cfg.dim, cfg.dstate)).astype(np.float32) for _ in range(2)]
+    srcs_dev = [torch.from_numpy(s).cuda() for s in srcs]
+    state = torch.empty_like(srcs_dev[0])
+    x_dev = torch.empty((cfg.batch, cfg.dim), dtype=torch.bfloat16, device="cuda")
+    for k in range(cfg.steps):
+        st = I.decode_step_inputs(cfg, k, bias)
+        x_src = T.to_dev(st["x"], "bf16")
+        rest = {n: T.to_dev(st[n], "bf16") for n in ("dt", "B", "C", "z")}
+        torch.cuda.synchronize()
+        torch.mul(srcs_dev[k % 2], 1.0, out=state)  # kernels writing the step's inputs
+        torch.mul(x_src, 1, out=x_dev)
+        out = lib.selective_state_update(state, x_dev, rest["dt"], Ad, rest["B"], rest["C"], D=Dd, z=rest["z"])
+        ref, h = _oracle_step(srcs[k % 2].astype(np.float64), st, A.astype(np.float64), D.astype(np.float64),
+                              "bf16")
+        T.check_out(T.from_dev(out), ref, "bf16", what=f"step {k}")
+        T.check_state(T.from_dev(state), h, "bf16", what=f"step {k}")
+    assert lib.device_status() == 0
