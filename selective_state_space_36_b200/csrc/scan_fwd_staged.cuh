@@ -161,9 +161,10 @@ scan_fwd_staged_kernel(const ScanArgs args) {
     constexpr int T = Lay::T, S = Lay::S, CPB = Lay::CPB, NSP = Lay::NSP, ROW = Lay::ROW;
     constexpr int EPV = 16 / sizeof(IO);  // elements per 16-byte piece
     constexpr int ROWV = CPB / EPV;       // pieces per tile row
-    // the checkpoint pass stores a state every kCkptEvery steps: its step
-    // blocks are that long
-    constexpr int KSTEP = MODE == kCkpt ? kCkptEvery : KStep<G, CPL>::value;
+    // (the checkpoint pass stores a state every kCkptEvery steps: its step
+    // blocks are whole numbers of that spacing)
+    constexpr int KSTEP = KStep<G, CPL>::value;
+    static_assert(MODE != kCkpt || KSTEP % kCkptEvery == 0, "checkpoints fall on step-block pieces");
     // the checkpoint pass and the split's first pass produce states only:
     // no C rows staged, no readout
     constexpr bool kReadout = MODE != kCkpt && MODE != kSegAgg;
@@ -354,21 +355,36 @@ scan_fwd_staged_kernel(const ScanArgs args) {
                         duo[j][cc] = dlo[j][cc] * uvo[j][cc];
                     }
                 }
-                if (MODE == kCkpt) {
-                    // the state entering step tc + r0 (a multiple of the
-                    // checkpoint spacing: blocks are kCkptEvery steps long)
-                    float *cp = ck_base + ((tc + r0) / kCkptEvery) * ck_stride;
-#pragma unroll
-                    for (int p = 0; p < NS / 2; ++p) {
-                        if (q * NS + 2 * p < N) cp[2 * p] = h2[0][p].x;
-                        if (q * NS + 2 * p + 1 < N) cp[2 * p + 1] = h2[0][p].y;
-                    }
-                }
                 float dl[KSTEP][CPL], du[KSTEP][CPL], y[KSTEP][CPL];
                 exchange_steps_cpl<KSTEP, G, CPL, LS>(dlo, duo, dl, du);
-                recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, kReadout,
-                                MODE == kSegAgg ? SSM_SEGAGG_POLY_PAIRS : SSM_POLY_PAIRS>(
-                    dl, du, fBq + r0 * NSP, fCq + r0 * NSP, NSP, A2, h2, y, invA2);
+                if (MODE == kCkpt) {
+                    // the block in pieces of the checkpoint spacing, each
+                    // preceded by the store of the state entering it (step
+                    // tc + rs, a multiple of the spacing); pieces past the
+                    // end of the sequence store nothing
+                    constexpr int KC = kCkptEvery;
+#pragma unroll
+                    for (int hb = 0; hb < KSTEP / KC; ++hb) {
+                        const int rs = r0 + hb * KC;
+                        if (rs < nrows) {
+                            float *cp = ck_base + ((tc + rs) / KC) * ck_stride;
+#pragma unroll
+                            for (int p = 0; p < NS / 2; ++p) {
+                                if (q * NS + 2 * p < N) cp[2 * p] = h2[0][p].x;
+                                if (q * NS + 2 * p + 1 < N) cp[2 * p + 1] = h2[0][p].y;
+                            }
+                        }
+                        float yp[KC][CPL];
+                        recur_block_cpl<KC, NS, CPL, PRECISE, ZOH, false, SSM_POLY_PAIRS>(
+                            *reinterpret_cast<const float(*)[KC][CPL]>(&dl[hb * KC]),
+                            *reinterpret_cast<const float(*)[KC][CPL]>(&du[hb * KC]), fBq + rs * NSP,
+                            fCq + rs * NSP, NSP, A2, h2, yp, invA2);
+                    }
+                } else {
+                    recur_block_cpl<KSTEP, NS, CPL, PRECISE, ZOH, kReadout,
+                                    MODE == kSegAgg ? SSM_SEGAGG_POLY_PAIRS : SSM_POLY_PAIRS>(
+                        dl, du, fBq + r0 * NSP, fCq + r0 * NSP, NSP, A2, h2, y, invA2);
+                }
                 if (MODE == kCkpt) {
                     // no readout
                 } else if (MODE == kSegAgg) {
